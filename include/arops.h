@@ -1,0 +1,166 @@
+/*
+ * arops.h: per-token operators of autoregressive speech-model decode, as a C ABI.
+ *
+ * Four operators, each one hand-written CUDA kernel for NVIDIA B200 (sm_100a):
+ *
+ *   arops_rmsnorm      y = gamma * x / sqrt(mean(x^2) + eps)
+ *                      ("Optimising autoregressive speech models", §09
+ *                      "LayerNorm -> RMSNorm": the RMSNorm equation and module)
+ *   arops_add_rmsnorm  residual_out = x + residual_in (rounded to the dtype);
+ *                      y = RMSNorm(residual_out)
+ *                      ("Norm+Residual" in section 3 of the Triton kernel-fusion
+ *                      post for Qwen3-TTS, news.hada.io topic 27742)
+ *   arops_mrope_qk     multi-section rotary embedding of q and k
+ *                      ("M-RoPE" in the same section; rotation of q/k in the
+ *                      complex plane per forpes.ru post 233929, "Stage 2")
+ *   arops_swiglu       out = silu(gate) * up, silu(g) = g / (1 + e^-g)
+ *                      ("SwiGLU" in the same section)
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are caller-owned DEVICE memory, dense and row-major.
+ *     The library allocates and frees nothing and keeps no pointer after the
+ *     call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every call is asynchronous on that stream: it validates its
+ *     arguments on the host, enqueues one kernel and returns; it never
+ *     synchronises.  Faults inside a kernel surface at the caller's next
+ *     synchronisation, as with any CUDA library.
+ *   - The device is the caller's current CUDA device.
+ *   - A zero-sized problem (rows == 0, tokens == 0) is a no-op returning
+ *     AROPS_OK; its pointers are not inspected.
+ *   - Argument errors (null pointer, bad dtype, bad shape, eps < 0, ...) return
+ *     AROPS_ERR_INVALID (or AROPS_ERR_UNSUPPORTED for valid but unimplemented
+ *     sizes) before anything is launched.  A failed launch returns
+ *     AROPS_ERR_CUDA.  arops_last_error() then gives a one-line reason.
+ *   - Arithmetic is fp32 in registers whatever the storage dtype; each output
+ *     is rounded once, round-to-nearest-even, to the storage dtype.
+ *   - Pointers need not be aligned: 16-byte-aligned buffers whose row length is
+ *     a multiple of 16 bytes take the vectorised kernels, anything else takes an
+ *     element-wise kernel on the GPU with the same results.
+ *   - An output may be the same buffer as an input of the same shape (in-place);
+ *     partially overlapping buffers are undefined.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef AROPS_H
+#define AROPS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define AROPS_API __attribute__((visibility("default")))
+#else
+#define AROPS_API
+#endif
+
+typedef enum {
+    AROPS_OK = 0,
+    AROPS_ERR_INVALID = 1,     /* bad argument; nothing was launched */
+    AROPS_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim > 512) */
+    AROPS_ERR_CUDA = 3         /* the CUDA runtime reported an error at launch */
+} arops_status;
+
+typedef enum {
+    AROPS_F32 = 0,  /* IEEE binary32 storage */
+    AROPS_BF16 = 1  /* bfloat16 storage */
+} arops_dtype;
+
+/*
+ * RMSNorm over the last dimension ("Optimising autoregressive speech models",
+ * §09: gamma * x / sqrt(mean(x^2) + eps), eps inside the root, the mean over the
+ * row, a per-channel weight).
+ *   x     [rows, hidden]  dtype      input
+ *   gamma [hidden]        dtype      per-channel weight
+ *   y     [rows, hidden]  dtype      output (may be x)
+ *   eps >= 0 (1e-6 in the pages' module).  A zero row gives y = 0 for eps > 0;
+ *   eps == 0 on a zero row gives NaN, as the formula does.
+ * The sum of squares is accumulated in fp32.
+ */
+AROPS_API arops_status arops_rmsnorm(const void* x, const void* gamma, void* y,
+                                     int64_t rows, int64_t hidden, float eps,
+                                     arops_dtype dtype, void* stream);
+
+/*
+ * Fused residual add + RMSNorm ("Norm+Residual", Triton kernel-fusion post for
+ * Qwen3-TTS, section 3), in one pass over memory:
+ *   residual_out = round_dtype(x + residual_in)
+ *   y            = RMSNorm(residual_out) with weight gamma
+ * i.e. exactly "add, then normalise" on dtype tensors: the norm sees the
+ * rounded residual that is written back.
+ *   x, residual_in, residual_out, y: [rows, hidden] dtype; gamma: [hidden] dtype.
+ *   residual_out may be residual_in (the usual in-place update of the residual
+ *   stream); y may be x.
+ */
+AROPS_API arops_status arops_add_rmsnorm(const void* x, const void* residual_in,
+                                         void* residual_out, const void* gamma, void* y,
+                                         int64_t rows, int64_t hidden, float eps,
+                                         arops_dtype dtype, void* stream);
+
+/*
+ * Multi-section rotary embedding (M-RoPE) of q and k, rotate-half pairing.
+ * ("M-RoPE" in the Triton kernel-fusion post, section 3; RoPE as a rotation of
+ * Q and K in the complex plane, forpes.ru post 233929, "Stage 2".)
+ *
+ * For every token t, head h and pair index j in [0, head_dim/2):
+ *   row  = 0 if j < sections[0], 1 if j < sections[0] + sections[1], else 2
+ *   p    = pos[row * tokens + t]                      (rows t, h, w of the ids)
+ *   phi  = p * theta^(-2 j / head_dim)
+ *   (a, b) = (x[j], x[j + head_dim/2])
+ *   out[j] = a cos(phi) - b sin(phi),  out[j + head_dim/2] = b cos(phi) + a sin(phi)
+ *
+ *   q, q_out [tokens, n_q_heads, head_dim] dtype (q_out may be q)
+ *   k, k_out [tokens, n_k_heads, head_dim] dtype (k_out may be k)
+ *   pos      [3, tokens] int32 device array (rows t, h, w)
+ *   sections HOST array of 3 non-negative int32 summing to head_dim / 2
+ *   head_dim even, 2 <= head_dim <= 512; theta > 0 and finite.
+ *   n_k_heads may be 0 (k, k_out ignored); likewise n_q_heads.
+ * The angle is formed and reduced modulo 2*pi in fp64, then cos/sin are taken
+ * in fp32, per (token, j), in registers: no cos/sin table is read.
+ */
+AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out, void* k_out,
+                                      const int32_t* pos, int64_t tokens,
+                                      int32_t n_q_heads, int32_t n_k_heads, int32_t head_dim,
+                                      const int32_t* sections, float theta,
+                                      arops_dtype dtype, void* stream);
+
+/*
+ * SwiGLU activation ("SwiGLU" in the Triton kernel-fusion post, section 3):
+ *   out = silu(gate) * up,  silu(g) = g / (1 + e^-g), computed in fp32.
+ *   gate, up, out: [rows, inter] dtype, separate tensors (out may be gate or up).
+ */
+AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
+                                    int64_t rows, int64_t inter,
+                                    arops_dtype dtype, void* stream);
+
+/*
+ * Programmatic dependent launch.  When enabled (process-wide, default off),
+ * every kernel is launched with the programmatic-stream-serialisation attribute
+ * so that it can be scheduled while the previous kernel on the stream drains;
+ * each kernel waits for its predecessor's memory before touching global memory,
+ * so results and stream-order semantics are unchanged.  It only shortens the
+ * gaps between back-to-back launches (decode steps).  Returns the old setting.
+ */
+AROPS_API int arops_set_pdl(int enable);
+
+/* Number of kernels this library has launched in this process (all devices). */
+AROPS_API uint64_t arops_launch_count(void);
+
+/* Static string for a status code; never NULL. */
+AROPS_API const char* arops_status_string(arops_status status);
+
+/* Reason for the last non-OK status returned on the calling thread ("" if none). */
+AROPS_API const char* arops_last_error(void);
+
+/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+AROPS_API int arops_version(void);
+
+#define AROPS_VERSION 10000
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AROPS_H */

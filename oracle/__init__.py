@@ -174,7 +174,8 @@ class Oracle:
 
     # -- decode-step chain ---------------------------------------------------
     def decode_step(self, residual, layer_inputs: dict, step: int, eps: float = 1e-6,
-                    theta: float = 1e6, sections=(24, 20, 20), dtype: str = "bf16"):
+                    theta: float = 1e6, sections=(24, 20, 20), dtype: str = "bf16",
+                    outputs: bool = True):
         """One decode step over every layer, in the order add+RMSNorm, M-RoPE on
         q/k at position ``step`` in all three rows, add+RMSNorm, SwiGLU.
 
@@ -182,7 +183,8 @@ class Oracle:
         keys x_attn, gamma_attn, q, k, x_mlp, gamma_mlp, gate, up.  Every output
         is rounded to ``dtype`` at the operator boundary, as the GPU writes it.
         Returns (residual after the step, dict of per-layer outputs y_attn, q, k,
-        y_mlp, act)."""
+        y_mlp, act).  With ``outputs=False`` only the residual stream is
+        computed and the dict is empty."""
         res = _f64(residual)
         batch = res.shape[0]
         pos = np.full((3, batch), step, dtype=np.int32)
@@ -190,6 +192,10 @@ class Oracle:
         for layer in range(len(layer_inputs["x_attn"])):
             y, res = self.add_rmsnorm(layer_inputs["x_attn"][layer], res,
                                       layer_inputs["gamma_attn"][layer], eps, dtype)
+            if not outputs:
+                _, res = self.add_rmsnorm(layer_inputs["x_mlp"][layer], res,
+                                          layer_inputs["gamma_mlp"][layer], eps, dtype)
+                continue
             outs["y_attn"].append(self.round_to(y, dtype))
             qo, ko = self.mrope_qk(layer_inputs["q"][layer], layer_inputs["k"][layer], pos,
                                    sections, theta)
@@ -200,6 +206,8 @@ class Oracle:
             outs["y_mlp"].append(self.round_to(y, dtype))
             act = self.swiglu(layer_inputs["gate"][layer], layer_inputs["up"][layer])
             outs["act"].append(self.round_to(act, dtype))
+        if not outputs:
+            outs = {}
         return res, outs
 
 

@@ -1,0 +1,206 @@
+"""Python binding of libarops.so: per-token decode operators for B200 (sm_100a).
+
+Thin ctypes wrappers with the names of the C entry points in ``include/arops.h``
+(``arops_rmsnorm`` -> ``rmsnorm`` and so on).  They check that the tensors are
+CUDA, contiguous and of one dtype, then pass ``data_ptr()`` values, sizes and
+torch's current CUDA stream to the library.  Every step of every operator runs
+in the library's CUDA kernels; there is no fallback of any kind.  If the shared
+library has not been built, every call raises.
+
+Build the library with ``python -m swiglu_ar_tts_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "rmsnorm", "add_rmsnorm", "mrope_qk", "swiglu", "set_pdl", "launch_count",
+    "lib", "lib_path", "ArOpsError", "DTYPES",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libarops.so")
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+
+
+class ArOpsError(RuntimeError):
+    """A non-OK status from libarops; ``status`` holds the code."""
+
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libarops.so (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m swiglu_ar_tts_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        L.arops_rmsnorm.argtypes = [_vp, _vp, _vp, _i64, _i64, ctypes.c_float, ctypes.c_int, _vp]
+        L.arops_add_rmsnorm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_float,
+                                        ctypes.c_int, _vp]
+        L.arops_mrope_qk.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32,
+                                     ctypes.POINTER(_i32), ctypes.c_float, ctypes.c_int, _vp]
+        L.arops_swiglu.argtypes = [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
+        for fn in ("arops_rmsnorm", "arops_add_rmsnorm", "arops_mrope_qk", "arops_swiglu"):
+            getattr(L, fn).restype = ctypes.c_int
+        L.arops_set_pdl.argtypes = [ctypes.c_int]
+        L.arops_set_pdl.restype = ctypes.c_int
+        L.arops_launch_count.restype = ctypes.c_uint64
+        L.arops_status_string.argtypes = [ctypes.c_int]
+        L.arops_status_string.restype = ctypes.c_char_p
+        L.arops_last_error.restype = ctypes.c_char_p
+        L.arops_version.restype = ctypes.c_int
+        _lib = L
+        return L
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        L = lib()
+        raise ArOpsError(status, f"{L.arops_status_string(status).decode()}: "
+                                 f"{L.arops_last_error().decode()}")
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dtype_code(*ts: torch.Tensor) -> int:
+    dt = ts[0].dtype
+    if dt not in DTYPES:
+        raise TypeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
+    for t in ts:
+        if t.dtype != dt:
+            raise TypeError(f"dtype mismatch: {t.dtype} vs {dt}")
+    return DTYPES[dt]
+
+
+def _cuda_contig(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+            out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = gamma * x / sqrt(mean(x^2, -1) + eps); ``out`` may be ``x``."""
+    hidden = x.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    for n, t in (("x", x), ("gamma", gamma), ("out", out)):
+        _cuda_contig(n, t)
+    if gamma.shape != (hidden,) or out.shape != x.shape:
+        raise ValueError("shape mismatch")
+    code = _dtype_code(x, gamma, out)
+    rows = x.numel() // hidden if hidden else 0
+    with torch.cuda.device(x.device):
+        _check(lib().arops_rmsnorm(x.data_ptr(), gamma.data_ptr(), out.data_ptr(), rows, hidden,
+                                   float(eps), code, _stream(x)))
+    return out
+
+
+def add_rmsnorm(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                y: torch.Tensor | None = None, residual_out: torch.Tensor | None = None):
+    """residual_out = x + residual (rounded to the dtype); y = RMSNorm(residual_out).
+
+    ``residual_out`` defaults to ``residual`` (updated in place); ``y`` defaults to
+    a new tensor.  Returns ``(y, residual_out)``."""
+    hidden = x.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    if residual_out is None:
+        residual_out = residual
+    for n, t in (("x", x), ("residual", residual), ("gamma", gamma), ("y", y),
+                 ("residual_out", residual_out)):
+        _cuda_contig(n, t)
+    if (residual.shape != x.shape or y.shape != x.shape or residual_out.shape != x.shape
+            or gamma.shape != (hidden,)):
+        raise ValueError("shape mismatch")
+    code = _dtype_code(x, residual, gamma, y, residual_out)
+    rows = x.numel() // hidden if hidden else 0
+    with torch.cuda.device(x.device):
+        _check(lib().arops_add_rmsnorm(x.data_ptr(), residual.data_ptr(), residual_out.data_ptr(),
+                                       gamma.data_ptr(), y.data_ptr(), rows, hidden, float(eps),
+                                       code, _stream(x)))
+    return y, residual_out
+
+
+def mrope_qk(q: torch.Tensor, k: torch.Tensor, pos: torch.Tensor, sections=(24, 20, 20),
+             theta: float = 1e6, q_out: torch.Tensor | None = None,
+             k_out: torch.Tensor | None = None):
+    """Multi-section rotary embedding of q [T, Hq, D] and k [T, Hk, D] with int32
+    position ids pos [3, T] (rows t, h, w).  Outputs default to the inputs
+    (rotation in place).  Returns ``(q_out, k_out)``."""
+    if q_out is None:
+        q_out = q
+    if k_out is None:
+        k_out = k
+    for n, t in (("q", q), ("k", k), ("pos", pos), ("q_out", q_out), ("k_out", k_out)):
+        _cuda_contig(n, t)
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q and k must be [tokens, heads, head_dim]")
+    tokens, hq, d = q.shape
+    if k.shape[0] != tokens or k.shape[2] != d or q_out.shape != q.shape or k_out.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if pos.dtype != torch.int32 or tuple(pos.shape) != (3, tokens):
+        raise ValueError("pos must be int32 [3, tokens]")
+    code = _dtype_code(q, k, q_out, k_out)
+    sec = (_i32 * 3)(*[int(s) for s in sections])
+    with torch.cuda.device(q.device):
+        _check(lib().arops_mrope_qk(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(),
+                                    pos.data_ptr(), tokens, hq, k.shape[1], d, sec, float(theta),
+                                    code, _stream(q)))
+    return q_out, k_out
+
+
+def swiglu(gate: torch.Tensor, up: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """out = silu(gate) * up (fp32 math); ``out`` may be ``gate`` or ``up``."""
+    if out is None:
+        out = torch.empty_like(gate)
+    for n, t in (("gate", gate), ("up", up), ("out", out)):
+        _cuda_contig(n, t)
+    if up.shape != gate.shape or out.shape != gate.shape:
+        raise ValueError("shape mismatch")
+    code = _dtype_code(gate, up, out)
+    inter = gate.shape[-1] if gate.dim() else 1
+    rows = gate.numel() // inter if inter else 0
+    with torch.cuda.device(gate.device):
+        _check(lib().arops_swiglu(gate.data_ptr(), up.data_ptr(), out.data_ptr(), rows, inter,
+                                  code, _stream(gate)))
+    return out
+
+
+def set_pdl(enable: bool) -> bool:
+    """Turn programmatic dependent launch on or off; returns the old setting."""
+    return bool(lib().arops_set_pdl(1 if enable else 0))
+
+
+def launch_count() -> int:
+    """Kernels launched by libarops in this process so far."""
+    return int(lib().arops_launch_count())

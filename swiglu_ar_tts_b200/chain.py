@@ -1,0 +1,142 @@
+"""Decode-step chain over the library's operators.
+
+One decode step of an autoregressive speech decoder (one new token for each of
+``batch`` candidates, e.g. the 5 candidates generated together in the Triton
+kernel-fusion post for Qwen3-TTS, section 1) runs, for each layer:
+
+    add + RMSNorm  (attention input)      residual <- residual + x_attn
+    M-RoPE on q, k at the step's position (all three rows t/h/w = step)
+    add + RMSNorm  (MLP input)            residual <- residual + x_mlp
+    SwiGLU         (MLP activation)
+
+The projections, attention and MLP GEMMs between these operators are not part
+of this library; their outputs are stood in for by fixed per-layer buffers, so
+a step is exactly the 4 * layers operator launches.  The residual stream is the
+only state carried from layer to layer and from step to step.
+
+``DecodeChain`` owns the device buffers and launches each operator through the
+C ABI with pre-bound arguments (no per-call tensor checks), either eagerly on
+the current stream or replayed from a CUDA graph of one step.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import DTYPES, ArOpsError, lib
+from .inputs import EPS, SECTIONS, THETA, ChainShape, decode_chain_inputs
+
+
+class DecodeChain:
+    def __init__(self, shape: ChainShape, dtype: str = "bf16", seed: int = 0,
+                 device: str | torch.device = "cuda", eps: float = EPS, theta: float = THETA,
+                 sections=SECTIONS, host_inputs: dict | None = None):
+        self.shape = shape
+        self.dtype = dtype
+        self.eps = eps
+        self.theta = theta
+        self.sections = tuple(int(s) for s in sections)
+        self.device = torch.device(device)
+        host = host_inputs if host_inputs is not None else decode_chain_inputs(shape, dtype, seed)
+        self.host_inputs = host
+        d = self.device
+        self.residual0 = host["residual"].to(d)
+        self.residual = self.residual0.clone()
+        self.inp = {k: [t.to(d).contiguous() for t in v] for k, v in host.items() if k != "residual"}
+        L, B = shape.layers, shape.batch
+        self.y_attn = [torch.empty_like(t) for t in self.inp["x_attn"]]
+        self.y_mlp = [torch.empty_like(t) for t in self.inp["x_mlp"]]
+        self.q_out = [torch.empty_like(t) for t in self.inp["q"]]
+        self.k_out = [torch.empty_like(t) for t in self.inp["k"]]
+        self.act = [torch.empty_like(t) for t in self.inp["gate"]]
+        self.pos = torch.zeros(3, B, dtype=torch.int32, device=d)  # the step's position ids
+        self._graph: torch.cuda.CUDAGraph | None = None
+        self._graph_stream: int | None = None
+        self._bind()
+
+    # -- pre-bound C calls ----------------------------------------------------
+    def _bind(self) -> None:
+        L = lib()
+        sh = self.shape
+        code = DTYPES[self.residual.dtype]
+        eps = ctypes.c_float(self.eps)
+        theta = ctypes.c_float(self.theta)
+        self._sec = (ctypes.c_int32 * 3)(*self.sections)
+        res = self.residual.data_ptr()
+        B, H, I = sh.batch, sh.hidden, sh.inter
+        calls = []
+        for l in range(sh.layers):
+            calls.append((L.arops_add_rmsnorm, [self.inp["x_attn"][l].data_ptr(), res, res,
+                                                self.inp["gamma_attn"][l].data_ptr(),
+                                                self.y_attn[l].data_ptr(), B, H, eps, code]))
+            calls.append((L.arops_mrope_qk, [self.inp["q"][l].data_ptr(), self.inp["k"][l].data_ptr(),
+                                             self.q_out[l].data_ptr(), self.k_out[l].data_ptr(),
+                                             self.pos.data_ptr(), B, sh.n_q_heads, sh.n_k_heads,
+                                             sh.head_dim, self._sec, theta, code]))
+            calls.append((L.arops_add_rmsnorm, [self.inp["x_mlp"][l].data_ptr(), res, res,
+                                                self.inp["gamma_mlp"][l].data_ptr(),
+                                                self.y_mlp[l].data_ptr(), B, H, eps, code]))
+            calls.append((L.arops_swiglu, [self.inp["gate"][l].data_ptr(), self.inp["up"][l].data_ptr(),
+                                           self.act[l].data_ptr(), B, I, code]))
+        self._calls = calls
+
+    @property
+    def launches_per_step(self) -> int:
+        return len(self._calls)
+
+    def bytes_per_step(self) -> int:
+        """Algorithmic HBM bytes of one step: every operand read once, every
+        output written once (positions 12 B per row, norm weights once per norm)."""
+        sh = self.shape
+        e = self.residual.element_size()
+        B, H, I = sh.batch, sh.hidden, sh.inter
+        per_layer = (2 * (4 * B * H + H) * e  # two add+norms: x, res in; res', y out; gamma
+                     + 2 * B * (sh.n_q_heads + sh.n_k_heads) * sh.head_dim * e + 3 * B * 4
+                     + 3 * B * I * e)
+        return sh.layers * per_layer
+
+    # -- execution ---------------------------------------------------------------
+    def reset(self) -> None:
+        self.residual.copy_(self.residual0)
+
+    def set_position(self, step: int) -> None:
+        """Position ids of decode step ``step`` (all rows equal to the step)."""
+        self.pos.fill_(step)
+
+    def launch_step(self, stream: int | None = None) -> None:
+        """Enqueue the 4 * layers operator launches of one step (positions as set)."""
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        for fn, args in self._calls:
+            st = fn(*args, stream)
+            if st != 0:
+                L = lib()
+                raise ArOpsError(st, f"{L.arops_status_string(st).decode()}: "
+                                     f"{L.arops_last_error().decode()}")
+
+    def step(self, step: int) -> None:
+        self.set_position(step)
+        self.launch_step()
+
+    def capture(self) -> torch.cuda.CUDAGraph:
+        """Capture one step (positions read from ``self.pos``) as a CUDA graph."""
+        with torch.cuda.device(self.device):
+            saved = self.residual.clone()
+            s = torch.cuda.Stream(self.device)
+            s.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(s):  # warm-up outside capture
+                self.launch_step()
+            torch.cuda.current_stream(self.device).wait_stream(s)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.launch_step()
+            self.residual.copy_(saved)
+        self._graph = g
+        return g
+
+    def replay(self, step: int) -> None:
+        if self._graph is None:
+            self.capture()
+        self.set_position(step)
+        self._graph.replay()

@@ -1,0 +1,221 @@
+// extern "C" entry points of include/arops.h: argument validation, dispatch to
+// the kernel launchers, status codes and the thread-local error string.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace arops {
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+std::atomic<int> g_pdl{0};
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];  // 0 = not queried yet
+
+arops_status fail(arops_status st, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+arops_status ok()
+{
+    g_last_error[0] = '\0';
+    return AROPS_OK;
+}
+
+arops_status from_cuda(cudaError_t err, const char* op)
+{
+    if (err == cudaSuccess)
+        return ok();
+    return fail(AROPS_ERR_CUDA, "%s: CUDA error %d (%s): %s", op, (int)err, cudaGetErrorName(err),
+                cudaGetErrorString(err));
+}
+
+bool valid_dtype(arops_dtype d)
+{
+    return d == AROPS_F32 || d == AROPS_BF16;
+}
+
+}  // namespace
+
+cudaError_t current_device_info(DeviceInfo* info)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    int sms = (dev >= 0 && dev < kMaxDevices) ? g_sm_count[dev].load(std::memory_order_relaxed) : 0;
+    if (sms == 0) {
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess)
+            return err;
+        if (dev >= 0 && dev < kMaxDevices)
+            g_sm_count[dev].store(sms, std::memory_order_relaxed);
+    }
+    info->sm_count = sms;
+    return cudaSuccess;
+}
+
+bool pdl_enabled()
+{
+    return g_pdl.load(std::memory_order_relaxed) != 0;
+}
+
+void count_launch()
+{
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+}  // namespace arops
+
+using namespace arops;
+
+extern "C" {
+
+AROPS_API arops_status arops_rmsnorm(const void* x, const void* gamma, void* y, int64_t rows,
+                                     int64_t hidden, float eps, arops_dtype dtype, void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: unknown dtype %d", (int)dtype);
+    if (rows < 0 || hidden <= 0 || hidden > INT32_MAX)
+        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: bad shape rows=%lld hidden=%lld",
+                    (long long)rows, (long long)hidden);
+    if (!(eps >= 0.0f) || isinf(eps))
+        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: eps must be finite and >= 0");
+    if (rows == 0)
+        return ok();
+    if (!x || !gamma || !y)
+        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: null pointer");
+    return from_cuda(launch_norm(x, nullptr, nullptr, gamma, y, rows, hidden, eps, dtype,
+                                 static_cast<cudaStream_t>(stream)),
+                     "arops_rmsnorm");
+}
+
+AROPS_API arops_status arops_add_rmsnorm(const void* x, const void* residual_in,
+                                         void* residual_out, const void* gamma, void* y,
+                                         int64_t rows, int64_t hidden, float eps,
+                                         arops_dtype dtype, void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: unknown dtype %d", (int)dtype);
+    if (rows < 0 || hidden <= 0 || hidden > INT32_MAX)
+        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: bad shape rows=%lld hidden=%lld",
+                    (long long)rows, (long long)hidden);
+    if (!(eps >= 0.0f) || isinf(eps))
+        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: eps must be finite and >= 0");
+    if (rows == 0)
+        return ok();
+    if (!x || !residual_in || !residual_out || !gamma || !y)
+        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: null pointer");
+    if (y == residual_out)
+        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: y and residual_out are one buffer");
+    return from_cuda(launch_norm(x, residual_in, residual_out, gamma, y, rows, hidden, eps, dtype,
+                                 static_cast<cudaStream_t>(stream)),
+                     "arops_add_rmsnorm");
+}
+
+AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out, void* k_out,
+                                      const int32_t* pos, int64_t tokens, int32_t n_q_heads,
+                                      int32_t n_k_heads, int32_t head_dim,
+                                      const int32_t* sections, float theta, arops_dtype dtype,
+                                      void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: unknown dtype %d", (int)dtype);
+    if (tokens < 0 || n_q_heads < 0 || n_k_heads < 0)
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: negative size");
+    if (head_dim <= 0 || head_dim % 2 != 0)
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: head_dim must be even and > 0 (got %d)",
+                    (int)head_dim);
+    if (head_dim > 512)
+        return fail(AROPS_ERR_UNSUPPORTED, "arops_mrope_qk: head_dim %d > 512", (int)head_dim);
+    if (!sections)
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: sections is null");
+    if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
+        (int64_t)sections[0] + sections[1] + sections[2] != head_dim / 2)
+        return fail(AROPS_ERR_INVALID,
+                    "arops_mrope_qk: sections [%d,%d,%d] must be >= 0 and sum to head_dim/2 = %d",
+                    (int)sections[0], (int)sections[1], (int)sections[2], (int)head_dim / 2);
+    if (!(theta > 0.0f) || isinf(theta))
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: theta must be finite and > 0");
+    if (tokens == 0 || n_q_heads + n_k_heads == 0)
+        return ok();
+    if (!pos || (n_q_heads > 0 && (!q || !q_out)) || (n_k_heads > 0 && (!k || !k_out)))
+        return fail(AROPS_ERR_INVALID, "arops_mrope_qk: null pointer");
+    MropeArgs a;
+    a.q = q;
+    a.k = k;
+    a.q_out = q_out;
+    a.k_out = k_out;
+    a.pos = pos;
+    a.tokens = tokens;
+    a.n_q_heads = n_q_heads;
+    a.n_k_heads = n_k_heads;
+    a.head_dim = head_dim;
+    a.sections[0] = sections[0];
+    a.sections[1] = sections[1];
+    a.sections[2] = sections[2];
+    a.theta = theta;
+    return from_cuda(launch_mrope(a, dtype, static_cast<cudaStream_t>(stream)), "arops_mrope_qk");
+}
+
+AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out, int64_t rows,
+                                    int64_t inter, arops_dtype dtype, void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_swiglu: unknown dtype %d", (int)dtype);
+    if (rows < 0 || inter <= 0 || (rows > 0 && inter > INT64_MAX / rows))
+        return fail(AROPS_ERR_INVALID, "arops_swiglu: bad shape rows=%lld inter=%lld",
+                    (long long)rows, (long long)inter);
+    if (rows == 0)
+        return ok();
+    if (!gate || !up || !out)
+        return fail(AROPS_ERR_INVALID, "arops_swiglu: null pointer");
+    return from_cuda(launch_swiglu(gate, up, out, rows * inter, dtype,
+                                   static_cast<cudaStream_t>(stream)),
+                     "arops_swiglu");
+}
+
+AROPS_API int arops_set_pdl(int enable)
+{
+    return g_pdl.exchange(enable ? 1 : 0);
+}
+
+AROPS_API uint64_t arops_launch_count(void)
+{
+    return g_launches.load(std::memory_order_relaxed);
+}
+
+AROPS_API const char* arops_status_string(arops_status status)
+{
+    switch (status) {
+    case AROPS_OK: return "ok";
+    case AROPS_ERR_INVALID: return "invalid argument";
+    case AROPS_ERR_UNSUPPORTED: return "unsupported size";
+    case AROPS_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+AROPS_API const char* arops_last_error(void)
+{
+    return g_last_error;
+}
+
+AROPS_API int arops_version(void)
+{
+    return AROPS_VERSION;
+}
+
+}  // extern "C"

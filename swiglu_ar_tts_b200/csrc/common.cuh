@@ -1,0 +1,181 @@
+// Shared device helpers for the decode-operator kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <string>
+
+#include "arops.h"
+
+namespace arops {
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (PDL).  griddepcontrol.wait blocks until the
+// preceding grid on the stream has completed and its memory is visible; it is
+// a no-op when the kernel was launched without the PDL attribute.
+// griddepcontrol.launch_dependents lets the next PDL kernel be scheduled early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_allow_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// 16-byte vectors of the storage type, unpacked to / packed from fp32.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Vec;
+
+template <>
+struct Vec<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f)
+    {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float* f)
+    {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+
+// bf16 is the top half of an fp32 word, so widening is a shift; narrowing is
+// the hardware round-to-nearest-even conversion of two floats at once.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <>
+struct Vec<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f)
+    {
+        f[0] = __uint_as_float(v.x << 16);
+        f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+        f[2] = __uint_as_float(v.y << 16);
+        f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+        f[4] = __uint_as_float(v.z << 16);
+        f[5] = __uint_as_float(v.z & 0xFFFF0000u);
+        f[6] = __uint_as_float(v.w << 16);
+        f[7] = __uint_as_float(v.w & 0xFFFF0000u);
+    }
+    __device__ __forceinline__ static uint4 pack(const float* f)
+    {
+        return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+    }
+};
+
+// Scalar element access for the unaligned / ragged kernels.
+__device__ __forceinline__ float load_elem(const float* p) { return *p; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ float round_to(float v, const float*) { return v; }
+__device__ __forceinline__ float round_to(float v, const __nv_bfloat16*)
+{
+    return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// Streaming 16-byte loads/stores: data is touched once, so ask the caches to
+// evict it first.  These are coherent loads (not the read-only path) because
+// outputs may alias inputs.
+__device__ __forceinline__ uint4 ld_stream(const void* p)
+{
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void st_stream(void* p, const uint4& v)
+{
+    __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int sm_count;
+};
+
+// SM count of the current device (queried once per device).
+cudaError_t current_device_info(DeviceInfo* info);
+
+// Whether kernels are launched with the PDL attribute.
+bool pdl_enabled();
+
+// Counts one launch.
+void count_launch();
+
+// Launches `kernel` on `stream`, with the PDL attribute when enabled.
+template <typename... Params, typename... Args>
+cudaError_t launch(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (pdl_enabled()) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+    if (err == cudaSuccess)
+        count_launch();
+    return err;
+}
+
+inline bool aligned16(const void* p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b)
+{
+    return (a + b - 1) / b;
+}
+
+// Launchers (one per operator), called after argument validation.
+cudaError_t launch_norm(const void* x, const void* residual_in, void* residual_out,
+                        const void* gamma, void* y, int64_t rows, int64_t hidden, float eps,
+                        arops_dtype dtype, cudaStream_t stream);
+
+cudaError_t launch_swiglu(const void* gate, const void* up, void* out, int64_t n,
+                          arops_dtype dtype, cudaStream_t stream);
+
+struct MropeArgs {
+    const void* q;
+    const void* k;
+    void* q_out;
+    void* k_out;
+    const int32_t* pos;
+    int64_t tokens;
+    int32_t n_q_heads;
+    int32_t n_k_heads;
+    int32_t head_dim;
+    int32_t sections[3];
+    float theta;
+};
+
+cudaError_t launch_mrope(const MropeArgs& a, arops_dtype dtype, cudaStream_t stream);
+
+}  // namespace arops

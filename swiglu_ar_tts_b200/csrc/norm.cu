@@ -1,0 +1,301 @@
+// RMSNorm and fused residual-add + RMSNorm (sm_100a).
+//
+// RMSNorm: y = gamma * x / sqrt(mean(x^2) + eps) over each row
+// ("Optimising autoregressive speech models", §09, the RMSNorm equation and
+// module).  Norm+Residual (Triton kernel-fusion post for Qwen3-TTS, section 3):
+// residual_out = round(x + residual_in), y = RMSNorm(residual_out), in one pass.
+//
+// Design: the row lives in registers.  A row of `hidden` elements is split into
+// 16-byte vectors; a group of 32*GW threads owns the row and every thread holds
+// VPL vectors, so global memory is read once and written once (x, residual ->
+// residual_out, y) with fully coalesced 128-bit accesses.  The sum of squares is
+// accumulated in fp32, reduced with warp shuffles and, for GW > 1 warps per row,
+// one shared-memory step.  rsqrtf of (sum / hidden + eps) scales the row; the
+// product x * r * gamma is rounded once to the storage type.  gamma is re-read
+// per row through the read-only path, where it stays L1/L2 resident.
+//
+// Rows longer than 4096 vectors, and unaligned or ragged rows, take a looped
+// kernel that makes a second pass over the row (served from L2).
+#include "common.cuh"
+
+namespace arops {
+namespace {
+
+constexpr int kRowsPerSmallCta = 2;  // GW == 1: two warps, one row each
+
+template <typename T, bool ADD, int VPL, int GW>
+__global__ void __launch_bounds__(GW == 1 ? 32 * kRowsPerSmallCta : 32 * GW)
+norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
+                 const T* __restrict__ gamma, T* y, int64_t rows, int hidden, float eps)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr int G = 32 * GW;  // threads per row
+    constexpr int ROWS_PER_CTA = (GW == 1) ? kRowsPerSmallCta : 1;
+    const int nvec = hidden / E;
+    const int tid = threadIdx.x;
+    const int gt = (GW == 1) ? (tid & 31) : tid;
+    const int group = (GW == 1) ? (tid >> 5) : 0;
+    __shared__ float red[2][GW];
+
+    pdl_wait();
+    pdl_allow_dependents();
+
+    int parity = 0;
+    for (int64_t row = (int64_t)blockIdx.x * ROWS_PER_CTA + group; row < rows;
+         row += (int64_t)gridDim.x * ROWS_PER_CTA) {
+        const size_t base = (size_t)row * (size_t)hidden;
+        uint4 v[VPL];
+        float ss = 0.f;
+        if constexpr (ADD) {
+            uint4 r[VPL];
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int vi = gt + i * G;
+                if (vi < nvec) {
+                    v[i] = ld_stream(x + base + (size_t)vi * E);
+                    r[i] = ld_stream(residual_in + base + (size_t)vi * E);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int vi = gt + i * G;
+                if (vi < nvec) {
+                    float a[E], b[E];
+                    Vec<T>::unpack(v[i], a);
+                    Vec<T>::unpack(r[i], b);
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        a[e] = a[e] + b[e];
+                    v[i] = Vec<T>::pack(a);  // the residual, rounded to T
+                    st_stream(residual_out + base + (size_t)vi * E, v[i]);
+                    Vec<T>::unpack(v[i], a);  // normalise what was written
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        ss = fmaf(a[e], a[e], ss);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int vi = gt + i * G;
+                if (vi < nvec)
+                    v[i] = ld_stream(x + base + (size_t)vi * E);
+            }
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int vi = gt + i * G;
+                if (vi < nvec) {
+                    float a[E];
+                    Vec<T>::unpack(v[i], a);
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        ss = fmaf(a[e], a[e], ss);
+                }
+            }
+        }
+
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if constexpr (GW > 1) {
+            // parity double-buffering: the next row writes the other buffer, so
+            // one barrier per row is enough
+            if ((tid & 31) == 0)
+                red[parity][tid >> 5] = ss;
+            __syncthreads();
+            ss = 0.f;
+#pragma unroll
+            for (int w = 0; w < GW; ++w)
+                ss += red[parity][w];
+            parity ^= 1;
+        }
+        const float r = rsqrtf(ss / (float)hidden + eps);
+
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int vi = gt + i * G;
+            if (vi < nvec) {
+                float a[E], g[E];
+                Vec<T>::unpack(v[i], a);
+                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E)), g);
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    a[e] = a[e] * r * g[e];
+                st_stream(y + base + (size_t)vi * E, Vec<T>::pack(a));
+            }
+        }
+    }
+}
+
+// One CTA per row, two passes over the row.  VEC: 16-byte vectors (aligned,
+// hidden % E == 0); otherwise one element at a time.  Each thread touches the
+// same elements in both passes, so pass 2 reads back its own pass-1 writes.
+constexpr int kLoopThreads = 256;
+
+template <typename T, bool ADD, bool VEC>
+__global__ void __launch_bounds__(kLoopThreads)
+norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
+                   const T* __restrict__ gamma, T* y, int64_t rows, int64_t hidden, float eps)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr int W = kLoopThreads / 32;
+    const int tid = threadIdx.x;
+    __shared__ float red[2][W];
+
+    pdl_wait();
+    pdl_allow_dependents();
+
+    int parity = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+        const size_t base = (size_t)row * (size_t)hidden;
+        float ss = 0.f;
+        if constexpr (VEC) {
+            const int64_t nvec = hidden / E;
+            for (int64_t vi = tid; vi < nvec; vi += kLoopThreads) {
+                float a[E];
+                uint4 va = ld_stream(x + base + vi * E);
+                if constexpr (ADD) {
+                    float b[E];
+                    Vec<T>::unpack(va, a);
+                    Vec<T>::unpack(ld_stream(residual_in + base + vi * E), b);
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        a[e] = a[e] + b[e];
+                    va = Vec<T>::pack(a);
+                    st_stream(residual_out + base + vi * E, va);
+                }
+                Vec<T>::unpack(va, a);
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    ss = fmaf(a[e], a[e], ss);
+            }
+        } else {
+            for (int64_t i = tid; i < hidden; i += kLoopThreads) {
+                float a = load_elem(x + base + i);
+                if constexpr (ADD) {
+                    a = round_to(a + load_elem(residual_in + base + i), residual_out);
+                    store_elem(residual_out + base + i, a);
+                }
+                ss = fmaf(a, a, ss);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if ((tid & 31) == 0)
+            red[parity][tid >> 5] = ss;
+        __syncthreads();
+        ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+            ss += red[parity][w];
+        parity ^= 1;
+        const float r = rsqrtf(ss / (float)hidden + eps);
+
+        const T* src = ADD ? residual_out : x;
+        if constexpr (VEC) {
+            const int64_t nvec = hidden / E;
+            for (int64_t vi = tid; vi < nvec; vi += kLoopThreads) {
+                float a[E], g[E];
+                Vec<T>::unpack(ld_stream(src + base + vi * E), a);
+                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(gamma + vi * E)), g);
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    a[e] = a[e] * r * g[e];
+                st_stream(y + base + vi * E, Vec<T>::pack(a));
+            }
+        } else {
+            for (int64_t i = tid; i < hidden; i += kLoopThreads) {
+                const float a = load_elem(src + base + i);
+                store_elem(y + base + i, a * r * load_elem(gamma + i));
+            }
+        }
+    }
+}
+
+template <typename T, bool ADD, int VPL>
+cudaError_t launch_rows_gw1(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
+                            int hidden, float eps, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(ceil_div(rows, kRowsPerSmallCta), cap);
+    return launch(norm_rows_kernel<T, ADD, VPL, 1>, dim3((unsigned)grid),
+                  dim3(32 * kRowsPerSmallCta), 0, st, x, ri, ro, g, y, rows, hidden, eps);
+}
+
+template <typename T, bool ADD, int GW>
+cudaError_t launch_rows_gwn(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
+                            int hidden, float eps, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(rows, cap);
+    return launch(norm_rows_kernel<T, ADD, 8, GW>, dim3((unsigned)grid), dim3(32 * GW), 0, st,
+                  x, ri, ro, g, y, rows, hidden, eps);
+}
+
+template <typename T, bool ADD>
+cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void* gv, void* yv,
+                          int64_t rows, int64_t hidden, float eps, cudaStream_t st)
+{
+    const T* x = static_cast<const T*>(xv);
+    const T* ri = static_cast<const T*>(riv);
+    T* ro = static_cast<T*>(rov);
+    const T* g = static_cast<const T*>(gv);
+    T* y = static_cast<T*>(yv);
+    constexpr int E = Vec<T>::N;
+
+    DeviceInfo di;
+    cudaError_t err = current_device_info(&di);
+    if (err != cudaSuccess)
+        return err;
+    const int64_t cap = (int64_t)di.sm_count * 32;
+
+    const bool vec = (hidden % E == 0) && aligned16(x) && aligned16(g) && aligned16(y) &&
+                     (!ADD || (aligned16(ri) && aligned16(ro)));
+    if (vec) {
+        const int64_t nvec = hidden / E;
+        const int h = (int)hidden;
+        if (nvec <= 32)
+            return launch_rows_gw1<T, ADD, 1>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 64)
+            return launch_rows_gw1<T, ADD, 2>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 128)
+            return launch_rows_gw1<T, ADD, 4>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 256)
+            return launch_rows_gw1<T, ADD, 8>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 512)
+            return launch_rows_gwn<T, ADD, 2>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 1024)
+            return launch_rows_gwn<T, ADD, 4>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 2048)
+            return launch_rows_gwn<T, ADD, 8>(x, ri, ro, g, y, rows, h, eps, st, cap);
+        if (nvec <= 4096)
+            return launch_rows_gwn<T, ADD, 16>(x, ri, ro, g, y, rows, h, eps, st, cap);
+    }
+    const int64_t grid = std::min<int64_t>(rows, cap);
+    if (vec)
+        return launch(norm_looped_kernel<T, ADD, true>, dim3((unsigned)grid), dim3(kLoopThreads),
+                      0, st, x, ri, ro, g, y, rows, hidden, eps);
+    return launch(norm_looped_kernel<T, ADD, false>, dim3((unsigned)grid), dim3(kLoopThreads), 0,
+                  st, x, ri, ro, g, y, rows, hidden, eps);
+}
+
+}  // namespace
+
+cudaError_t launch_norm(const void* x, const void* residual_in, void* residual_out,
+                        const void* gamma, void* y, int64_t rows, int64_t hidden, float eps,
+                        arops_dtype dtype, cudaStream_t stream)
+{
+    const bool add = residual_in != nullptr;
+    if (dtype == AROPS_BF16) {
+        if (add)
+            return launch_norm_t<__nv_bfloat16, true>(x, residual_in, residual_out, gamma, y,
+                                                      rows, hidden, eps, stream);
+        return launch_norm_t<__nv_bfloat16, false>(x, nullptr, nullptr, gamma, y, rows, hidden,
+                                                   eps, stream);
+    }
+    if (add)
+        return launch_norm_t<float, true>(x, residual_in, residual_out, gamma, y, rows, hidden,
+                                          eps, stream);
+    return launch_norm_t<float, false>(x, nullptr, nullptr, gamma, y, rows, hidden, eps, stream);
+}
+
+}  // namespace arops

@@ -1,0 +1,97 @@
+"""Decode-step chain (28 layers x 4 operators) on the GPU against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import swiglu_ar_tts_b200 as ops
+from swiglu_ar_tts_b200.chain import DecodeChain
+from swiglu_ar_tts_b200.inputs import ChainShape
+from tolerance import check, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _pair_scale(x):
+    half = x.shape[-1] // 2
+    m = np.maximum(np.abs(x[..., :half]), np.abs(x[..., half:]))
+    return np.concatenate([m, m], axis=-1)
+
+
+def _compare_step(chain, outs):
+    for l in range(chain.shape.layers):
+        check(chain.y_attn[l], outs["y_attn"][l], "bf16", what=f"y_attn[{l}]")
+        check(chain.y_mlp[l], outs["y_mlp"][l], "bf16", what=f"y_mlp[{l}]")
+        check(chain.act[l], outs["act"][l], "bf16", what=f"act[{l}]")
+        check(chain.q_out[l], outs["q"][l], "bf16", _pair_scale(to_f64(chain.host_inputs["q"][l])),
+              what=f"q[{l}]")
+        check(chain.k_out[l], outs["k"][l], "bf16", _pair_scale(to_f64(chain.host_inputs["k"][l])),
+              what=f"k[{l}]")
+
+
+def _oracle_inputs(chain):
+    return {k: [to_f64(t) for t in v] for k, v in chain.host_inputs.items() if k != "residual"}
+
+
+def test_decode_chain_batch5_300_steps():
+    """28 layers x 300 steps at batch 5: the residual is bit-exact after every
+    step; every operator output matches at sampled steps."""
+    chain = DecodeChain(ChainShape(batch=5))
+    orc = oracle.get()
+    inp = _oracle_inputs(chain)
+    res = to_f64(chain.residual0.cpu())
+    sampled = {0, 1, 2, 150, 299}
+    for s in range(300):
+        chain.step(s)
+        res, outs = orc.decode_step(res, inp, s, chain.eps, chain.theta, chain.sections, "bf16",
+                                    outputs=s in sampled)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_f64(chain.residual), res), f"residual differs at step {s}"
+        if s in sampled:
+            _compare_step(chain, outs)
+
+
+@pytest.mark.parametrize("batch", [5, 256])
+def test_graph_replay_equals_eager(batch):
+    eager = DecodeChain(ChainShape(batch=batch), seed=7)
+    graph = DecodeChain(ChainShape(batch=batch), host_inputs=eager.host_inputs)
+    graph.capture()
+    for s in range(4):
+        eager.step(s)
+        graph.replay(s)
+    torch.cuda.synchronize()
+    assert torch.equal(eager.residual, graph.residual)
+    for l in range(eager.shape.layers):
+        for name in ("y_attn", "y_mlp", "act", "q_out", "k_out"):
+            assert torch.equal(getattr(eager, name)[l], getattr(graph, name)[l]), (name, l)
+
+
+def test_pdl_gives_identical_results():
+    shape = ChainShape(batch=256, layers=4)
+    a = DecodeChain(shape, seed=3)
+    b = DecodeChain(shape, host_inputs=a.host_inputs)
+    for s in range(3):
+        a.step(s)
+    old = ops.set_pdl(True)
+    try:
+        for s in range(3):
+            b.step(s)
+        b2 = DecodeChain(shape, host_inputs=a.host_inputs)
+        b2.capture()
+        for s in range(3):
+            b2.replay(s)
+    finally:
+        ops.set_pdl(old)
+    torch.cuda.synchronize()
+    for other in (b, b2):
+        assert torch.equal(a.residual, other.residual)
+        for l in range(shape.layers):
+            assert torch.equal(a.act[l], other.act[l]) and torch.equal(a.q_out[l], other.q_out[l])
+
+
+def test_launch_count_per_step():
+    chain = DecodeChain(ChainShape(batch=5, layers=3))
+    before = ops.launch_count()
+    chain.step(0)
+    torch.cuda.synchronize()
+    assert ops.launch_count() - before == 12 == chain.launches_per_step

@@ -1,0 +1,83 @@
+"""SwiGLU on the GPU against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import swiglu_ar_tts_b200 as ops
+from swiglu_ar_tts_b200 import inputs
+from gpu_util import Guarded, dev, misaligned
+from tolerance import check, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(rows, inter, dtype, seed=0):
+    inp = inputs.swiglu_inputs(rows, inter, dtype, seed)
+    out = ops.swiglu(dev(inp["gate"]), dev(inp["up"]))
+    torch.cuda.synchronize()
+    return out, oracle.get().swiglu(inp["gate"], inp["up"])
+
+
+def test_swiglu_bf16_8192x6144():
+    """The SwiGLU workload: gate ~ N(0, 2^2), up ~ N(0,1), separate [8192 x 6144]."""
+    out, exact = _run(8192, 6144, "bf16")
+    st = check(out, exact, "bf16", what="swiglu 8192x6144")
+    assert st["max_ulp"] <= 1.0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 8), (1, 1), (3, 13), (5, 6144), (7, 1001), (64, 6144),
+                                   (1, 8 * 256 * 4 + 5), (300, 4097)])
+def test_swiglu_shapes(dtype, shape):
+    out, exact = _run(*shape, dtype, seed=shape[0] * 7 + shape[1])
+    check(out, exact, dtype, what=f"swiglu {dtype} {shape}")
+
+
+def test_swiglu_special_values():
+    """g = +-0 gives +-0 exactly; large |g| tends to g*u or to 0."""
+    g = torch.tensor([0.0, -0.0, 1.0, -1.0, 2.0, 20.0, -20.0, 80.0, -80.0, -100.0, 88.0, -88.0,
+                      1e-30, -1e-30, 3.0, -3.0], dtype=torch.float32)
+    u = torch.tensor([1.0, 1.0, 1.0, 1.0, 1.0, 1.5, 1.5, -2.0, -2.0, 1.0, 1.0, 1.0, 1.0, 1.0, 0.0,
+                      -0.0], dtype=torch.float32)
+    for dt in (torch.float32, torch.bfloat16):
+        gd, ud = g.to(dt).cuda(), u.to(dt).cuda()
+        out = ops.swiglu(gd, ud)
+        torch.cuda.synchronize()
+        exact = oracle.get().swiglu(g.to(dt), u.to(dt))
+        o = to_f64(out)
+        assert o[0] == 0.0 and o[1] == 0.0
+        check(out, exact, "bf16" if dt == torch.bfloat16 else "f32", what=f"special {dt}")
+
+
+def test_swiglu_in_place_and_guarded():
+    inp = inputs.swiglu_inputs(9, 777, "bf16", 5)
+    gate = dev(inp["gate"])
+    out = Guarded((9, 777), torch.bfloat16, fill=gate)
+    ops.swiglu(out.t, dev(inp["up"]), out=out.t)  # out aliases gate
+    torch.cuda.synchronize()
+    out.check()
+    check(out.t, oracle.get().swiglu(inp["gate"], inp["up"]), "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_swiglu_misaligned(dtype):
+    inp = inputs.swiglu_inputs(4, 1000, dtype, 6)
+    out = ops.swiglu(misaligned(dev(inp["gate"])), misaligned(dev(inp["up"]), 3))
+    torch.cuda.synchronize()
+    check(out, oracle.get().swiglu(inp["gate"], inp["up"]), dtype)
+
+
+def test_swiglu_empty():
+    g = torch.empty(0, 6144, dtype=torch.bfloat16, device="cuda")
+    assert ops.swiglu(g, g).shape == (0, 6144)
+    torch.cuda.synchronize()
+
+
+def test_swiglu_matches_oracle_rounding_mostly_exactly():
+    """fp32 math differs from the correctly rounded result only next to a
+    rounding boundary, so nearly every element is bit-exact."""
+    out, exact = _run(256, 6144, "bf16", seed=17)
+    o_hat = oracle.get().round_to(exact, "bf16")
+    frac = np.count_nonzero(to_f64(out) != o_hat) / o_hat.size
+    assert frac < 1e-3, frac

@@ -145,6 +145,25 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  */
 AROPS_API int arops_set_pdl(int enable);
 
+/*
+ * Kernel family selection (process-wide).  Enabled (the default), 16-byte
+ * aligned rows are processed by the streaming kernels, which stage rows through
+ * shared memory with bulk asynchronous copies; disabled, by the register
+ * kernels.  Both compute the same results; the switch exists so that both can
+ * be tested and measured.  Returns the old setting.
+ */
+AROPS_API int arops_set_streaming(int enable);
+
+/*
+ * Device-side error bits of the current device, OR-ed by kernels that abandon
+ * their work: AROPS_DEVICE_ERR_TIMEOUT means a bulk copy into shared memory did
+ * not complete within a second (the kernel's outputs are then undefined).  The
+ * call synchronises the device (it is a plain copy from device memory) and, if
+ * `clear` is non-zero, resets the bits.  Healthy runs always read 0.
+ */
+#define AROPS_DEVICE_ERR_TIMEOUT 1u
+AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear);
+
 /* Number of kernels this library has launched in this process (all devices). */
 AROPS_API uint64_t arops_launch_count(void);
 

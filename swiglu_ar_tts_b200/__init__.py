@@ -18,7 +18,8 @@ import threading
 import torch
 
 __all__ = [
-    "rmsnorm", "add_rmsnorm", "mrope_qk", "swiglu", "set_pdl", "launch_count",
+    "rmsnorm", "add_rmsnorm", "mrope_qk", "swiglu", "set_pdl", "set_streaming",
+    "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
 ]
 
@@ -70,6 +71,10 @@ def lib() -> ctypes.CDLL:
             getattr(L, fn).restype = ctypes.c_int
         L.arops_set_pdl.argtypes = [ctypes.c_int]
         L.arops_set_pdl.restype = ctypes.c_int
+        L.arops_set_streaming.argtypes = [ctypes.c_int]
+        L.arops_set_streaming.restype = ctypes.c_int
+        L.arops_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+        L.arops_device_errors.restype = ctypes.c_int
         L.arops_launch_count.restype = ctypes.c_uint64
         L.arops_status_string.argtypes = [ctypes.c_int]
         L.arops_status_string.restype = ctypes.c_char_p
@@ -199,6 +204,19 @@ def swiglu(gate: torch.Tensor, up: torch.Tensor, out: torch.Tensor | None = None
 def set_pdl(enable: bool) -> bool:
     """Turn programmatic dependent launch on or off; returns the old setting."""
     return bool(lib().arops_set_pdl(1 if enable else 0))
+
+
+def set_streaming(enable: bool) -> bool:
+    """Choose the shared-memory streaming kernels (default) or the register
+    kernels; returns the old setting.  Both give the same results."""
+    return bool(lib().arops_set_streaming(1 if enable else 0))
+
+
+def device_errors(clear: bool = True) -> int:
+    """Device-side error bits (1 = a bulk copy timed out); synchronises."""
+    v = ctypes.c_uint32(0)
+    _check(lib().arops_device_errors(ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)
 
 
 def launch_count() -> int:

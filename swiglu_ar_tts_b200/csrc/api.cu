@@ -14,6 +14,7 @@ namespace {
 
 thread_local char g_last_error[512] = "";
 std::atomic<int> g_pdl{0};
+std::atomic<int> g_streaming{1};
 std::atomic<uint64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
@@ -49,6 +50,32 @@ bool valid_dtype(arops_dtype d)
 
 }  // namespace
 
+// The device error word: kernels that abandon their work (a bounded wait ran
+// out) OR a bit into it; arops_device_errors reads and clears it.
+__device__ unsigned int g_device_errors = 0;
+
+namespace {
+std::atomic<unsigned*> g_error_word[kMaxDevices];
+}
+
+cudaError_t device_error_word(unsigned** word)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    unsigned* p = (dev >= 0 && dev < kMaxDevices) ? g_error_word[dev].load() : nullptr;
+    if (p == nullptr) {
+        err = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_errors);
+        if (err != cudaSuccess)
+            return err;
+        if (dev >= 0 && dev < kMaxDevices)
+            g_error_word[dev].store(p);
+    }
+    *word = p;
+    return cudaSuccess;
+}
+
 cudaError_t current_device_info(DeviceInfo* info)
 {
     int dev = 0;
@@ -70,6 +97,11 @@ cudaError_t current_device_info(DeviceInfo* info)
 bool pdl_enabled()
 {
     return g_pdl.load(std::memory_order_relaxed) != 0;
+}
+
+bool streaming_enabled()
+{
+    return g_streaming.load(std::memory_order_relaxed) != 0;
 }
 
 void count_launch()
@@ -187,9 +219,30 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
                      "arops_swiglu");
 }
 
+AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear)
+{
+    if (!errors)
+        return fail(AROPS_ERR_INVALID, "arops_device_errors: errors is null");
+    unsigned v = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_device_errors, sizeof(v));
+    if (err == cudaSuccess && clear) {
+        const unsigned zero = 0;
+        err = cudaMemcpyToSymbol(g_device_errors, &zero, sizeof(zero));
+    }
+    if (err != cudaSuccess)
+        return from_cuda(err, "arops_device_errors");
+    *errors = v;
+    return ok();
+}
+
 AROPS_API int arops_set_pdl(int enable)
 {
     return g_pdl.exchange(enable ? 1 : 0);
+}
+
+AROPS_API int arops_set_streaming(int enable)
+{
+    return g_streaming.exchange(enable ? 1 : 0);
 }
 
 AROPS_API uint64_t arops_launch_count(void)

@@ -114,8 +114,15 @@ struct DeviceInfo {
 // SM count of the current device (queried once per device).
 cudaError_t current_device_info(DeviceInfo* info);
 
+// Device address of the library's error word on the current device (resolved
+// once per device with cudaGetSymbolAddress).
+cudaError_t device_error_word(unsigned** word);
+
 // Whether kernels are launched with the PDL attribute.
 bool pdl_enabled();
+
+// Whether the shared-memory streaming (bulk-copy) kernels may be chosen.
+bool streaming_enabled();
 
 // Counts one launch.
 void count_launch();
@@ -152,6 +159,35 @@ inline bool aligned16(const void* p)
 inline int64_t ceil_div(int64_t a, int64_t b)
 {
     return (a + b - 1) / b;
+}
+
+__host__ __device__ inline uint32_t round_up(uint32_t a, uint32_t b)
+{
+    return (a + b - 1) / b * b;
+}
+
+// Shared memory an SM offers to one CTA / to all its CTAs (B200: 227 / 228 KB).
+constexpr uint32_t kMaxSmemPerCta = 227u * 1024u;
+constexpr uint32_t kSmemPerSm = 228u * 1024u;
+
+// Resident CTAs per SM for `kernel` at this block size and dynamic smem.  For
+// kernels that use dynamic shared memory it first raises the kernel's limit
+// (above the 48 KB default) and asks for the largest shared-memory carveout:
+// otherwise the driver may configure only as much shared memory as one CTA
+// needs, and the CTAs the grid was sized for would run in waves.
+template <typename K>
+cudaError_t resident_ctas(K kernel, int threads, size_t smem, int* ctas)
+{
+    if (smem > 0) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, kernel, threads, smem);
 }
 
 // Launchers (one per operator), called after argument validation.

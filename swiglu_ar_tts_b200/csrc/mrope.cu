@@ -19,6 +19,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace arops {
 namespace {
@@ -75,6 +76,23 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
         const int32_t ph = __ldg(pos + tokens + t);
         const int32_t pw = __ldg(pos + 2 * tokens + t);
 
+        // the first batch of heads is loaded before the angles are evaluated, so
+        // the q/k loads and the position loads share one memory latency
+        uint4 lo[U], hi[U];
+        auto load_batch = [&](int h0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int h = h0 + u * G;
+                if (h < nh) {
+                    const T* src = (h < hq) ? q + ((size_t)t * hq + h) * D
+                                            : k + ((size_t)t * hk + (h - hq)) * D;
+                    lo[u] = ld_stream(src + j0);
+                    hi[u] = ld_stream(src + HALF + j0);
+                }
+            }
+        };
+        load_batch(hg);
+
         // this lane's share of the E angles of block pv ...
         float cs[F], sn[F];
 #pragma unroll
@@ -92,17 +110,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
         }
 
         for (int h0 = hg; h0 < nh; h0 += G * U) {
-            uint4 lo[U], hi[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int h = h0 + u * G;
-                if (h < nh) {
-                    const T* src = (h < hq) ? q + ((size_t)t * hq + h) * D
-                                            : k + ((size_t)t * hk + (h - hq)) * D;
-                    lo[u] = ld_stream(src + j0);
-                    hi[u] = ld_stream(src + HALF + j0);
-                }
-            }
+            if (h0 != hg)
+                load_batch(h0);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int h = h0 + u * G;
@@ -121,6 +130,134 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
                     st_stream(dst + HALF + j0, Vec<T>::pack(ob));
                 }
             }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming kernel (default for 16-byte-aligned q/k).  Each warp owns tokens
+// gw, gw + nw, ... (gw = global warp index, nw = warps in the grid) and a ring
+// of `slots` shared-memory slots, each holding one token's q and k heads.  Lane
+// 0 keeps `slots` tokens in flight as bulk copies (TMA); the warp evaluates the
+// token's angles (positions are fetched one token ahead) while its copy is in
+// flight, then rotates the heads out of shared memory and stores them.  Warps
+// never wait on each other, so an SM has ~30 tokens (~180 KB) requested at once.
+// ---------------------------------------------------------------------------
+constexpr int kTmaWarps = 4;
+
+template <typename T, int P>
+__global__ void __launch_bounds__(32 * kTmaWarps)
+mrope_tma_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __restrict__ pos,
+                 int64_t tokens, int hq, int hk, int slots, const __grid_constant__ MropeParams prm,
+                 unsigned* err_word)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr int G = 32 / P;
+    constexpr int HALF = P * E;
+    constexpr int D = 2 * HALF;
+    constexpr int F = (E >= G) ? E / G : 1;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int pv = lane % P;
+    const int hg = lane / P;
+    const int j0 = pv * E;
+    const int nh = hq + hk;
+    const uint32_t q_bytes = (uint32_t)hq * D * sizeof(T);
+    const uint32_t k_bytes = (uint32_t)hk * D * sizeof(T);
+    const uint32_t slot = round_up(q_bytes + k_bytes, 128);
+    unsigned char* ring = smem + (size_t)warp * slots * slot;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kTmaWarps * slots * slot) +
+                     warp * slots;
+    const int64_t gw = (int64_t)blockIdx.x * kTmaWarps + warp;
+    const int64_t nw = (int64_t)gridDim.x * kTmaWarps;
+    const int64_t my = tokens > gw ? (tokens - 1 - gw) / nw + 1 : 0;
+
+    if (lane == 0) {
+        for (int i = 0; i < slots; ++i)
+            mbar_init(smem_addr(&bars[i]), 1);
+        mbar_init_fence();
+    }
+    __syncwarp();
+
+    pdl_wait();
+    pdl_allow_dependents();
+
+    int64_t issued = 0;  // lane 0 only
+    auto issue = [&](int64_t j) {
+        const int64_t t = gw + j * nw;
+        const int sidx = (int)(j % slots);
+        const uint32_t bar = smem_addr(&bars[sidx]);
+        unsigned char* dst = ring + (size_t)sidx * slot;
+        mbar_arrive_expect_tx(bar, q_bytes + k_bytes);
+        if (q_bytes)
+            bulk_load(smem_addr(dst), q + t * hq * D, q_bytes, bar);
+        if (k_bytes)
+            bulk_load(smem_addr(dst + q_bytes), k + t * hk * D, k_bytes, bar);
+    };
+    if (lane == 0)
+        for (; issued < slots && issued < my; ++issued)
+            issue(issued);
+
+    int32_t npt = 0, nph = 0, npw = 0;
+    if (my > 0) {
+        npt = __ldg(pos + gw);
+        nph = __ldg(pos + tokens + gw);
+        npw = __ldg(pos + 2 * tokens + gw);
+    }
+    for (int64_t j = 0; j < my; ++j) {
+        const int64_t t = gw + j * nw;
+        const int32_t pt = npt, ph = nph, pw = npw;
+        if (j + 1 < my) {  // the next token's positions, one step ahead
+            npt = __ldg(pos + t + nw);
+            nph = __ldg(pos + tokens + t + nw);
+            npw = __ldg(pos + 2 * tokens + t + nw);
+        }
+        float cs[F], sn[F];
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            const int jj = j0 + ((hg * F + f) % E);
+            rope_cos_sin(prm.inv_freq[jj], position_of(jj, prm, pt, ph, pw), &cs[f], &sn[f]);
+        }
+        float c[E], s[E];
+#pragma unroll
+        for (int m = 0; m < E; ++m) {
+            const int src = pv + P * ((m / F) % G);
+            c[m] = __shfl_sync(0xFFFFFFFFu, cs[m % F], src);
+            s[m] = __shfl_sync(0xFFFFFFFFu, sn[m % F], src);
+        }
+
+        const int sidx = (int)(j % slots);
+        const bool ok = mbar_wait(smem_addr(&bars[sidx]), (uint32_t)((j / slots) & 1));
+        if (__any_sync(0xFFFFFFFFu, !ok)) {
+            if (lane == 0) {
+                record_device_error(err_word, kDeviceErrTimeout);
+                for (int64_t kk = j; kk < issued; ++kk)
+                    mbar_wait(smem_addr(&bars[kk % slots]), (uint32_t)((kk / slots) & 1));
+            }
+            return;
+        }
+        const unsigned char* src = ring + (size_t)sidx * slot;
+        for (int h = hg; h < nh; h += G) {
+            float a[E], b[E], oa[E], ob[E];
+            const unsigned char* hp = src + (size_t)h * D * sizeof(T);
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(hp + j0 * sizeof(T)), a);
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(hp + (HALF + j0) * sizeof(T)), b);
+#pragma unroll
+            for (int m = 0; m < E; ++m) {
+                oa[m] = a[m] * c[m] - b[m] * s[m];
+                ob[m] = b[m] * c[m] + a[m] * s[m];
+            }
+            T* dst = (h < hq) ? q_out + ((size_t)t * hq + h) * D
+                              : k_out + ((size_t)t * hk + (h - hq)) * D;
+            st_stream(dst + j0, Vec<T>::pack(oa));
+            st_stream(dst + HALF + j0, Vec<T>::pack(ob));
+        }
+        __syncwarp();  // every lane has read the slot; it can take the next copy
+        if (lane == 0 && issued < my) {
+            issue(issued);
+            ++issued;
         }
     }
 }
@@ -168,6 +305,53 @@ cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t 
                   a.pos, a.tokens, (int)a.n_q_heads, (int)a.n_k_heads, prm);
 }
 
+// Streaming launch; cudaErrorNotSupported when two slots per warp do not fit.
+template <typename T, int P>
+cudaError_t launch_tma(const MropeArgs& a, const MropeParams& prm, cudaStream_t st,
+                       const DeviceInfo& di)
+{
+    const uint32_t tok = (uint32_t)(a.n_q_heads + a.n_k_heads) * a.head_dim * sizeof(T);
+    const uint32_t slot = round_up(tok, 128);
+    // ~96 KB of slots per CTA lets two CTAs (8 warps) share an SM
+    int slots = (int)std::min<uint32_t>(8, (96u * 1024u) / (kTmaWarps * slot));
+    slots = std::max(slots, 2);
+    const uint32_t smem = (uint32_t)kTmaWarps * slots * (slot + 8) + 128;
+    if (smem > kMaxSmemPerCta)
+        return cudaErrorNotSupported;
+    auto kernel = mrope_tma_kernel<T, P>;
+    int per_sm = 0;
+    cudaError_t err = resident_ctas(kernel, 32 * kTmaWarps, smem, &per_sm);
+    if (err != cudaSuccess)
+        return err;
+    if (per_sm < 1)
+        return cudaErrorNotSupported;
+    unsigned* word = nullptr;
+    err = device_error_word(&word);
+    if (err != cudaSuccess)
+        return err;
+    const int64_t grid =
+        std::min<int64_t>(ceil_div(a.tokens, kTmaWarps), (int64_t)di.sm_count * per_sm);
+    return launch(kernel, dim3((unsigned)grid), dim3(32 * kTmaWarps), smem, st,
+                  static_cast<const T*>(a.q), static_cast<const T*>(a.k),
+                  static_cast<T*>(a.q_out), static_cast<T*>(a.k_out), a.pos, a.tokens,
+                  (int)a.n_q_heads, (int)a.n_k_heads, slots, prm, word);
+}
+
+template <typename T>
+cudaError_t try_tma(const MropeArgs& a, const MropeParams& prm, cudaStream_t st,
+                    const DeviceInfo& di, int p)
+{
+    switch (p) {
+    case 1: return launch_tma<T, 1>(a, prm, st, di);
+    case 2: return launch_tma<T, 2>(a, prm, st, di);
+    case 4: return launch_tma<T, 4>(a, prm, st, di);
+    case 8: return launch_tma<T, 8>(a, prm, st, di);
+    case 16: return launch_tma<T, 16>(a, prm, st, di);
+    case 32: return launch_tma<T, 32>(a, prm, st, di);
+    default: return cudaErrorNotSupported;
+    }
+}
+
 template <typename T>
 cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStream_t st)
 {
@@ -180,6 +364,11 @@ cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStrea
     const bool aligned = aligned16(a.q) && aligned16(a.q_out) &&
                          (a.n_k_heads == 0 || (aligned16(a.k) && aligned16(a.k_out)));
     const int64_t cap = (int64_t)di.sm_count * 64;
+    if (aligned && half % E == 0 && streaming_enabled()) {
+        err = try_tma<T>(a, prm, st, di, half / E);
+        if (err != cudaErrorNotSupported)
+            return err;
+    }
     if (aligned && half % E == 0) {
         switch (half / E) {
         case 1: return launch_vec<T, 1>(a, prm, st, cap);

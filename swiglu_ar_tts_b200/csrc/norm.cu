@@ -5,7 +5,9 @@
 // module).  Norm+Residual (Triton kernel-fusion post for Qwen3-TTS, section 3):
 // residual_out = round(x + residual_in), y = RMSNorm(residual_out), in one pass.
 //
-// Design: the row lives in registers.  A row of `hidden` elements is split into
+// Two designs.  The streaming kernel (below) stages rows through shared memory
+// with bulk copies and is the default for 16-byte-aligned rows.  The register
+// kernels keep the row in registers:  a row of `hidden` elements is split into
 // 16-byte vectors; a group of 32*GW threads owns the row and every thread holds
 // VPL vectors, so global memory is read once and written once (x, residual ->
 // residual_out, y) with fully coalesced 128-bit accesses.  The sum of squares is
@@ -17,9 +19,140 @@
 // Rows longer than 4096 vectors, and unaligned or ragged rows, take a looped
 // kernel that makes a second pass over the row (served from L2).
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace arops {
 namespace {
+
+// ---------------------------------------------------------------------------
+// Streaming kernel (the default for 16-byte-aligned rows).  A persistent CTA
+// owns rows blockIdx.x, blockIdx.x + gridDim.x, ...  One thread keeps `stages`
+// rows in flight as bulk copies (TMA) into a ring of shared-memory slots, each
+// slot holding the row of x (and of the residual); gamma is copied once per
+// CTA.  As a row lands, the CTA adds the residual, writes residual_out, reduces
+// the sum of squares (warp shuffles, then one shared-memory step), and writes
+// y.  With several CTAs per SM and 4 stages, an SM has its whole share of a
+// 4096 x 2048 problem requested within the first microsecond, so the kernel
+// runs at the rate DRAM returns data rather than at the rate warps can issue
+// dependent loads.
+// ---------------------------------------------------------------------------
+template <typename T, bool ADD, int THREADS>
+__global__ void __launch_bounds__(THREADS)
+norm_tma_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
+                T* y, int64_t rows, int hidden, float eps, int stages, unsigned* err_word)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr int W = THREADS / 32;
+    constexpr int NT = ADD ? 2 : 1;  // tensors streamed per row
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red[W];
+
+    const int tid = threadIdx.x;
+    const int nvec = hidden / E;
+    const uint32_t row_bytes = (uint32_t)hidden * (uint32_t)sizeof(T);
+    const uint32_t slot = round_up(row_bytes, 128);
+    unsigned char* s_gamma = smem;
+    unsigned char* s_ring = smem + slot;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s_ring + (size_t)stages * NT * slot);
+    const uint32_t gamma_bar = smem_addr(&bars[stages]);
+    const int64_t my_rows =
+        rows > (int64_t)blockIdx.x ? (rows - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s <= stages; ++s)
+            mbar_init(smem_addr(&bars[s]), 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    pdl_wait();
+    pdl_allow_dependents();
+
+    int64_t issued = 0;  // meaningful in thread 0 only
+    auto issue = [&](int64_t j) {
+        const int s = (int)(j % stages);
+        const int64_t row = (int64_t)blockIdx.x + j * gridDim.x;
+        const uint32_t bar = smem_addr(&bars[s]);
+        unsigned char* dst = s_ring + (size_t)s * NT * slot;
+        mbar_arrive_expect_tx(bar, NT * row_bytes);
+        bulk_load(smem_addr(dst), x + row * hidden, row_bytes, bar);
+        if constexpr (ADD)
+            bulk_load(smem_addr(dst + slot), residual_in + row * hidden, row_bytes, bar);
+    };
+    if (tid == 0) {
+        mbar_arrive_expect_tx(gamma_bar, row_bytes);
+        bulk_load(smem_addr(s_gamma), gamma, row_bytes, gamma_bar);
+        for (; issued < stages && issued < my_rows; ++issued)
+            issue(issued);
+    }
+
+    bool ok = mbar_wait(gamma_bar, 0);
+    for (int64_t j = 0; j < my_rows; ++j) {
+        const int s = (int)(j % stages);
+        ok = ok && mbar_wait(smem_addr(&bars[s]), (uint32_t)((j / stages) & 1));
+        if (__syncthreads_or(!ok)) {
+            // a copy did not land in time: record it, let this CTA's copies
+            // still in flight finish (bounded), and give up
+            if (tid == 0) {
+                record_device_error(err_word, kDeviceErrTimeout);
+                mbar_wait(gamma_bar, 0);
+                for (int64_t k = j; k < issued; ++k)
+                    mbar_wait(smem_addr(&bars[k % stages]), (uint32_t)((k / stages) & 1));
+            }
+            return;
+        }
+        // every thread is past row j-1 (it reached the barrier above), so row
+        // j-1's slot can take row j-1+stages; at j == 0 no slot is free yet
+        if (tid == 0 && j >= 1 && issued < my_rows) {
+            issue(issued);
+            ++issued;
+        }
+
+        const int64_t row = (int64_t)blockIdx.x + j * gridDim.x;
+        unsigned char* sx = s_ring + (size_t)s * NT * slot;
+        float ss = 0.f;
+        for (int v = tid; v < nvec; v += THREADS) {
+            uint4 va = *reinterpret_cast<const uint4*>(sx + (size_t)v * 16);
+            float a[E];
+            if constexpr (ADD) {
+                float b[E];
+                Vec<T>::unpack(va, a);
+                Vec<T>::unpack(*reinterpret_cast<const uint4*>(sx + slot + (size_t)v * 16), b);
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    a[e] = a[e] + b[e];
+                va = Vec<T>::pack(a);  // the residual rounded to T
+                st_stream(residual_out + row * hidden + (int64_t)v * E, va);
+                *reinterpret_cast<uint4*>(sx + (size_t)v * 16) = va;  // kept for the second pass
+            }
+            Vec<T>::unpack(va, a);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                ss = fmaf(a[e], a[e], ss);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if ((tid & 31) == 0)
+            red[tid >> 5] = ss;
+        __syncthreads();
+        ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+            ss += red[w];
+        const float r = rsqrtf(ss / (float)hidden + eps);
+
+        for (int v = tid; v < nvec; v += THREADS) {
+            float a[E], g[E];
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), a);
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(s_gamma + (size_t)v * 16), g);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                a[e] = a[e] * r * g[e];
+            st_stream(y + row * hidden + (int64_t)v * E, Vec<T>::pack(a));
+        }
+    }
+}
 
 constexpr int kRowsPerSmallCta = 2;  // GW == 1: two warps, one row each
 
@@ -213,6 +346,50 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
     }
 }
 
+// Chooses block size and ring depth for the streaming kernel; returns
+// cudaErrorNotSupported when two ring slots and gamma do not fit in one CTA's
+// shared memory (very long rows), so that the register kernels take over.
+template <typename T, bool ADD, int THREADS>
+cudaError_t launch_norm_tma_t(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
+                              int hidden, float eps, cudaStream_t st, const DeviceInfo& di)
+{
+    constexpr int NT = ADD ? 2 : 1;
+    const uint32_t slot = round_up((uint32_t)hidden * sizeof(T), 128);
+    const uint32_t fixed = slot + 8 * 9 + 128;  // gamma, barriers, slack
+    int stages = 4;
+    while (stages > 2 && fixed + (uint32_t)stages * NT * slot > kMaxSmemPerCta)
+        --stages;
+    const uint32_t smem = fixed + (uint32_t)stages * NT * slot;
+    if (smem > kMaxSmemPerCta)
+        return cudaErrorNotSupported;
+    auto kernel = norm_tma_kernel<T, ADD, THREADS>;
+    int per_sm = 0;
+    cudaError_t err = resident_ctas(kernel, THREADS, smem, &per_sm);
+    if (err != cudaSuccess)
+        return err;
+    if (per_sm < 1)
+        return cudaErrorNotSupported;
+    unsigned* word = nullptr;
+    err = device_error_word(&word);
+    if (err != cudaSuccess)
+        return err;
+    const int64_t grid = std::min<int64_t>(rows, (int64_t)di.sm_count * per_sm);
+    return launch(kernel, dim3((unsigned)grid), dim3(THREADS), smem, st, x, ri, ro, g, y, rows,
+                  hidden, eps, stages, word);
+}
+
+template <typename T, bool ADD>
+cudaError_t launch_norm_tma(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
+                            int hidden, float eps, cudaStream_t st, const DeviceInfo& di)
+{
+    const int nvec = hidden / Vec<T>::N;
+    if (nvec <= 64)
+        return launch_norm_tma_t<T, ADD, 64>(x, ri, ro, g, y, rows, hidden, eps, st, di);
+    if (nvec <= 128)
+        return launch_norm_tma_t<T, ADD, 128>(x, ri, ro, g, y, rows, hidden, eps, st, di);
+    return launch_norm_tma_t<T, ADD, 256>(x, ri, ro, g, y, rows, hidden, eps, st, di);
+}
+
 template <typename T, bool ADD, int VPL>
 cudaError_t launch_rows_gw1(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
                             int hidden, float eps, cudaStream_t st, int64_t cap)
@@ -250,6 +427,11 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
 
     const bool vec = (hidden % E == 0) && aligned16(x) && aligned16(g) && aligned16(y) &&
                      (!ADD || (aligned16(ri) && aligned16(ro)));
+    if (vec && streaming_enabled()) {
+        err = launch_norm_tma<T, ADD>(x, ri, ro, g, y, rows, (int)hidden, eps, st, di);
+        if (err != cudaErrorNotSupported)
+            return err;
+    }
     if (vec) {
         const int64_t nvec = hidden / E;
         const int h = (int)hidden;

@@ -7,6 +7,7 @@
 // cache hints, and a grid-stride loop over a grid sized to the SM count.  The
 // ragged tail (n % 8 elements) is handled by block 0 in the same launch.
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace arops {
 namespace {
@@ -77,6 +78,95 @@ swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming kernel (default for 16-byte-aligned buffers with n % 8 == 0).  The
+// flat array is cut into chunks of kChunk elements; warp gw of the grid owns
+// chunks gw, gw + nw, ... and a ring of `slots` shared-memory slots, each
+// holding one chunk of gate and of up.  Lane 0 keeps `slots` chunks in flight
+// as bulk copies (TMA); the warp computes a chunk as soon as it lands and
+// stores it with coalesced 16-byte stores.  No thread ever waits on another
+// warp, and an SM keeps ~190 KB of reads outstanding at all times.
+// ---------------------------------------------------------------------------
+constexpr int kChunk = 2048;  // elements per chunk and tensor
+constexpr int kTmaWarps = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(32 * kTmaWarps)
+swiglu_tma_kernel(const T* gate, const T* up, T* out, int64_t n, int slots, unsigned* err_word)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr uint32_t kBytes = kChunk * sizeof(T);
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    unsigned char* ring = smem + (size_t)warp * slots * 2 * kBytes;
+    uint64_t* bars =
+        reinterpret_cast<uint64_t*>(smem + (size_t)kTmaWarps * slots * 2 * kBytes) + warp * slots;
+    const int64_t gw = (int64_t)blockIdx.x * kTmaWarps + warp;
+    const int64_t nw = (int64_t)gridDim.x * kTmaWarps;
+    const int64_t chunks = (n + kChunk - 1) / kChunk;
+    const int64_t my = chunks > gw ? (chunks - 1 - gw) / nw + 1 : 0;
+
+    if (lane == 0) {
+        for (int i = 0; i < slots; ++i)
+            mbar_init(smem_addr(&bars[i]), 1);
+        mbar_init_fence();
+    }
+    __syncwarp();
+
+    pdl_wait();
+    pdl_allow_dependents();
+
+    int64_t issued = 0;  // lane 0 only
+    auto issue = [&](int64_t j) {
+        const int64_t c = gw + j * nw;
+        const int64_t base = c * kChunk;
+        const int64_t left = n - base;
+        const uint32_t bytes = (uint32_t)((left < kChunk ? left : kChunk) * sizeof(T));
+        const int sidx = (int)(j % slots);
+        const uint32_t bar = smem_addr(&bars[sidx]);
+        unsigned char* dst = ring + (size_t)sidx * 2 * kBytes;
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_load(smem_addr(dst), gate + base, bytes, bar);
+        bulk_load(smem_addr(dst + kBytes), up + base, bytes, bar);
+    };
+    if (lane == 0)
+        for (; issued < slots && issued < my; ++issued)
+            issue(issued);
+
+    for (int64_t j = 0; j < my; ++j) {
+        const int sidx = (int)(j % slots);
+        const bool ok = mbar_wait(smem_addr(&bars[sidx]), (uint32_t)((j / slots) & 1));
+        if (__any_sync(0xFFFFFFFFu, !ok)) {
+            if (lane == 0) {
+                record_device_error(err_word, kDeviceErrTimeout);
+                for (int64_t k = j; k < issued; ++k)
+                    mbar_wait(smem_addr(&bars[k % slots]), (uint32_t)((k / slots) & 1));
+            }
+            return;
+        }
+        const int64_t base = (gw + j * nw) * kChunk;
+        const int64_t left = n - base;
+        const int nv = (int)((left < kChunk ? left : kChunk) / E);
+        const unsigned char* sg = ring + (size_t)sidx * 2 * kBytes;
+#pragma unroll 4
+        for (int v = lane; v < nv; v += 32) {
+            float a[E], b[E];
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), a);
+            Vec<T>::unpack(*reinterpret_cast<const uint4*>(sg + kBytes + (size_t)v * 16), b);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                a[e] = silu<T>(a[e]) * b[e];
+            st_stream(out + base + (int64_t)v * E, Vec<T>::pack(a));
+        }
+        __syncwarp();  // the slot has been read; it can take the next copy
+        if (lane == 0 && issued < my) {
+            issue(issued);
+            ++issued;
+        }
+    }
+}
+
 // Unaligned buffers: one element per thread per iteration.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -102,9 +192,32 @@ cudaError_t launch_swiglu_t(const void* gv, const void* uv, void* ov, int64_t n,
     if (err != cudaSuccess)
         return err;
     constexpr int E = Vec<T>::N;
-    // 8 resident CTAs of 256 threads fill an SM's 2048 thread slots
-    const int64_t resident = (int64_t)di.sm_count * 8;
-    if (aligned16(g) && aligned16(u) && aligned16(o)) {
+    const bool aligned = aligned16(g) && aligned16(u) && aligned16(o);
+    if (aligned && n % E == 0 && streaming_enabled()) {
+        // 3 slots of 8 KB per warp: 96 KB per CTA, two CTAs per SM
+        const int slots = 3;
+        const uint32_t smem = kTmaWarps * slots * (2 * kChunk * sizeof(T) + 8) + 128;
+        auto kernel = swiglu_tma_kernel<T>;
+        int per_sm = 0;
+        err = resident_ctas(kernel, 32 * kTmaWarps, smem, &per_sm);
+        if (err != cudaSuccess)
+            return err;
+        unsigned* word = nullptr;
+        err = device_error_word(&word);
+        if (err != cudaSuccess)
+            return err;
+        const int64_t chunks = ceil_div(n, kChunk);
+        const int64_t grid = std::min<int64_t>(ceil_div(chunks, kTmaWarps),
+                                               (int64_t)di.sm_count * std::max(per_sm, 1));
+        return launch(kernel, dim3((unsigned)grid), dim3(32 * kTmaWarps), smem, st, g, u, o, n,
+                      slots, word);
+    }
+    int per_sm = 0;
+    err = resident_ctas(swiglu_vec_kernel<T, kUnroll>, kThreads, 0, &per_sm);
+    if (err != cudaSuccess)
+        return err;
+    const int64_t resident = (int64_t)di.sm_count * std::max(per_sm, 1);
+    if (aligned) {
         const int64_t nvec = n / E;
         const int64_t want = std::max<int64_t>(1, ceil_div(nvec, (int64_t)kThreads * kUnroll));
         const int64_t grid = std::min<int64_t>(want, resident);

@@ -1,0 +1,116 @@
+"""Per-operator timing on one GPU (CUDA events; inputs rotated through > 4x L2).
+
+    python -m swiglu_ar_tts_b200.opbench --op swiglu --iters 50
+    python -m swiglu_ar_tts_b200.opbench --op all
+
+Shapes are the operators' workload sizes (add+RMSNorm bf16 4096x2048, SwiGLU
+bf16 8192x6144, M-RoPE bf16 4096 tokens x 16/8 heads x 128, RMSNorm fp32
+64x1024, decode steps at batch 5 and 256); ``--rows`` scales the row count.
+Prints one line per operator: median and mean microseconds per launch and the
+algorithmic HBM GB/s (every operand read once, every output written once).
+
+Each operator gets enough copies of its buffers to cover 512 MB (4x the L2) and
+successive launches cycle through them, so every launch reads from DRAM and
+pays for the write-back of earlier launches, as it does in steady state.  With
+``--copies 1`` it is also the small driver used for ncu captures.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import statistics
+
+import torch
+
+from . import add_rmsnorm, mrope_qk, rmsnorm, set_pdl, set_streaming, swiglu
+from . import inputs as I
+from .chain import DecodeChain
+
+OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
+
+
+def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
+    """Returns (launch callable, algorithmic bytes, shape description) for one
+    copy of the operator's buffers."""
+    if op == "rmsnorm":
+        r = rows or 64
+        t = {k: v.to(dev) for k, v in I.rmsnorm_inputs(r, 1024, "f32", seed).items()}
+        y = torch.empty_like(t["x"])
+        return (lambda: rmsnorm(t["x"], t["gamma"], I.EPS, out=y)), (2 * r * 1024 + 1024) * 4, f"f32 {r}x1024"
+    if op == "add_rmsnorm":
+        r = rows or 4096
+        t = {k: v.to(dev) for k, v in I.add_rmsnorm_inputs(r, I.HIDDEN, "bf16", seed).items()}
+        y, ro = torch.empty_like(t["x"]), torch.empty_like(t["x"])
+        return ((lambda: add_rmsnorm(t["x"], t["residual"], t["gamma"], I.EPS, y=y, residual_out=ro)),
+                (4 * r * I.HIDDEN + I.HIDDEN) * 2, f"bf16 {r}x{I.HIDDEN}")
+    if op == "swiglu":
+        r = rows or 8192
+        t = {k: v.to(dev) for k, v in I.swiglu_inputs(r, I.INTER, "bf16", seed).items()}
+        o = torch.empty_like(t["gate"])
+        return (lambda: swiglu(t["gate"], t["up"], out=o)), 3 * r * I.INTER * 2, f"bf16 {r}x{I.INTER}"
+    if op == "mrope_qk":
+        r = rows or 4096
+        t = {k: v.to(dev) for k, v in I.mrope_inputs(r, seed=seed).items()}
+        qo, ko = torch.empty_like(t["q"]), torch.empty_like(t["k"])
+        nb = 2 * r * (I.N_Q_HEADS + I.N_K_HEADS) * I.HEAD_DIM * 2 + 3 * r * 4
+        return ((lambda: mrope_qk(t["q"], t["k"], t["pos"], I.SECTIONS, I.THETA, q_out=qo, k_out=ko)),
+                nb, f"bf16 {r} tokens")
+    if op in ("decode5", "decode256"):
+        b = rows or (5 if op == "decode5" else 256)
+        c = DecodeChain(I.ChainShape(batch=b), device=dev, seed=seed)
+        c.capture()
+        c.set_position(7)
+        return (lambda: c._graph.replay()), c.bytes_per_step(), f"28 layers, batch {b}, graph"
+    raise ValueError(op)
+
+
+def make_rotation(op: str, rows: int | None, dev: torch.device, copies: int | None):
+    fn, nbytes, desc = make(op, rows, dev)
+    n = copies if copies is not None else max(1, min(64, -(-(512 << 20) // nbytes)))
+    fns = [fn] + [make(op, rows, dev, seed=100 + i)[0] for i in range(n - 1)]
+    return fns, nbytes, f"{desc}, {n} copies"
+
+
+def time_op(fns, iters: int) -> list[float]:
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    torch.cuda._sleep(int(1e7))  # let the host queue ahead of the device
+    for i, (a, b) in enumerate(ev):
+        a.record()
+        fns[i % len(fns)]()
+        b.record()
+    torch.cuda.synchronize()
+    return [1e3 * a.elapsed_time(b) for a, b in ev]
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", default="all", choices=("all",) + OPS)
+    ap.add_argument("--iters", type=int, default=50)
+    ap.add_argument("--rows", type=int, default=None)
+    ap.add_argument("--copies", type=int, default=None,
+                    help="buffer copies to rotate through (default: enough for 512 MB)")
+    ap.add_argument("--pdl", action="store_true")
+    ap.add_argument("--registers", action="store_true", help="register kernels instead of streaming")
+    ap.add_argument("--json", action="store_true")
+    a = ap.parse_args()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    set_pdl(a.pdl)
+    set_streaming(not a.registers)
+    for op in (OPS if a.op == "all" else (a.op,)):
+        fns, nbytes, desc = make_rotation(op, a.rows, dev, a.copies)
+        us = time_op(fns, a.iters)
+        med = statistics.median(us)
+        rec = {"op": op, "shape": desc, "bytes": nbytes, "us_median": round(med, 3),
+               "us_mean": round(statistics.fmean(us), 3), "us_min": round(min(us), 3),
+               "gbs_median": round(nbytes / (med * 1e-6) / 1e9, 1)}
+        print(json.dumps(rec) if a.json else
+              f"{op:12s} {desc:40s} median {med:9.3f} us  min {min(us):9.3f} us  "
+              f"{rec['gbs_median']:8.1f} GB/s", flush=True)
+
+
+if __name__ == "__main__":
+    main()

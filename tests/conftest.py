@@ -9,3 +9,33 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(params=["streaming", "registers"])
+def family(request):
+    """Runs a test once with the shared-memory streaming kernels and once with
+    the register kernels (the library's two kernel families)."""
+    import swiglu_ar_tts_b200 as ops
+
+    old = ops.set_streaming(request.param == "streaming")
+    yield request.param
+    ops.set_streaming(old)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors(request):
+    """Every GPU test must leave the library's device error word at 0 (no
+    bounded wait in any kernel ran out)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+
+    import swiglu_ar_tts_b200 as ops
+
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+        assert ops.device_errors(clear=True) == 0

@@ -39,7 +39,7 @@ def _run(inp, sections=SECTIONS, theta=THETA, in_place=False):
 
 
 @pytest.mark.parametrize("in_place", [False, True])
-def test_mrope_4096_tokens(in_place):
+def test_mrope_4096_tokens(in_place, family):
     """The M-RoPE workload: q [4096 x 16 x 128], k [4096 x 8 x 128], theta 1e6,
     sections [24, 20, 20]; 1024 text tokens then a 48 x 8 x 8 t/h/w grid."""
     inp = inputs.mrope_inputs(4096)
@@ -58,7 +58,7 @@ def test_mrope_positions_layout():
     assert int(pos[1, 1024 + 8]) == 1 and int(pos[2, 1024 + 9]) == 1
 
 
-def test_mrope_section_masks_bit_exact():
+def test_mrope_section_masks_bit_exact(family):
     """Only one of t/h/w nonzero: pairs outside that row's section are returned
     bit for bit; pairs inside move."""
     inp = inputs.mrope_inputs(3, seed=40)
@@ -77,7 +77,7 @@ def test_mrope_section_masks_bit_exact():
         _compare(qo, ko, {"q": inp["q"], "k": inp["k"], "pos": pos}, what=f"mask row {row}")
 
 
-def test_mrope_equal_rows_is_1d_rope_and_large_positions():
+def test_mrope_equal_rows_is_1d_rope_and_large_positions(family):
     inp = inputs.mrope_inputs(64, seed=41)
     p = torch.tensor([0, 1, 2, 3, 1000, 1071, 4095, 65535, 1 << 20, (1 << 31) - 1, -5, -1000] + list(range(52)),
                      dtype=torch.int32)
@@ -92,14 +92,14 @@ def test_mrope_equal_rows_is_1d_rope_and_large_positions():
     (16, (4, 2, 2)), (32, (8, 4, 4)), (512, (128, 64, 64)), (96, (16, 16, 16)), (2, (1, 0, 0)),
     (10, (2, 2, 1)),
 ])
-def test_mrope_head_dims(dtype, head_dim, sections):
+def test_mrope_head_dims(dtype, head_dim, sections, family):
     inp = inputs.mrope_inputs(37, n_q_heads=5, n_k_heads=3, head_dim=head_dim, dtype=dtype, seed=head_dim)
     qo, ko = _run(inp, sections=sections)
     _compare(qo, ko, inp, sections=sections, dtype=dtype, what=f"D={head_dim} {dtype}")
 
 
 @pytest.mark.parametrize("hq,hk", [(16, 0), (0, 8), (1, 1), (7, 5), (32, 4), (40, 40)])
-def test_mrope_head_counts(hq, hk):
+def test_mrope_head_counts(hq, hk, family):
     inp = inputs.mrope_inputs(19, n_q_heads=hq, n_k_heads=hk, seed=hq * 10 + hk)
     q, k, pos = dev(inp["q"]), dev(inp["k"]), dev(inp["pos"])
     qo, ko = torch.empty_like(q), torch.empty_like(k)
@@ -128,7 +128,7 @@ def test_mrope_misaligned_and_guarded():
     _compare(qo.t, ko.t, inp, what="misaligned")
 
 
-def test_mrope_guarded_vector_path():
+def test_mrope_guarded_vector_path(family):
     inp = inputs.mrope_inputs(33, seed=44)
     qo = Guarded(tuple(inp["q"].shape), torch.bfloat16)
     ko = Guarded(tuple(inp["k"].shape), torch.bfloat16)

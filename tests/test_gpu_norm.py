@@ -23,7 +23,7 @@ def _run_rmsnorm(rows, hidden, dtype, seed=0, eps=EPS):
     return y, exact
 
 
-def test_rmsnorm_f32_64x1024():
+def test_rmsnorm_f32_64x1024(family):
     """The fp32 workload: 64 rows x 1024, gamma = 1 + 0.1 N(0,1), eps 1e-6."""
     y, exact = _run_rmsnorm(64, 1024, "f32")
     st = check(y, exact, "f32", what="rmsnorm f32 64x1024")
@@ -38,14 +38,14 @@ HIDDEN = [8, 16, 24, 40, 256, 512, 1000, 1024, 2048, 4104, 8192, 16384, 32768, 4
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("hidden", HIDDEN)
-def test_rmsnorm_shapes(dtype, hidden):
+def test_rmsnorm_shapes(dtype, hidden, family):
     rows = 37 if hidden <= 16384 else 5
     y, exact = _run_rmsnorm(rows, hidden, dtype, seed=hidden)
     check(y, exact, dtype, what=f"rmsnorm {dtype} {rows}x{hidden}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_rmsnorm_large_bf16_prefill(dtype):
+def test_rmsnorm_large_bf16_prefill(dtype, family):
     y, exact = _run_rmsnorm(4096, 2048, dtype, seed=3)
     check(y, exact, dtype, what="rmsnorm 4096x2048")
 
@@ -80,7 +80,7 @@ def test_rmsnorm_misaligned(dtype):
 
 
 @pytest.mark.parametrize("hidden", [2048, 100, 40000])
-def test_rmsnorm_guard_bands(hidden):
+def test_rmsnorm_guard_bands(hidden, family):
     inp = inputs.rmsnorm_inputs(7, hidden, "bf16", 12)
     out = Guarded((7, hidden), torch.bfloat16)
     ops.rmsnorm(dev(inp["x"]), dev(inp["gamma"]), EPS, out=out.t)
@@ -111,7 +111,7 @@ def _run_add(rows, hidden, dtype, seed=0, in_place=False, eps=EPS):
 
 
 @pytest.mark.parametrize("in_place", [False, True])
-def test_add_rmsnorm_bf16_4096x2048(in_place):
+def test_add_rmsnorm_bf16_4096x2048(in_place, family):
     """The fused add+norm workload: x ~ N(0,1), residual ~ N(0,2^2), [4096 x 2048]."""
     y, r_out, y_exact, r_exact = _run_add(4096, 2048, "bf16", in_place=in_place)
     assert np.array_equal(to_f64(r_out), r_exact), "residual_out must be bit-exact"
@@ -120,14 +120,14 @@ def test_add_rmsnorm_bf16_4096x2048(in_place):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("hidden", HIDDEN)
-def test_add_rmsnorm_shapes(dtype, hidden):
+def test_add_rmsnorm_shapes(dtype, hidden, family):
     rows = 21 if hidden <= 16384 else 3
     y, r_out, y_exact, r_exact = _run_add(rows, hidden, dtype, seed=hidden + 1)
     assert np.array_equal(to_f64(r_out), r_exact)
     check(y, y_exact, dtype, what=f"add_rmsnorm {dtype} {rows}x{hidden}")
 
 
-def test_add_rmsnorm_is_add_then_norm_on_gpu():
+def test_add_rmsnorm_is_add_then_norm_on_gpu(family):
     """The fused kernel equals the add written back, then RMSNorm of it, both on
     the GPU (bit for bit: the norm sees exactly the written residual)."""
     inp = inputs.add_rmsnorm_inputs(64, 2048, "bf16", 21)
@@ -138,7 +138,7 @@ def test_add_rmsnorm_is_add_then_norm_on_gpu():
     assert torch.equal(y, y2)
 
 
-def test_add_rmsnorm_misaligned_and_guarded():
+def test_add_rmsnorm_misaligned_and_guarded(family):
     inp = inputs.add_rmsnorm_inputs(5, 2048, "bf16", 22)
     x = misaligned(dev(inp["x"]))
     r = misaligned(dev(inp["residual"]))

@@ -19,7 +19,7 @@ def _run(rows, inter, dtype, seed=0):
     return out, oracle.get().swiglu(inp["gate"], inp["up"])
 
 
-def test_swiglu_bf16_8192x6144():
+def test_swiglu_bf16_8192x6144(family):
     """The SwiGLU workload: gate ~ N(0, 2^2), up ~ N(0,1), separate [8192 x 6144]."""
     out, exact = _run(8192, 6144, "bf16")
     st = check(out, exact, "bf16", what="swiglu 8192x6144")
@@ -29,12 +29,12 @@ def test_swiglu_bf16_8192x6144():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("shape", [(1, 8), (1, 1), (3, 13), (5, 6144), (7, 1001), (64, 6144),
                                    (1, 8 * 256 * 4 + 5), (300, 4097)])
-def test_swiglu_shapes(dtype, shape):
+def test_swiglu_shapes(dtype, shape, family):
     out, exact = _run(*shape, dtype, seed=shape[0] * 7 + shape[1])
     check(out, exact, dtype, what=f"swiglu {dtype} {shape}")
 
 
-def test_swiglu_special_values():
+def test_swiglu_special_values(family):
     """g = +-0 gives +-0 exactly; large |g| tends to g*u or to 0."""
     g = torch.tensor([0.0, -0.0, 1.0, -1.0, 2.0, 20.0, -20.0, 80.0, -80.0, -100.0, 88.0, -88.0,
                       1e-30, -1e-30, 3.0, -3.0], dtype=torch.float32)
@@ -50,7 +50,7 @@ def test_swiglu_special_values():
         check(out, exact, "bf16" if dt == torch.bfloat16 else "f32", what=f"special {dt}")
 
 
-def test_swiglu_in_place_and_guarded():
+def test_swiglu_in_place_and_guarded(family):
     inp = inputs.swiglu_inputs(9, 777, "bf16", 5)
     gate = dev(inp["gate"])
     out = Guarded((9, 777), torch.bfloat16, fill=gate)

@@ -192,14 +192,10 @@ class Step:
         self.mr = {k: v.to(d) for k, v in h["mrope_qk"].items()}
         self.mr["q_out"] = torch.empty_like(self.mr["q"])
         self.mr["k_out"] = torch.empty_like(self.mr["k"])
-        old = ops.set_pdl(pdl)
-        try:
-            self.chain5 = DecodeChain(inputs.ChainShape(batch=5), device=d)
-            self.chain256 = DecodeChain(inputs.ChainShape(batch=256), device=d, seed=1000)
-            self.chain5.capture()
-            self.chain256.capture()
-        finally:
-            ops.set_pdl(old)
+        self.chain5 = DecodeChain(inputs.ChainShape(batch=5), device=d, pdl=pdl)
+        self.chain256 = DecodeChain(inputs.ChainShape(batch=256), device=d, seed=1000, pdl=pdl)
+        self.chain5.capture()
+        self.chain256.capture()
         self.decode_step_index = 0
         self.bytes = {
             "rmsnorm": (2 * 64 * 1024 + 1024) * 4,

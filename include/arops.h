@@ -146,11 +146,15 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
 AROPS_API int arops_set_pdl(int enable);
 
 /*
- * Kernel family selection (process-wide).  Enabled (the default), 16-byte
- * aligned rows are processed by the streaming kernels, which stage rows through
- * shared memory with bulk asynchronous copies; disabled, by the register
- * kernels.  Both compute the same results; the switch exists so that both can
- * be tested and measured.  Returns the old setting.
+ * Kernel family selection (process-wide).  Disabled (the default), every
+ * operator runs its register kernel: 16-byte coalesced loads straight into
+ * registers.  Enabled, 16-byte-aligned rows go to the streaming kernels, which
+ * stage data through shared memory with bulk asynchronous copies (TMA) under
+ * time-bounded mbarrier waits.  Both families compute the same results within
+ * the stated tolerance (the norm kernels may differ in the last bit, as their
+ * sums of squares are accumulated in a different order); on B200 the register
+ * kernels measured as fast or faster for every operator, so streaming is kept
+ * as an option for measurement.  Returns the old setting.
  */
 AROPS_API int arops_set_streaming(int enable);
 

@@ -207,8 +207,8 @@ def set_pdl(enable: bool) -> bool:
 
 
 def set_streaming(enable: bool) -> bool:
-    """Choose the shared-memory streaming kernels (default) or the register
-    kernels; returns the old setting.  Both give the same results."""
+    """Choose the shared-memory streaming kernels or the register kernels (the
+    default); returns the old setting.  Both give results within tolerance."""
     return bool(lib().arops_set_streaming(1 if enable else 0))
 
 

@@ -16,7 +16,10 @@ only state carried from layer to layer and from step to step.
 
 ``DecodeChain`` owns the device buffers and launches each operator through the
 C ABI with pre-bound arguments (no per-call tensor checks), either eagerly on
-the current stream or replayed from a CUDA graph of one step.
+the current stream or replayed from a CUDA graph of one step.  By default the
+launches use programmatic dependent launch: each kernel is scheduled while its
+predecessor drains and prefetches its first inputs into L2 before waiting for
+it, which removes most of the per-launch gap of a 112-kernel step.
 """
 from __future__ import annotations
 
@@ -31,12 +34,13 @@ from .inputs import EPS, SECTIONS, THETA, ChainShape, decode_chain_inputs
 class DecodeChain:
     def __init__(self, shape: ChainShape, dtype: str = "bf16", seed: int = 0,
                  device: str | torch.device = "cuda", eps: float = EPS, theta: float = THETA,
-                 sections=SECTIONS, host_inputs: dict | None = None):
+                 sections=SECTIONS, host_inputs: dict | None = None, pdl: bool = True):
         self.shape = shape
         self.dtype = dtype
         self.eps = eps
         self.theta = theta
         self.sections = tuple(int(s) for s in sections)
+        self.pdl = pdl
         self.device = torch.device(device)
         host = host_inputs if host_inputs is not None else decode_chain_inputs(shape, dtype, seed)
         self.host_inputs = host
@@ -108,12 +112,16 @@ class DecodeChain:
         """Enqueue the 4 * layers operator launches of one step (positions as set)."""
         if stream is None:
             stream = torch.cuda.current_stream(self.device).cuda_stream
-        for fn, args in self._calls:
-            st = fn(*args, stream)
-            if st != 0:
-                L = lib()
-                raise ArOpsError(st, f"{L.arops_status_string(st).decode()}: "
-                                     f"{L.arops_last_error().decode()}")
+        L = lib()
+        old = L.arops_set_pdl(1 if self.pdl else 0)
+        try:
+            for fn, args in self._calls:
+                st = fn(*args, stream)
+                if st != 0:
+                    raise ArOpsError(st, f"{L.arops_status_string(st).decode()}: "
+                                         f"{L.arops_last_error().decode()}")
+        finally:
+            L.arops_set_pdl(old)
 
     def step(self, step: int) -> None:
         self.set_position(step)

@@ -14,7 +14,7 @@ namespace {
 
 thread_local char g_last_error[512] = "";
 std::atomic<int> g_pdl{0};
-std::atomic<int> g_streaming{1};
+std::atomic<int> g_streaming{0};
 std::atomic<uint64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;

@@ -28,6 +28,22 @@ __device__ __forceinline__ void pdl_allow_dependents()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Hint to bring [p, p + bytes) into L2 (one bulk prefetch; p and bytes must be
+// multiples of 16).  Issued before pdl_wait() to overlap a kernel's first DRAM
+// reads with its predecessor: L2 is the point of coherence for global memory,
+// so a prefetch can never make a later load see stale data.  (No L1 prefetch is
+// ever issued before the wait, since L1 is not coherent.)
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Hint to bring the 128-byte line holding p into L2 (any alignment).
+__device__ __forceinline__ void prefetch_l2_line(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte vectors of the storage type, unpacked to / packed from fp32.
 // ---------------------------------------------------------------------------

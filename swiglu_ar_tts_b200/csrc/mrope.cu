@@ -24,13 +24,27 @@
 namespace arops {
 namespace {
 
-constexpr int kMaxHalf = 256;  // head_dim <= 512
-
 struct MropeParams {
-    int32_t sec0;   // pairs j < sec0 take row 0 (t)
-    int32_t sec01;  // pairs sec0 <= j < sec01 take row 1 (h); the rest row 2 (w)
-    double inv_freq[kMaxHalf];  // theta^(-2j/head_dim), j < head_dim/2
+    int32_t sec0;       // pairs j < sec0 take row 0 (t)
+    int32_t sec01;      // pairs sec0 <= j < sec01 take row 1 (h); the rest row 2 (w)
+    double freq_scale;  // 2 log2(theta) / head_dim: inverse frequency j is 2^(-j * freq_scale)
 };
+
+// theta^(-2j/head_dim) = 2^(-j * 2 log2(theta) / head_dim), the textbook RoPE
+// inverse frequency, in fp64.
+__device__ __forceinline__ double inv_freq_of(int j, const MropeParams& prm)
+{
+    return exp2(-(double)j * prm.freq_scale);
+}
+
+// Each CTA tabulates the head's inverse frequencies in shared memory once; this
+// touches no global memory, so it runs before the dependency wait.
+__device__ __forceinline__ void fill_inv_freq(double* table, int half, const MropeParams& prm)
+{
+    for (int j = threadIdx.x; j < half; j += blockDim.x)
+        table[j] = inv_freq_of(j, prm);
+    __syncthreads();
+}
 
 constexpr double kTwoPi = 6.283185307179586;
 constexpr double kInvTwoPi = 0.15915494309189535;
@@ -66,7 +80,23 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     const int hg = lane / P;
     const int j0 = pv * E;
     const int nh = hq + hk;
+    __shared__ double inv_freq[HALF];
 
+    // this warp's first token (q and k heads, positions) into L2 while the
+    // previous kernel drains
+    {
+        const int64_t t0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+        if (lane == 0 && t0 < tokens) {
+            if (hq > 0)
+                prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
+            if (hk > 0)
+                prefetch_l2(k + (size_t)t0 * hk * D, (uint32_t)(hk * D * sizeof(T)));
+            prefetch_l2_line(pos + t0);
+            prefetch_l2_line(pos + tokens + t0);
+            prefetch_l2_line(pos + 2 * tokens + t0);
+        }
+    }
+    fill_inv_freq(inv_freq, HALF, prm);
     pdl_wait();
     pdl_allow_dependents();
 
@@ -98,7 +128,7 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
 #pragma unroll
         for (int f = 0; f < F; ++f) {
             const int j = j0 + ((hg * F + f) % E);
-            rope_cos_sin(prm.inv_freq[j], position_of(j, prm, pt, ph, pw), &cs[f], &sn[f]);
+            rope_cos_sin(inv_freq[j], position_of(j, prm, pt, ph, pw), &cs[f], &sn[f]);
         }
         // ... gathered from the lanes that evaluated them
         float c[E], s[E];
@@ -173,13 +203,14 @@ mrope_tma_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     const int64_t gw = (int64_t)blockIdx.x * kTmaWarps + warp;
     const int64_t nw = (int64_t)gridDim.x * kTmaWarps;
     const int64_t my = tokens > gw ? (tokens - 1 - gw) / nw + 1 : 0;
+    __shared__ double inv_freq[HALF];
 
     if (lane == 0) {
         for (int i = 0; i < slots; ++i)
             mbar_init(smem_addr(&bars[i]), 1);
         mbar_init_fence();
     }
-    __syncwarp();
+    fill_inv_freq(inv_freq, HALF, prm);
 
     pdl_wait();
     pdl_allow_dependents();
@@ -218,7 +249,7 @@ mrope_tma_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
 #pragma unroll
         for (int f = 0; f < F; ++f) {
             const int jj = j0 + ((hg * F + f) % E);
-            rope_cos_sin(prm.inv_freq[jj], position_of(jj, prm, pt, ph, pw), &cs[f], &sn[f]);
+            rope_cos_sin(inv_freq[jj], position_of(jj, prm, pt, ph, pw), &cs[f], &sn[f]);
         }
         float c[E], s[E];
 #pragma unroll
@@ -281,7 +312,7 @@ mrope_scalar_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* _
         const int32_t p = position_of(j, prm, __ldg(pos + t), __ldg(pos + tokens + t),
                                       __ldg(pos + 2 * tokens + t));
         float c, s;
-        rope_cos_sin(prm.inv_freq[j], p, &c, &s);
+        rope_cos_sin(inv_freq_of(j, prm), p, &c, &s);
         const size_t off = (h < hq) ? ((size_t)t * hq + h) * 2 * half
                                     : ((size_t)t * hk + (h - hq)) * 2 * half;
         const T* src = (h < hq) ? q : k;
@@ -295,14 +326,30 @@ mrope_scalar_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* _
 
 constexpr int kHeadUnroll = 8;
 
+template <typename T, int P, int U>
+cudaError_t launch_vec_u(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens, kWarpsPerCta), cap);
+    return launch(mrope_vec_kernel<T, P, U>, dim3((unsigned)grid), dim3(32 * kWarpsPerCta), 0, st,
+                  static_cast<const T*>(a.q), static_cast<const T*>(a.k),
+                  static_cast<T*>(a.q_out), static_cast<T*>(a.k_out), a.pos, a.tokens,
+                  (int)a.n_q_heads, (int)a.n_k_heads, prm);
+}
+
+// Heads per lane per pass: just enough passes to cover every head at once (6
+// for 16 + 8 heads of 128), so no registers are held for absent heads.
 template <typename T, int P>
 cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
 {
-    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens, kWarpsPerCta), cap);
-    return launch(mrope_vec_kernel<T, P, kHeadUnroll>, dim3((unsigned)grid),
-                  dim3(32 * kWarpsPerCta), 0, st, static_cast<const T*>(a.q),
-                  static_cast<const T*>(a.k), static_cast<T*>(a.q_out), static_cast<T*>(a.k_out),
-                  a.pos, a.tokens, (int)a.n_q_heads, (int)a.n_k_heads, prm);
+    constexpr int G = 32 / P;
+    const int passes = (int)ceil_div(a.n_q_heads + a.n_k_heads, G);
+    if (passes <= 2)
+        return launch_vec_u<T, P, 2>(a, prm, st, cap);
+    if (passes <= 4)
+        return launch_vec_u<T, P, 4>(a, prm, st, cap);
+    if (passes <= 6)
+        return launch_vec_u<T, P, 6>(a, prm, st, cap);
+    return launch_vec_u<T, P, kHeadUnroll>(a, prm, st, cap);
 }
 
 // Streaming launch; cudaErrorNotSupported when two slots per warp do not fit.
@@ -393,13 +440,9 @@ cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStrea
 cudaError_t launch_mrope(const MropeArgs& a, arops_dtype dtype, cudaStream_t stream)
 {
     MropeParams prm;
-    const int half = a.head_dim / 2;
     prm.sec0 = a.sections[0];
     prm.sec01 = a.sections[0] + a.sections[1];
-    // textbook RoPE inverse frequencies, formed in fp64 on the host
-    for (int j = 0; j < kMaxHalf; ++j)
-        prm.inv_freq[j] = (j < half) ? pow((double)a.theta, -2.0 * (double)j / (double)a.head_dim)
-                                     : 0.0;
+    prm.freq_scale = 2.0 * log2((double)a.theta) / (double)a.head_dim;
     if (dtype == AROPS_BF16)
         return launch_mrope_t<__nv_bfloat16>(a, prm, stream);
     return launch_mrope_t<float>(a, prm, stream);

@@ -13,8 +13,9 @@
 // residual_out, y) with fully coalesced 128-bit accesses.  The sum of squares is
 // accumulated in fp32, reduced with warp shuffles and, for GW > 1 warps per row,
 // one shared-memory step.  rsqrtf of (sum / hidden + eps) scales the row; the
-// product x * r * gamma is rounded once to the storage type.  gamma is re-read
-// per row through the read-only path, where it stays L1/L2 resident.
+// product x * r * gamma is rounded once to the storage type.  gamma is read
+// through the read-only path together with each row (it stays L1/L2 resident),
+// so a row costs one memory round trip, which matters most for decode batches.
 //
 // Rows longer than 4096 vectors, and unaligned or ragged rows, take a looped
 // kernel that makes a second pass over the row (served from L2).
@@ -170,6 +171,18 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
     const int group = (GW == 1) ? (tid >> 5) : 0;
     __shared__ float red[2][GW];
 
+    // this group's first row and gamma into L2 while the previous kernel drains
+    {
+        const int64_t row0 = (int64_t)blockIdx.x * ROWS_PER_CTA + group;
+        const uint32_t row_bytes = (uint32_t)hidden * sizeof(T);
+        if (gt == 0 && row0 < rows) {
+            prefetch_l2(x + (size_t)row0 * hidden, row_bytes);
+            if constexpr (ADD)
+                prefetch_l2(residual_in + (size_t)row0 * hidden, row_bytes);
+        }
+        if (tid == 0 && blockIdx.x < 64)  // later CTAs find gamma in L2 already
+            prefetch_l2(gamma, row_bytes);
+    }
     pdl_wait();
     pdl_allow_dependents();
 
@@ -177,8 +190,16 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
     for (int64_t row = (int64_t)blockIdx.x * ROWS_PER_CTA + group; row < rows;
          row += (int64_t)gridDim.x * ROWS_PER_CTA) {
         const size_t base = (size_t)row * (size_t)hidden;
-        uint4 v[VPL];
+        uint4 v[VPL], gv[VPL];
         float ss = 0.f;
+        // gamma is loaded with the row, not after the reduction: a load issued
+        // after the shuffles would add a dependent round trip to every row
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int vi = gt + i * G;
+            if (vi < nvec)
+                gv[i] = __ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E));
+        }
         if constexpr (ADD) {
             uint4 r[VPL];
 #pragma unroll
@@ -250,7 +271,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
             if (vi < nvec) {
                 float a[E], g[E];
                 Vec<T>::unpack(v[i], a);
-                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E)), g);
+                Vec<T>::unpack(gv[i], g);
 #pragma unroll
                 for (int e = 0; e < E; ++e)
                     a[e] = a[e] * r * g[e];

@@ -29,6 +29,9 @@ from .chain import DecodeChain
 OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
 
 
+CHAIN_PDL = True
+
+
 def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
     """Returns (launch callable, algorithmic bytes, shape description) for one
     copy of the operator's buffers."""
@@ -57,7 +60,7 @@ def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
                 nb, f"bf16 {r} tokens")
     if op in ("decode5", "decode256"):
         b = rows or (5 if op == "decode5" else 256)
-        c = DecodeChain(I.ChainShape(batch=b), device=dev, seed=seed)
+        c = DecodeChain(I.ChainShape(batch=b), device=dev, seed=seed, pdl=CHAIN_PDL)
         c.capture()
         c.set_position(7)
         return (lambda: c._graph.replay()), c.bytes_per_step(), f"28 layers, batch {b}, graph"
@@ -94,12 +97,17 @@ def main() -> None:
     ap.add_argument("--copies", type=int, default=None,
                     help="buffer copies to rotate through (default: enough for 512 MB)")
     ap.add_argument("--pdl", action="store_true")
-    ap.add_argument("--registers", action="store_true", help="register kernels instead of streaming")
+    ap.add_argument("--streaming", action="store_true",
+                    help="shared-memory streaming kernels instead of the default register kernels")
+    ap.add_argument("--no-chain-pdl", action="store_true",
+                    help="decode steps without programmatic dependent launch")
     ap.add_argument("--json", action="store_true")
     a = ap.parse_args()
     dev = torch.device("cuda", torch.cuda.current_device())
+    global CHAIN_PDL
+    CHAIN_PDL = not a.no_chain_pdl
     set_pdl(a.pdl)
-    set_streaming(not a.registers)
+    set_streaming(a.streaming)
     for op in (OPS if a.op == "all" else (a.op,)):
         fns, nbytes, desc = make_rotation(op, a.rows, dev, a.copies)
         us = time_op(fns, a.iters)

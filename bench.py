@@ -13,8 +13,11 @@ synthetic input:
 ``value`` is the step's algorithmic HBM bytes (every operand read once, every
 output written once) divided by its device time, in GB/s, summed over ranks.
 The JSON line also gives per-operator times and GB/s, microseconds per decode
-step, the roofline of the dominant kernel (SwiGLU), an end-to-end figure with
-host buffers, and the oracle timed on the host cores.
+step, the time, share and GB/s of each kernel type (the decode graphs are split
+across their kernels by timing each operator's launches as a graph of its
+own), the roofline of the dominant kernel and of the largest single launch
+(SwiGLU), an end-to-end figure with host buffers, and the oracle timed on the
+host cores.
 
 L2: the step touches ~1 GB of distinct data, 8x the 126 MB L2, and no operator
 reuses data of another, so every operator's inputs were last touched hundreds
@@ -312,6 +315,65 @@ class Step:
 
 
 # ---------------------------------------------------------------------------
+# attribution of the decode graphs to kernel types
+# ---------------------------------------------------------------------------
+KERNEL_OF = {"add_rmsnorm": "norm_rows_kernel", "rmsnorm": "norm_rows_kernel",
+             "mrope_qk": "mrope_vec_kernel", "swiglu": "swiglu_vec_kernel"}
+
+
+def decode_split(chain, reps: int = 10) -> dict:
+    """Fraction of a decode step spent in each operator's kernels.
+
+    The step's launches are grouped by operator (56 add+RMSNorm, 28 M-RoPE, 28
+    SwiGLU for 28 layers); each group is captured as a graph of its own and
+    timed, and the step's measured time is split in proportion.  Returns
+    {op: (fraction, launches, algorithmic bytes)}."""
+    import ctypes  # noqa: F401
+
+    from swiglu_ar_tts_b200 import lib
+
+    L = lib()
+    names = {L.arops_add_rmsnorm: "add_rmsnorm", L.arops_mrope_qk: "mrope_qk",
+             L.arops_swiglu: "swiglu"}
+    groups: dict[str, list] = {}
+    for fn, a in chain._calls:
+        key = next(v for k, v in names.items() if k is fn or k.__name__ == fn.__name__)
+        groups.setdefault(key, []).append((fn, a))
+    sh = chain.shape
+    e = chain.residual.element_size()
+    per_launch_bytes = {
+        "add_rmsnorm": (4 * sh.batch * sh.hidden + sh.hidden) * e,
+        "mrope_qk": 2 * sh.batch * (sh.n_q_heads + sh.n_k_heads) * sh.head_dim * e + 3 * sh.batch * 4,
+        "swiglu": 3 * sh.batch * sh.inter * e,
+    }
+    saved = chain.residual.clone()
+    times = {}
+    old = L.arops_set_pdl(1 if chain.pdl else 0)
+    try:
+        for key, calls in groups.items():
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                st = torch.cuda.current_stream().cuda_stream
+                for fn, a in calls:
+                    fn(*a, st)
+            for _ in range(2):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times[key] = e0.elapsed_time(e1) / reps
+            del g
+    finally:
+        L.arops_set_pdl(old)
+    chain.residual.copy_(saved)
+    total = sum(times.values())
+    return {k: (times[k] / total, len(groups[k]), len(groups[k]) * per_launch_bytes[k]) for k in times}
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timings
 # ---------------------------------------------------------------------------
 def oracle_step(fraction: int = 1, decode_b256_rows: int | None = None) -> tuple[float, int, str]:
@@ -487,14 +549,43 @@ def main() -> None:
         gbs = step.bytes[name] / (us * 1e-6) / 1e9
         ops_report[name] = {"us": round(us, 3), "bytes": step.bytes[name], "gbs": round(gbs, 1),
                             "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4)}
-    sw_us = 1e3 * per_op_ms[Step.OPS.index("swiglu")]
+    # time per kernel type in the step: prefill operators are timed directly;
+    # each decode graph is split across its operators' kernels (decode_split)
+    kernels: dict[str, dict] = {}
+
+    def add_time(kernel, us, launches, nbytes):
+        k = kernels.setdefault(kernel, {"us": 0.0, "launches": 0, "bytes": 0})
+        k["us"] += us
+        k["launches"] += launches
+        k["bytes"] += nbytes
+
+    for name in ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk"):
+        add_time(KERNEL_OF[name], ops_report[name]["us"], 1, step.bytes[name])
+    for name, chain in (("decode_b5", step.chain5), ("decode_b256", step.chain256)):
+        for op, (frac, launches, nbytes) in decode_split(chain).items():
+            add_time(KERNEL_OF[op], frac * ops_report[name]["us"], launches, nbytes)
+    step_us = 1e3 * ms_per_step
+    for k in kernels.values():
+        k["share"] = round(k["us"] / step_us, 4)
+        k["gbs"] = round(k["bytes"] / (k["us"] * 1e-6) / 1e9, 1)
+        k["us"] = round(k["us"], 2)
+    dominant = max(kernels, key=lambda k: kernels[k]["us"])
+    dk = kernels[dominant]
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": dk["gbs"], "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dk["gbs"] / peak, 4),
+                "traffic": None, "launches_per_step": dk["launches"],
+                "algorithmic_bytes_per_step": dk["bytes"],
+                "note": "dominant by share of step time; its launches span prefill and decode "
+                        "sizes, so no single ncu capture gives their DRAM traffic"}
+    sw_us = ops_report["swiglu"]["us"]
     sw_gbs = step.bytes["swiglu"] / (sw_us * 1e-6) / 1e9
-    traffic = ncu_traffic("swiglu_vec_kernel", ("swiglu_ar_tts_b200/csrc/swiglu.cu",
-                                                "swiglu_ar_tts_b200/csrc/common.cuh"))
-    roofline = {"kernel": "swiglu_vec_kernel<bf16> (8192x6144)", "bound": "hbm",
-                "achieved": round(sw_gbs, 1), "peak": peak, "peak_kind": peak_kind,
-                "unit": "GB/s", "frac": round(sw_gbs / peak, 4), "traffic": traffic,
-                "algorithmic_bytes": step.bytes["swiglu"]}
+    roofline_swiglu = {"kernel": "swiglu_vec_kernel<bf16> 8192x6144 (largest single launch)",
+                       "bound": "hbm", "achieved": round(sw_gbs, 1), "peak": peak,
+                       "peak_kind": peak_kind, "unit": "GB/s", "frac": round(sw_gbs / peak, 4),
+                       "traffic": ncu_traffic("swiglu_vec_kernel",
+                                              ("swiglu_ar_tts_b200/csrc/swiglu.cu",
+                                               "swiglu_ar_tts_b200/csrc/common.cuh")),
+                       "algorithmic_bytes": step.bytes["swiglu"]}
 
     # end to end: pinned host buffers in and out, through the same public calls
     step.setup_e2e()
@@ -547,6 +638,8 @@ def main() -> None:
                                "batch256": ops_report["decode_b256"]["us"]},
         "ops": ops_report,
         "roofline": roofline,
+        "roofline_swiglu": roofline_swiglu,
+        "kernels": kernels,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": eager_launches + args.steps * (step.kernels_per_step - 4),

@@ -314,6 +314,22 @@ class Step:
             dst.copy_(src, **nb)
 
 
+def reduce_max(x: float, pg=None, device=None) -> float:
+    """Max of ``x`` over the ranks of process group ``pg`` (identity without one).
+    Used for every time in a multi-GPU run, so ranks agree on the slowest."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, step_bytes: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job GB/s: every rank processed ``step_bytes`` per step (replicas),
+    over the slowest rank's device time."""
+    return world * step_bytes * steps / (total_ms_max * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------------------
 # attribution of the decode graphs to kernel types
 # ---------------------------------------------------------------------------
@@ -495,11 +511,7 @@ def main() -> None:
             pg.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, pg, device)
 
     import swiglu_ar_tts_b200 as ops
 
@@ -540,7 +552,7 @@ def main() -> None:
     total_ms = max_over_ranks(float(sum(step_ms)))
     ms_per_step = total_ms / args.steps
     step_bytes = sum(step.bytes[o] for o in Step.OPS)
-    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    value = aggregate_value(world, step_bytes, args.steps, total_ms)
 
     peak, peak_kind = measured_hbm_peak()
     ops_report = {}

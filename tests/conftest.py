@@ -39,3 +39,15 @@ def _no_device_errors(request):
     if torch.cuda.is_available():
         torch.cuda.synchronize()
         assert ops.device_errors(clear=True) == 0
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Compile libarops.so (nvcc, sm_100a) and the C oracle if they are missing
+    or older than their sources, so every test runs against the current code."""
+    from swiglu_ar_tts_b200 import build
+
+    import oracle
+
+    build.build()
+    oracle.build()

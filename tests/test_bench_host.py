@@ -1,0 +1,94 @@
+"""Host-side logic of bench.py on CPU: algorithmic byte counts, the multi-rank
+max-over-ranks reduction (gloo, world size 2), the reference arm's rank rule,
+and the ncu traffic record's staleness check."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from swiglu_ar_tts_b200.chain import DecodeChain  # noqa: E402
+from swiglu_ar_tts_b200.inputs import ChainShape  # noqa: E402
+
+
+def test_decode_step_algorithmic_bytes():
+    """Per decode step: 28 x (B x 81,932 + 8,192) bytes (two add+norms, M-RoPE
+    with 12 B of positions per row, SwiGLU, four gamma reads)."""
+    for batch, want in ((5, 11_699_856), (256, 587_517_952)):
+        shape = ChainShape(batch=batch)
+        from swiglu_ar_tts_b200.inputs import decode_chain_inputs
+
+        c = DecodeChain(shape, device="cpu", host_inputs=decode_chain_inputs(shape))
+        assert c.bytes_per_step() == want
+        assert c.launches_per_step == 112
+
+
+def test_prefill_algorithmic_bytes():
+    assert (2 * 64 * 1024 + 1024) * 4 == 528_384
+    assert (4 * 4096 * 2048 + 2048) * 2 == 67_112_960
+    assert 3 * 8192 * 6144 * 2 == 301_989_888
+    assert 2 * 4096 * 24 * 128 * 2 + 3 * 4096 * 4 == 50_380_800
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local = [3.0, 5.0][rank]  # rank 1 is slower
+    m = bench.reduce_max(local, dist, torch.device("cpu"))
+    v = bench.aggregate_value(world, 1_000_000_000, 10, m)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, m, v))
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29517
+    ps = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, m, v in res:
+        assert m == 5.0  # both ranks see the slowest rank's time
+        assert v == pytest.approx(2 * 1e9 * 10 / 5e-3 / 1e9)
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3", "--gpus", "2"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+
+
+def test_reduce_max_without_group_is_identity():
+    assert bench.reduce_max(2.5) == 2.5
+
+
+def test_traffic_record_tracks_kernel_source(tmp_path):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["swiglu_vec_kernel"]
+    got = bench.ncu_traffic("swiglu_vec_kernel", tuple(rec["sources"]))
+    if rec["source_digest"] == bench.source_digest(*rec["sources"]):
+        assert got == rec["dram_bytes_per_launch"]
+    else:  # the kernel changed since the capture: the bench must report null
+        assert got is None
+    assert bench.ncu_traffic("no_such_kernel", tuple(rec["sources"])) is None
+
+
+def test_hbm_peak_source():
+    peak, kind = bench.measured_hbm_peak()
+    assert kind in ("measured", "fallback") and peak > 1000

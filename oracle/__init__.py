@@ -88,6 +88,11 @@ class Oracle:
                                       _c_i32_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, _c_i32_p, ctypes.c_double]
         L.oracle_swiglu.argtypes = [_c_double_p, _c_double_p, _c_double_p, ctypes.c_int64]
+        L.oracle_layernorm.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_double_p,
+                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_double]
+        L.oracle_add_layernorm.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_double_p,
+                                           _c_double_p, _c_double_p, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_double, ctypes.c_int]
         L.oracle_mutant.restype = ctypes.c_int
         assert L.oracle_mutant() == mutant
 
@@ -162,6 +167,38 @@ class Oracle:
                                   _ptr(pos, _c_i32_p), tokens, hq, hk, d,
                                   _ptr(sec, _c_i32_p), float(theta))
         return q_out, k_out
+
+    def layernorm(self, x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
+        """gamma * (x - mean) / sqrt(var + eps) + beta over the last dimension
+        (population variance)."""
+        x = _f64(x)
+        gamma = _f64(gamma)
+        beta = _f64(beta)
+        hidden = x.shape[-1]
+        rows = x.size // hidden if hidden else 0
+        assert gamma.shape == (hidden,) and beta.shape == (hidden,)
+        y = np.empty_like(x)
+        self._lib.oracle_layernorm(_ptr(x, _c_double_p), _ptr(gamma, _c_double_p),
+                                   _ptr(beta, _c_double_p), _ptr(y, _c_double_p), rows, hidden,
+                                   float(eps))
+        return y
+
+    def add_layernorm(self, x, residual, gamma, beta, eps: float = 1e-6, dtype: str = "bf16"):
+        """Returns (y, residual_out) with residual_out = round(x + residual)."""
+        x = _f64(x)
+        residual = _f64(residual)
+        gamma = _f64(gamma)
+        beta = _f64(beta)
+        hidden = x.shape[-1]
+        rows = x.size // hidden if hidden else 0
+        y = np.empty_like(x)
+        res_out = np.empty_like(x)
+        code = {"f32": 0, "bf16": 1}[dtype]
+        self._lib.oracle_add_layernorm(_ptr(x, _c_double_p), _ptr(residual, _c_double_p),
+                                       _ptr(gamma, _c_double_p), _ptr(beta, _c_double_p),
+                                       _ptr(y, _c_double_p), _ptr(res_out, _c_double_p), rows,
+                                       hidden, float(eps), code)
+        return y, res_out
 
     def swiglu(self, gate, up) -> np.ndarray:
         gate = _f64(gate)

@@ -188,6 +188,53 @@ void oracle_add_rmsnorm(const double* x, const double* residual, const double* g
 }
 
 /* ------------------------------------------------------------------------- */
+/* LayerNorm ("Optimising autoregressive speech models", §09, the LayerNorm     */
+/* equation): y = gamma * (x - mean) / sqrt(variance + eps) + beta, with the    */
+/* mean and the (population) variance taken over the row.                      */
+/* ------------------------------------------------------------------------- */
+void oracle_layernorm(const double* x, const double* gamma, const double* beta, double* y,
+                      int64_t rows, int64_t hidden, double eps)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* xr = x + r * hidden;
+        double* yr = y + r * hidden;
+        double sum = 0.0;
+        for (int64_t i = 0; i < hidden; ++i)
+            sum += xr[i];
+        double mean = sum / (double)hidden;
+        double sq = 0.0;
+        for (int64_t i = 0; i < hidden; ++i) {
+            double d = xr[i] - mean;
+            sq += d * d;
+        }
+#if ORACLE_MUTANT == 13
+        double var = sq / (double)(hidden - 1); /* planted: unbiased variance */
+#else
+        double var = sq / (double)hidden;
+#endif
+        double denom = sqrt(var + eps);
+        for (int64_t i = 0; i < hidden; ++i) {
+#if ORACLE_MUTANT == 14
+            yr[i] = gamma[i] * (xr[i] - mean) / denom; /* planted: beta dropped */
+#else
+            yr[i] = gamma[i] * (xr[i] - mean) / denom + beta[i];
+#endif
+        }
+    }
+}
+
+/* Residual add + LayerNorm: the same "add, round to the dtype, then norm" as
+ * oracle_add_rmsnorm, with LayerNorm as the norm. */
+void oracle_add_layernorm(const double* x, const double* residual, const double* gamma,
+                          const double* beta, double* y, double* residual_out,
+                          int64_t rows, int64_t hidden, double eps, int dtype)
+{
+    for (int64_t i = 0; i < rows * hidden; ++i)
+        residual_out[i] = round_to_dtype(x[i] + residual[i], dtype);
+    oracle_layernorm(residual_out, gamma, beta, y, rows, hidden, eps);
+}
+
+/* ------------------------------------------------------------------------- */
 /* Multi-section rotary embedding (M-RoPE) on q and k.                          */
 /* Rotation of (x[j], x[j + D/2]) by the angle p * theta^(-2j/D), the textbook */
 /* RoPE frequency, with the position p taken from row t, h or w of the         */

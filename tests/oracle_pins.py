@@ -224,6 +224,67 @@ def pin_add_rmsnorm_is_add_then_norm(orc):
 
 
 # ---------------------------------------------------------------------------
+# LayerNorm
+# ---------------------------------------------------------------------------
+
+
+def pin_layernorm_two_element_closed_form(orc):
+    """x = (a, b): mean (a+b)/2, variance ((a-b)/2)^2, so at eps = 0 the row
+    normalises to (+1, -1) * sign(a-b): y = (gamma_0 + beta_0, -gamma_1 + beta_1)."""
+    gamma = np.array([1.5, -0.5])
+    beta = np.array([0.25, 2.0])
+    for a, b in ((3.0, 1.0), (-2.0, 7.0), (1e-3, -4e-3)):
+        y = orc.layernorm(np.array([[a, b]]), gamma, beta, 0.0)
+        sgn = 1.0 if a > b else -1.0
+        np.testing.assert_allclose(y[0], [sgn * gamma[0] + beta[0], -sgn * gamma[1] + beta[1]],
+                                   rtol=1e-14, atol=1e-14)
+    # with eps: the deviation is divided by sqrt(d^2 + eps), d = (a - b)/2
+    y = orc.layernorm(np.array([[3.0, 1.0]]), np.ones(2), np.zeros(2), 0.5)
+    np.testing.assert_allclose(y[0], [1 / math.sqrt(1.5), -1 / math.sqrt(1.5)], rtol=1e-15)
+
+
+def pin_layernorm_constant_row_is_beta(orc):
+    """A constant row has zero deviation: y = beta exactly (eps > 0)."""
+    beta = np.linspace(-1, 1, 32)
+    y = orc.layernorm(np.full((3, 32), 7.25), np.full(32, 3.0), beta, 1e-6)
+    assert np.array_equal(y, np.tile(beta, (3, 1)))
+
+
+def pin_layernorm_moments(orc):
+    """gamma = 1, beta = 0, eps = 0: every output row has mean 0 and population
+    variance 1; shifting the input row by a constant changes nothing."""
+    rng = np.random.default_rng(60)
+    x = rng.standard_normal((8, 500)) * 3 + 11
+    y = orc.layernorm(x, np.ones(500), np.zeros(500), 0.0)
+    np.testing.assert_allclose(y.mean(axis=1), 0, atol=1e-13)
+    np.testing.assert_allclose(y.var(axis=1), 1, rtol=1e-12)
+    np.testing.assert_allclose(orc.layernorm(x + 100.0, np.ones(500), np.zeros(500), 0.0), y,
+                               atol=1e-11)
+
+
+def pin_layernorm_zero_mean_is_rmsnorm_plus_beta(orc):
+    """On rows with mean exactly 0, LayerNorm is RMSNorm followed by + beta."""
+    rng = np.random.default_rng(61)
+    h = rng.standard_normal((4, 64))
+    x = np.concatenate([h, -h], axis=1)  # every row sums to exactly 0
+    gamma = 1 + 0.1 * rng.standard_normal(128)
+    beta = rng.standard_normal(128)
+    np.testing.assert_allclose(orc.layernorm(x, gamma, beta, 1e-6),
+                               orc.rmsnorm(x, gamma, 1e-6) + beta, rtol=1e-13, atol=1e-14)
+
+
+def pin_add_layernorm_is_add_then_norm(orc):
+    x = _bf16_tensor((8, 256), 62)
+    r = _bf16_tensor((8, 256), 63, std=2.0)
+    gamma = (_bf16_tensor((256,), 64) * 0.1 + 1).bfloat16()
+    beta = (_bf16_tensor((256,), 65) * 0.1).bfloat16()
+    y, res_out = orc.add_layernorm(x, r, gamma, beta, 1e-6, "bf16")
+    summed = (x.float() + r.float()).bfloat16()
+    assert np.array_equal(res_out, summed.double().numpy())
+    np.testing.assert_array_equal(y, orc.layernorm(summed, gamma, beta, 1e-6))
+
+
+# ---------------------------------------------------------------------------
 # M-RoPE
 # ---------------------------------------------------------------------------
 SECTIONS = (24, 20, 20)

@@ -23,6 +23,8 @@ MUTANTS = {
     10: "rotation in the wrong direction",
     11: "sign of the exponent in the sigmoid",
     12: "sigmoid without the g factor",
+    13: "LayerNorm with the unbiased variance",
+    14: "LayerNorm without beta",
 }
 
 

@@ -337,6 +337,19 @@ KERNEL_OF = {"add_rmsnorm": "norm_rows_kernel", "rmsnorm": "norm_rows_kernel",
              "mrope_qk": "mrope_vec_kernel", "swiglu": "swiglu_vec_kernel"}
 
 
+OP_OF_SYMBOL = {"arops_add_rmsnorm": "add_rmsnorm", "arops_add_layernorm": "add_layernorm",
+                "arops_mrope_qk": "mrope_qk", "arops_swiglu": "swiglu"}
+KERNEL_OF["add_layernorm"] = "norm_rows_kernel"
+
+
+def group_decode_calls(chain) -> dict:
+    """The decode step's pre-bound calls grouped by operator (symbol name)."""
+    groups: dict[str, list] = {}
+    for fn, a in chain._calls:
+        groups.setdefault(OP_OF_SYMBOL[fn.__name__], []).append((fn, a))
+    return groups
+
+
 def decode_split(chain, reps: int = 10) -> dict:
     """Fraction of a decode step spent in each operator's kernels.
 
@@ -344,21 +357,15 @@ def decode_split(chain, reps: int = 10) -> dict:
     SwiGLU for 28 layers); each group is captured as a graph of its own and
     timed, and the step's measured time is split in proportion.  Returns
     {op: (fraction, launches, algorithmic bytes)}."""
-    import ctypes  # noqa: F401
-
     from swiglu_ar_tts_b200 import lib
 
     L = lib()
-    names = {L.arops_add_rmsnorm: "add_rmsnorm", L.arops_mrope_qk: "mrope_qk",
-             L.arops_swiglu: "swiglu"}
-    groups: dict[str, list] = {}
-    for fn, a in chain._calls:
-        key = next(v for k, v in names.items() if k is fn or k.__name__ == fn.__name__)
-        groups.setdefault(key, []).append((fn, a))
+    groups = group_decode_calls(chain)
     sh = chain.shape
     e = chain.residual.element_size()
     per_launch_bytes = {
         "add_rmsnorm": (4 * sh.batch * sh.hidden + sh.hidden) * e,
+        "add_layernorm": (4 * sh.batch * sh.hidden + 2 * sh.hidden) * e,
         "mrope_qk": 2 * sh.batch * (sh.n_q_heads + sh.n_k_heads) * sh.head_dim * e + 3 * sh.batch * 4,
         "swiglu": 3 * sh.batch * sh.inter * e,
     }
@@ -599,6 +606,34 @@ def main() -> None:
                                                "swiglu_ar_tts_b200/csrc/common.cuh")),
                        "algorithmic_bytes": step.bytes["swiglu"]}
 
+    # the LayerNorm -> RMSNorm swap of "Optimising autoregressive speech models"
+    # §09: the same decode step with add + LayerNorm in every norm, timed alone
+    # (outside the timed steps) against the add + RMSNorm step
+    swap = {}
+    for batch, chain in ((5, step.chain5), (256, step.chain256)):
+        from swiglu_ar_tts_b200.chain import DecodeChain
+        from swiglu_ar_tts_b200.inputs import ChainShape
+
+        ln = DecodeChain(ChainShape(batch=batch), device=device, seed=2000 + batch,
+                         pdl=not args.no_pdl, norm="layer")
+        ln.capture()
+        t = {}
+        for name, c in (("rmsnorm", chain), ("layernorm", ln)):
+            c.set_position(3)
+            for _ in range(3):
+                c._graph.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(20):
+                c._graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t[name] = 1e3 * e0.elapsed_time(e1) / 20
+        swap[f"batch{batch}"] = {"us_rmsnorm_step": round(t["rmsnorm"], 2),
+                                 "us_layernorm_step": round(t["layernorm"], 2),
+                                 "rmsnorm_saves": round(1 - t["rmsnorm"] / t["layernorm"], 4)}
+        del ln
+
     # end to end: pinned host buffers in and out, through the same public calls
     step.setup_e2e()
     torch.cuda.synchronize()
@@ -652,6 +687,7 @@ def main() -> None:
         "roofline": roofline,
         "roofline_swiglu": roofline_swiglu,
         "kernels": kernels,
+        "layernorm_to_rmsnorm": swap,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": eager_launches + args.steps * (step.kernels_per_step - 4),

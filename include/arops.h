@@ -100,6 +100,29 @@ AROPS_API arops_status arops_add_rmsnorm(const void* x, const void* residual_in,
                                          arops_dtype dtype, void* stream);
 
 /*
+ * LayerNorm over the last dimension ("Optimising autoregressive speech models",
+ * §09, the LayerNorm equation): y = gamma * (x - mean) / sqrt(var + eps) + beta,
+ * mean and population variance over the row.  The variance is taken from the
+ * row's deviations (a second reduction over the row held in registers), not
+ * from E[x^2] - E[x]^2.  Layout and conventions as arops_rmsnorm; beta is
+ * [hidden] dtype.  This is the norm that the pages' §09 replaces by RMSNorm;
+ * it is here to measure that swap.
+ */
+AROPS_API arops_status arops_layernorm(const void* x, const void* gamma, const void* beta, void* y,
+                                       int64_t rows, int64_t hidden, float eps,
+                                       arops_dtype dtype, void* stream);
+
+/*
+ * Residual add + LayerNorm: residual_out = round_dtype(x + residual_in),
+ * y = LayerNorm(residual_out) (the LayerNorm counterpart of arops_add_rmsnorm).
+ */
+AROPS_API arops_status arops_add_layernorm(const void* x, const void* residual_in,
+                                           void* residual_out, const void* gamma,
+                                           const void* beta, void* y, int64_t rows,
+                                           int64_t hidden, float eps, arops_dtype dtype,
+                                           void* stream);
+
+/*
  * Multi-section rotary embedding (M-RoPE) of q and k, rotate-half pairing.
  * ("M-RoPE" in the Triton kernel-fusion post, section 3; RoPE as a rotation of
  * Q and K in the complex plane, forpes.ru post 233929, "Stage 2".)

@@ -212,7 +212,7 @@ class Oracle:
     # -- decode-step chain ---------------------------------------------------
     def decode_step(self, residual, layer_inputs: dict, step: int, eps: float = 1e-6,
                     theta: float = 1e6, sections=(24, 20, 20), dtype: str = "bf16",
-                    outputs: bool = True):
+                    outputs: bool = True, norm: str = "rms"):
         """One decode step over every layer, in the order add+RMSNorm, M-RoPE on
         q/k at position ``step`` in all three rows, add+RMSNorm, SwiGLU.
 
@@ -221,25 +221,29 @@ class Oracle:
         is rounded to ``dtype`` at the operator boundary, as the GPU writes it.
         Returns (residual after the step, dict of per-layer outputs y_attn, q, k,
         y_mlp, act).  With ``outputs=False`` only the residual stream is
-        computed and the dict is empty."""
+        computed and the dict is empty.  ``norm="layer"`` uses add + LayerNorm
+        with betas from layer_inputs["beta_attn"] / ["beta_mlp"]."""
         res = _f64(residual)
         batch = res.shape[0]
         pos = np.full((3, batch), step, dtype=np.int32)
         outs = {"y_attn": [], "q": [], "k": [], "y_mlp": [], "act": []}
+        def add_norm(x, r, key, layer):
+            if norm == "layer":
+                return self.add_layernorm(x, r, layer_inputs["gamma_" + key][layer],
+                                          layer_inputs["beta_" + key][layer], eps, dtype)
+            return self.add_rmsnorm(x, r, layer_inputs["gamma_" + key][layer], eps, dtype)
+
         for layer in range(len(layer_inputs["x_attn"])):
-            y, res = self.add_rmsnorm(layer_inputs["x_attn"][layer], res,
-                                      layer_inputs["gamma_attn"][layer], eps, dtype)
+            y, res = add_norm(layer_inputs["x_attn"][layer], res, "attn", layer)
             if not outputs:
-                _, res = self.add_rmsnorm(layer_inputs["x_mlp"][layer], res,
-                                          layer_inputs["gamma_mlp"][layer], eps, dtype)
+                _, res = add_norm(layer_inputs["x_mlp"][layer], res, "mlp", layer)
                 continue
             outs["y_attn"].append(self.round_to(y, dtype))
             qo, ko = self.mrope_qk(layer_inputs["q"][layer], layer_inputs["k"][layer], pos,
                                    sections, theta)
             outs["q"].append(self.round_to(qo, dtype))
             outs["k"].append(self.round_to(ko, dtype))
-            y, res = self.add_rmsnorm(layer_inputs["x_mlp"][layer], res,
-                                      layer_inputs["gamma_mlp"][layer], eps, dtype)
+            y, res = add_norm(layer_inputs["x_mlp"][layer], res, "mlp", layer)
             outs["y_mlp"].append(self.round_to(y, dtype))
             act = self.swiglu(layer_inputs["gate"][layer], layer_inputs["up"][layer])
             outs["act"].append(self.round_to(act, dtype))

@@ -18,7 +18,8 @@ import threading
 import torch
 
 __all__ = [
-    "rmsnorm", "add_rmsnorm", "mrope_qk", "swiglu", "set_pdl", "set_streaming",
+    "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "swiglu", "set_pdl",
+    "set_streaming",
     "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
 ]
@@ -67,7 +68,12 @@ def lib() -> ctypes.CDLL:
         L.arops_mrope_qk.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32,
                                      ctypes.POINTER(_i32), ctypes.c_float, ctypes.c_int, _vp]
         L.arops_swiglu.argtypes = [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
-        for fn in ("arops_rmsnorm", "arops_add_rmsnorm", "arops_mrope_qk", "arops_swiglu"):
+        L.arops_layernorm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_float,
+                                      ctypes.c_int, _vp]
+        L.arops_add_layernorm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                          ctypes.c_float, ctypes.c_int, _vp]
+        for fn in ("arops_rmsnorm", "arops_add_rmsnorm", "arops_mrope_qk", "arops_swiglu",
+                   "arops_layernorm", "arops_add_layernorm"):
             getattr(L, fn).restype = ctypes.c_int
         L.arops_set_pdl.argtypes = [ctypes.c_int]
         L.arops_set_pdl.restype = ctypes.c_int
@@ -153,6 +159,50 @@ def add_rmsnorm(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor, ep
         _check(lib().arops_add_rmsnorm(x.data_ptr(), residual.data_ptr(), residual_out.data_ptr(),
                                        gamma.data_ptr(), y.data_ptr(), rows, hidden, float(eps),
                                        code, _stream(x)))
+    return y, residual_out
+
+
+def layernorm(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, eps: float = 1e-6,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = gamma * (x - mean) / sqrt(var + eps) + beta over the last dimension."""
+    hidden = x.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    for n, t in (("x", x), ("gamma", gamma), ("beta", beta), ("out", out)):
+        _cuda_contig(n, t)
+    if gamma.shape != (hidden,) or beta.shape != (hidden,) or out.shape != x.shape:
+        raise ValueError("shape mismatch")
+    code = _dtype_code(x, gamma, beta, out)
+    rows = x.numel() // hidden if hidden else 0
+    with torch.cuda.device(x.device):
+        _check(lib().arops_layernorm(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                     out.data_ptr(), rows, hidden, float(eps), code, _stream(x)))
+    return out
+
+
+def add_layernorm(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
+                  beta: torch.Tensor, eps: float = 1e-6, y: torch.Tensor | None = None,
+                  residual_out: torch.Tensor | None = None):
+    """residual_out = x + residual (rounded); y = LayerNorm(residual_out).
+    ``residual_out`` defaults to ``residual`` (in place).  Returns ``(y, residual_out)``."""
+    hidden = x.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    if residual_out is None:
+        residual_out = residual
+    for n, t in (("x", x), ("residual", residual), ("gamma", gamma), ("beta", beta), ("y", y),
+                 ("residual_out", residual_out)):
+        _cuda_contig(n, t)
+    if (residual.shape != x.shape or y.shape != x.shape or residual_out.shape != x.shape
+            or gamma.shape != (hidden,) or beta.shape != (hidden,)):
+        raise ValueError("shape mismatch")
+    code = _dtype_code(x, residual, gamma, beta, y, residual_out)
+    rows = x.numel() // hidden if hidden else 0
+    with torch.cuda.device(x.device):
+        _check(lib().arops_add_layernorm(x.data_ptr(), residual.data_ptr(),
+                                         residual_out.data_ptr(), gamma.data_ptr(),
+                                         beta.data_ptr(), y.data_ptr(), rows, hidden, float(eps),
+                                         code, _stream(x)))
     return y, residual_out
 
 

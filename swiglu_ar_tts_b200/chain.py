@@ -9,6 +9,10 @@ kernel-fusion post for Qwen3-TTS, section 1) runs, for each layer:
     add + RMSNorm  (MLP input)            residual <- residual + x_mlp
     SwiGLU         (MLP activation)
 
+With ``norm="layer"`` both norms are add + LayerNorm (with a beta per norm),
+the architecture that "Optimising autoregressive speech models" §09 swaps for
+RMSNorm; timing both chains measures that swap.
+
 The projections, attention and MLP GEMMs between these operators are not part
 of this library; their outputs are stood in for by fixed per-layer buffers, so
 a step is exactly the 4 * layers operator launches.  The residual stream is the
@@ -28,21 +32,31 @@ import ctypes
 import torch
 
 from . import DTYPES, ArOpsError, lib
-from .inputs import EPS, SECTIONS, THETA, ChainShape, decode_chain_inputs
+from .inputs import EPS, SECTIONS, THETA, ChainShape, decode_chain_inputs, normal
 
 
 class DecodeChain:
     def __init__(self, shape: ChainShape, dtype: str = "bf16", seed: int = 0,
                  device: str | torch.device = "cuda", eps: float = EPS, theta: float = THETA,
-                 sections=SECTIONS, host_inputs: dict | None = None, pdl: bool = True):
+                 sections=SECTIONS, host_inputs: dict | None = None, pdl: bool = True,
+                 norm: str = "rms"):
         self.shape = shape
         self.dtype = dtype
         self.eps = eps
         self.theta = theta
         self.sections = tuple(int(s) for s in sections)
         self.pdl = pdl
+        if norm not in ("rms", "layer"):
+            raise ValueError(norm)
+        self.norm = norm
         self.device = torch.device(device)
         host = host_inputs if host_inputs is not None else decode_chain_inputs(shape, dtype, seed)
+        if norm == "layer" and "beta_attn" not in host:
+            host = dict(host)
+            host["beta_attn"] = [normal((shape.hidden,), seed + 500_000 + 2 * l, std=0.1, dtype=dtype)
+                                 for l in range(shape.layers)]
+            host["beta_mlp"] = [normal((shape.hidden,), seed + 500_001 + 2 * l, std=0.1, dtype=dtype)
+                                for l in range(shape.layers)]
         self.host_inputs = host
         d = self.device
         self.residual0 = host["residual"].to(d)
@@ -70,17 +84,24 @@ class DecodeChain:
         res = self.residual.data_ptr()
         B, H, I = sh.batch, sh.hidden, sh.inter
         calls = []
+        def norm_call(x, gamma, beta, y):
+            if self.norm == "layer":
+                return (L.arops_add_layernorm, [x.data_ptr(), res, res, gamma.data_ptr(),
+                                                beta.data_ptr(), y.data_ptr(), B, H, eps, code])
+            return (L.arops_add_rmsnorm, [x.data_ptr(), res, res, gamma.data_ptr(),
+                                          y.data_ptr(), B, H, eps, code])
+
         for l in range(sh.layers):
-            calls.append((L.arops_add_rmsnorm, [self.inp["x_attn"][l].data_ptr(), res, res,
-                                                self.inp["gamma_attn"][l].data_ptr(),
-                                                self.y_attn[l].data_ptr(), B, H, eps, code]))
+            ba = self.inp["beta_attn"][l] if self.norm == "layer" else None
+            bm = self.inp["beta_mlp"][l] if self.norm == "layer" else None
+            calls.append(norm_call(self.inp["x_attn"][l], self.inp["gamma_attn"][l], ba,
+                                   self.y_attn[l]))
             calls.append((L.arops_mrope_qk, [self.inp["q"][l].data_ptr(), self.inp["k"][l].data_ptr(),
                                              self.q_out[l].data_ptr(), self.k_out[l].data_ptr(),
                                              self.pos.data_ptr(), B, sh.n_q_heads, sh.n_k_heads,
                                              sh.head_dim, self._sec, theta, code]))
-            calls.append((L.arops_add_rmsnorm, [self.inp["x_mlp"][l].data_ptr(), res, res,
-                                                self.inp["gamma_mlp"][l].data_ptr(),
-                                                self.y_mlp[l].data_ptr(), B, H, eps, code]))
+            calls.append(norm_call(self.inp["x_mlp"][l], self.inp["gamma_mlp"][l], bm,
+                                   self.y_mlp[l]))
             calls.append((L.arops_swiglu, [self.inp["gate"][l].data_ptr(), self.inp["up"][l].data_ptr(),
                                            self.act[l].data_ptr(), B, I, code]))
         self._calls = calls
@@ -95,7 +116,8 @@ class DecodeChain:
         sh = self.shape
         e = self.residual.element_size()
         B, H, I = sh.batch, sh.hidden, sh.inter
-        per_layer = (2 * (4 * B * H + H) * e  # two add+norms: x, res in; res', y out; gamma
+        weights = 2 if self.norm == "layer" else 1  # gamma (and beta) per norm
+        per_layer = (2 * (4 * B * H + weights * H) * e  # two add+norms: x, res in; res', y out
                      + 2 * B * (sh.n_q_heads + sh.n_k_heads) * sh.head_dim * e + 3 * B * 4
                      + 3 * B * I * e)
         return sh.layers * per_layer

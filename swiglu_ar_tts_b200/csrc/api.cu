@@ -115,23 +115,44 @@ using namespace arops;
 
 extern "C" {
 
+}  // extern "C"
+
+namespace {
+
+// Shared validation and dispatch of the four norm entry points.
+arops_status norm_entry(const char* name, const void* x, const void* residual_in,
+                        void* residual_out, const void* gamma, const void* beta, void* y,
+                        int64_t rows, int64_t hidden, float eps, arops_dtype dtype, void* stream,
+                        bool add, bool ln)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "%s: unknown dtype %d", name, (int)dtype);
+    if (rows < 0 || hidden <= 0 || hidden > INT32_MAX)
+        return fail(AROPS_ERR_INVALID, "%s: bad shape rows=%lld hidden=%lld", name,
+                    (long long)rows, (long long)hidden);
+    if (!(eps >= 0.0f) || isinf(eps))
+        return fail(AROPS_ERR_INVALID, "%s: eps must be finite and >= 0", name);
+    if (rows == 0)
+        return ok();
+    if (!x || !gamma || !y || (add && (!residual_in || !residual_out)) || (ln && !beta))
+        return fail(AROPS_ERR_INVALID, "%s: null pointer", name);
+    if (add && y == residual_out)
+        return fail(AROPS_ERR_INVALID, "%s: y and residual_out are one buffer", name);
+    return from_cuda(launch_norm(x, add ? residual_in : nullptr, add ? residual_out : nullptr,
+                                 gamma, ln ? beta : nullptr, y, rows, hidden, eps, dtype,
+                                 static_cast<cudaStream_t>(stream)),
+                     name);
+}
+
+}  // namespace
+
+extern "C" {
+
 AROPS_API arops_status arops_rmsnorm(const void* x, const void* gamma, void* y, int64_t rows,
                                      int64_t hidden, float eps, arops_dtype dtype, void* stream)
 {
-    if (!valid_dtype(dtype))
-        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: unknown dtype %d", (int)dtype);
-    if (rows < 0 || hidden <= 0 || hidden > INT32_MAX)
-        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: bad shape rows=%lld hidden=%lld",
-                    (long long)rows, (long long)hidden);
-    if (!(eps >= 0.0f) || isinf(eps))
-        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: eps must be finite and >= 0");
-    if (rows == 0)
-        return ok();
-    if (!x || !gamma || !y)
-        return fail(AROPS_ERR_INVALID, "arops_rmsnorm: null pointer");
-    return from_cuda(launch_norm(x, nullptr, nullptr, gamma, y, rows, hidden, eps, dtype,
-                                 static_cast<cudaStream_t>(stream)),
-                     "arops_rmsnorm");
+    return norm_entry("arops_rmsnorm", x, nullptr, nullptr, gamma, nullptr, y, rows, hidden, eps,
+                      dtype, stream, false, false);
 }
 
 AROPS_API arops_status arops_add_rmsnorm(const void* x, const void* residual_in,
@@ -139,22 +160,26 @@ AROPS_API arops_status arops_add_rmsnorm(const void* x, const void* residual_in,
                                          int64_t rows, int64_t hidden, float eps,
                                          arops_dtype dtype, void* stream)
 {
-    if (!valid_dtype(dtype))
-        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: unknown dtype %d", (int)dtype);
-    if (rows < 0 || hidden <= 0 || hidden > INT32_MAX)
-        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: bad shape rows=%lld hidden=%lld",
-                    (long long)rows, (long long)hidden);
-    if (!(eps >= 0.0f) || isinf(eps))
-        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: eps must be finite and >= 0");
-    if (rows == 0)
-        return ok();
-    if (!x || !residual_in || !residual_out || !gamma || !y)
-        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: null pointer");
-    if (y == residual_out)
-        return fail(AROPS_ERR_INVALID, "arops_add_rmsnorm: y and residual_out are one buffer");
-    return from_cuda(launch_norm(x, residual_in, residual_out, gamma, y, rows, hidden, eps, dtype,
-                                 static_cast<cudaStream_t>(stream)),
-                     "arops_add_rmsnorm");
+    return norm_entry("arops_add_rmsnorm", x, residual_in, residual_out, gamma, nullptr, y, rows,
+                      hidden, eps, dtype, stream, true, false);
+}
+
+AROPS_API arops_status arops_layernorm(const void* x, const void* gamma, const void* beta, void* y,
+                                       int64_t rows, int64_t hidden, float eps, arops_dtype dtype,
+                                       void* stream)
+{
+    return norm_entry("arops_layernorm", x, nullptr, nullptr, gamma, beta, y, rows, hidden, eps,
+                      dtype, stream, false, true);
+}
+
+AROPS_API arops_status arops_add_layernorm(const void* x, const void* residual_in,
+                                           void* residual_out, const void* gamma,
+                                           const void* beta, void* y, int64_t rows,
+                                           int64_t hidden, float eps, arops_dtype dtype,
+                                           void* stream)
+{
+    return norm_entry("arops_add_layernorm", x, residual_in, residual_out, gamma, beta, y, rows,
+                      hidden, eps, dtype, stream, true, true);
 }
 
 AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out, void* k_out,

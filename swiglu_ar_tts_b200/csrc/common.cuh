@@ -207,9 +207,10 @@ cudaError_t resident_ctas(K kernel, int threads, size_t smem, int* ctas)
 }
 
 // Launchers (one per operator), called after argument validation.
+// residual_in == nullptr: no residual add; beta == nullptr: RMSNorm, else LayerNorm.
 cudaError_t launch_norm(const void* x, const void* residual_in, void* residual_out,
-                        const void* gamma, void* y, int64_t rows, int64_t hidden, float eps,
-                        arops_dtype dtype, cudaStream_t stream);
+                        const void* gamma, const void* beta, void* y, int64_t rows,
+                        int64_t hidden, float eps, arops_dtype dtype, cudaStream_t stream);
 
 cudaError_t launch_swiglu(const void* gate, const void* up, void* out, int64_t n,
                           arops_dtype dtype, cudaStream_t stream);

@@ -157,10 +157,53 @@ norm_tma_kernel(const T* x, const T* residual_in, T* residual_out, const T* __re
 
 constexpr int kRowsPerSmallCta = 2;  // GW == 1: two warps, one row each
 
-template <typename T, bool ADD, int VPL, int GW>
+// Sum of v over the threads that own one row: shuffles, then (GW > 1) one
+// shared-memory step.  `red` holds two buffers used alternately; every call
+// flips `parity`, so one barrier per reduction is enough however many
+// reductions a row takes (RMSNorm one, LayerNorm two).
+template <int GW>
+__device__ __forceinline__ float group_sum(float v, float (*red)[GW], int& parity, int tid)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if constexpr (GW > 1) {
+        if ((tid & 31) == 0)
+            red[parity][tid >> 5] = v;
+        __syncthreads();
+        v = 0.f;
+#pragma unroll
+        for (int w = 0; w < GW; ++w)
+            v += red[parity][w];
+        parity ^= 1;
+    }
+    return v;
+}
+
+// Value of thread 0 of the row's group, given to every thread of the group:
+// a shuffle for one warp per row, shared memory and a barrier for several.
+template <int GW>
+__device__ __forceinline__ float row_broadcast(float v, float& slot, int tid)
+{
+    if constexpr (GW == 1) {
+        return __shfl_sync(0xFFFFFFFFu, v, 0);
+    } else {
+        __syncthreads();  // the previous row is done with the slot
+        if (tid == 0)
+            slot = v;
+        __syncthreads();
+        return slot;
+    }
+}
+
+// LN = false: RMSNorm, y = x * rsqrt(mean(x^2) + eps) * gamma.
+// LN = true:  LayerNorm, y = (x - mean) * rsqrt(mean((x - mean)^2) + eps) * gamma + beta,
+//             the variance taken from the row held in registers (two reductions),
+//             both sums taken over the row shifted by its first element.
+template <typename T, bool ADD, bool LN, int VPL, int GW>
 __global__ void __launch_bounds__(GW == 1 ? 32 * kRowsPerSmallCta : 32 * GW)
-norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
-                 const T* __restrict__ gamma, T* y, int64_t rows, int hidden, float eps)
+norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
+                 const T* __restrict__ beta, T* y, int64_t rows, int hidden, float eps)
 {
     constexpr int E = Vec<T>::N;
     constexpr int G = 32 * GW;  // threads per row
@@ -170,8 +213,9 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
     const int gt = (GW == 1) ? (tid & 31) : tid;
     const int group = (GW == 1) ? (tid >> 5) : 0;
     __shared__ float red[2][GW];
+    __shared__ float shift;
 
-    // this group's first row and gamma into L2 while the previous kernel drains
+    // this group's first row and the weights into L2 while the previous kernel drains
     {
         const int64_t row0 = (int64_t)blockIdx.x * ROWS_PER_CTA + group;
         const uint32_t row_bytes = (uint32_t)hidden * sizeof(T);
@@ -180,8 +224,11 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
             if constexpr (ADD)
                 prefetch_l2(residual_in + (size_t)row0 * hidden, row_bytes);
         }
-        if (tid == 0 && blockIdx.x < 64)  // later CTAs find gamma in L2 already
+        if (tid == 0 && blockIdx.x < 64) {  // later CTAs find them in L2 already
             prefetch_l2(gamma, row_bytes);
+            if constexpr (LN)
+                prefetch_l2(beta, row_bytes);
+        }
     }
     pdl_wait();
     pdl_allow_dependents();
@@ -190,16 +237,19 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
     for (int64_t row = (int64_t)blockIdx.x * ROWS_PER_CTA + group; row < rows;
          row += (int64_t)gridDim.x * ROWS_PER_CTA) {
         const size_t base = (size_t)row * (size_t)hidden;
-        uint4 v[VPL], gv[VPL];
-        float ss = 0.f;
-        // gamma is loaded with the row, not after the reduction: a load issued
-        // after the shuffles would add a dependent round trip to every row
+        uint4 v[VPL], gv[VPL], bv[LN ? VPL : 1];
+        // the weights are loaded with the row, not after the reduction: a load
+        // issued after the shuffles would add a dependent round trip to every row
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
             const int vi = gt + i * G;
-            if (vi < nvec)
+            if (vi < nvec) {
                 gv[i] = __ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E));
+                if constexpr (LN)
+                    bv[i] = __ldg(reinterpret_cast<const uint4*>(beta + (size_t)vi * E));
+            }
         }
+        float s1 = 0.f;  // sum of x^2 (RMSNorm) or of x (LayerNorm)
         if constexpr (ADD) {
             uint4 r[VPL];
 #pragma unroll
@@ -222,10 +272,6 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
                         a[e] = a[e] + b[e];
                     v[i] = Vec<T>::pack(a);  // the residual, rounded to T
                     st_stream(residual_out + base + (size_t)vi * E, v[i]);
-                    Vec<T>::unpack(v[i], a);  // normalise what was written
-#pragma unroll
-                    for (int e = 0; e < E; ++e)
-                        ss = fmaf(a[e], a[e], ss);
                 }
             }
         } else {
@@ -235,6 +281,32 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
                 if (vi < nvec)
                     v[i] = ld_stream(x + base + (size_t)vi * E);
             }
+        }
+        // LayerNorm sums the row shifted by its first element c: the mean's
+        // rounding error then scales with the row's spread, not with its offset
+        float c = 0.f;
+        if constexpr (LN) {
+            float a0[E];
+            Vec<T>::unpack(v[0], a0);  // thread 0 of the group holds element 0
+            c = row_broadcast<GW>(a0[0], shift, tid);
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int vi = gt + i * G;
+            if (vi < nvec) {
+                float a[E];
+                Vec<T>::unpack(v[i], a);  // for add+norm: exactly what was written
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    s1 = LN ? s1 + (a[e] - c) : fmaf(a[e], a[e], s1);
+            }
+        }
+        s1 = group_sum<GW>(s1, red, parity, tid);
+
+        float mean = 0.f, r;  // for LayerNorm: the mean of the shifted row
+        if constexpr (LN) {
+            mean = s1 / (float)hidden;
+            float s2 = 0.f;
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const int vi = gt + i * G;
@@ -242,28 +314,17 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
                     float a[E];
                     Vec<T>::unpack(v[i], a);
 #pragma unroll
-                    for (int e = 0; e < E; ++e)
-                        ss = fmaf(a[e], a[e], ss);
+                    for (int e = 0; e < E; ++e) {
+                        const float d = (a[e] - c) - mean;
+                        s2 = fmaf(d, d, s2);
+                    }
                 }
             }
+            s2 = group_sum<GW>(s2, red, parity, tid);
+            r = rsqrtf(s2 / (float)hidden + eps);
+        } else {
+            r = rsqrtf(s1 / (float)hidden + eps);
         }
-
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-        if constexpr (GW > 1) {
-            // parity double-buffering: the next row writes the other buffer, so
-            // one barrier per row is enough
-            if ((tid & 31) == 0)
-                red[parity][tid >> 5] = ss;
-            __syncthreads();
-            ss = 0.f;
-#pragma unroll
-            for (int w = 0; w < GW; ++w)
-                ss += red[parity][w];
-            parity ^= 1;
-        }
-        const float r = rsqrtf(ss / (float)hidden + eps);
 
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
@@ -272,24 +333,34 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out,
                 float a[E], g[E];
                 Vec<T>::unpack(v[i], a);
                 Vec<T>::unpack(gv[i], g);
+                if constexpr (LN) {
+                    float b[E];
+                    Vec<T>::unpack(bv[i], b);
 #pragma unroll
-                for (int e = 0; e < E; ++e)
-                    a[e] = a[e] * r * g[e];
+                    for (int e = 0; e < E; ++e)
+                        a[e] = ((a[e] - c) - mean) * r * g[e] + b[e];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        a[e] = a[e] * r * g[e];
+                }
                 st_stream(y + base + (size_t)vi * E, Vec<T>::pack(a));
             }
         }
     }
 }
 
-// One CTA per row, two passes over the row.  VEC: 16-byte vectors (aligned,
-// hidden % E == 0); otherwise one element at a time.  Each thread touches the
-// same elements in both passes, so pass 2 reads back its own pass-1 writes.
+// One CTA per row, passes over the row: RMSNorm two (sum of squares, output),
+// LayerNorm three (sum, squared deviations, output); later passes are served
+// from L2.  VEC: 16-byte vectors (aligned, hidden % E == 0); otherwise one
+// element at a time.  Each thread touches the same elements in every pass, so
+// later passes read back its own pass-1 writes of residual_out.
 constexpr int kLoopThreads = 256;
 
-template <typename T, bool ADD, bool VEC>
+template <typename T, bool ADD, bool LN, bool VEC>
 __global__ void __launch_bounds__(kLoopThreads)
-norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
-                   const T* __restrict__ gamma, T* y, int64_t rows, int64_t hidden, float eps)
+norm_looped_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
+                   const T* __restrict__ beta, T* y, int64_t rows, int64_t hidden, float eps)
 {
     constexpr int E = Vec<T>::N;
     constexpr int W = kLoopThreads / 32;
@@ -299,10 +370,25 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
     pdl_wait();
     pdl_allow_dependents();
 
+    __shared__ float shift;
     int parity = 0;
     for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
         const size_t base = (size_t)row * (size_t)hidden;
-        float ss = 0.f;
+        float s1 = 0.f;
+        // LayerNorm: the row's first element (after the residual add), shifted
+        // out of both sums as in the register kernel
+        float c = 0.f;
+        if constexpr (LN) {
+            __syncthreads();  // the previous row is done with `shift`
+            if (tid == 0) {
+                float a0 = load_elem(x + base);
+                if constexpr (ADD)
+                    a0 = round_to(a0 + load_elem(residual_in + base), residual_out);
+                shift = a0;
+            }
+            __syncthreads();
+            c = shift;
+        }
         if constexpr (VEC) {
             const int64_t nvec = hidden / E;
             for (int64_t vi = tid; vi < nvec; vi += kLoopThreads) {
@@ -321,7 +407,7 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
                 Vec<T>::unpack(va, a);
 #pragma unroll
                 for (int e = 0; e < E; ++e)
-                    ss = fmaf(a[e], a[e], ss);
+                    s1 = LN ? s1 + (a[e] - c) : fmaf(a[e], a[e], s1);
             }
         } else {
             for (int64_t i = tid; i < hidden; i += kLoopThreads) {
@@ -330,38 +416,66 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out,
                     a = round_to(a + load_elem(residual_in + base + i), residual_out);
                     store_elem(residual_out + base + i, a);
                 }
-                ss = fmaf(a, a, ss);
+                s1 = LN ? s1 + (a - c) : fmaf(a, a, s1);
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-        if ((tid & 31) == 0)
-            red[parity][tid >> 5] = ss;
-        __syncthreads();
-        ss = 0.f;
-#pragma unroll
-        for (int w = 0; w < W; ++w)
-            ss += red[parity][w];
-        parity ^= 1;
-        const float r = rsqrtf(ss / (float)hidden + eps);
+        s1 = group_sum<W>(s1, red, parity, tid);
 
         const T* src = ADD ? residual_out : x;
+        float mean = 0.f, r;
+        if constexpr (LN) {
+            mean = s1 / (float)hidden;
+            float s2 = 0.f;
+            if constexpr (VEC) {
+                const int64_t nvec = hidden / E;
+                for (int64_t vi = tid; vi < nvec; vi += kLoopThreads) {
+                    float a[E];
+                    Vec<T>::unpack(ld_stream(src + base + vi * E), a);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const float d = (a[e] - c) - mean;
+                        s2 = fmaf(d, d, s2);
+                    }
+                }
+            } else {
+                for (int64_t i = tid; i < hidden; i += kLoopThreads) {
+                    const float d = (load_elem(src + base + i) - c) - mean;
+                    s2 = fmaf(d, d, s2);
+                }
+            }
+            s2 = group_sum<W>(s2, red, parity, tid);
+            r = rsqrtf(s2 / (float)hidden + eps);
+        } else {
+            r = rsqrtf(s1 / (float)hidden + eps);
+        }
+
         if constexpr (VEC) {
             const int64_t nvec = hidden / E;
             for (int64_t vi = tid; vi < nvec; vi += kLoopThreads) {
                 float a[E], g[E];
                 Vec<T>::unpack(ld_stream(src + base + vi * E), a);
                 Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(gamma + vi * E)), g);
+                if constexpr (LN) {
+                    float b[E];
+                    Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(beta + vi * E)), b);
 #pragma unroll
-                for (int e = 0; e < E; ++e)
-                    a[e] = a[e] * r * g[e];
+                    for (int e = 0; e < E; ++e)
+                        a[e] = ((a[e] - c) - mean) * r * g[e] + b[e];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        a[e] = a[e] * r * g[e];
+                }
                 st_stream(y + base + vi * E, Vec<T>::pack(a));
             }
         } else {
             for (int64_t i = tid; i < hidden; i += kLoopThreads) {
                 const float a = load_elem(src + base + i);
-                store_elem(y + base + i, a * r * load_elem(gamma + i));
+                if constexpr (LN)
+                    store_elem(y + base + i,
+                               ((a - c) - mean) * r * load_elem(gamma + i) + load_elem(beta + i));
+                else
+                    store_elem(y + base + i, a * r * load_elem(gamma + i));
             }
         }
     }
@@ -411,32 +525,34 @@ cudaError_t launch_norm_tma(const T* x, const T* ri, T* ro, const T* g, T* y, in
     return launch_norm_tma_t<T, ADD, 256>(x, ri, ro, g, y, rows, hidden, eps, st, di);
 }
 
-template <typename T, bool ADD, int VPL>
-cudaError_t launch_rows_gw1(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
-                            int hidden, float eps, cudaStream_t st, int64_t cap)
+template <typename T, bool ADD, bool LN, int VPL>
+cudaError_t launch_rows_gw1(const T* x, const T* ri, T* ro, const T* g, const T* b, T* y,
+                            int64_t rows, int hidden, float eps, cudaStream_t st, int64_t cap)
 {
     const int64_t grid = std::min<int64_t>(ceil_div(rows, kRowsPerSmallCta), cap);
-    return launch(norm_rows_kernel<T, ADD, VPL, 1>, dim3((unsigned)grid),
-                  dim3(32 * kRowsPerSmallCta), 0, st, x, ri, ro, g, y, rows, hidden, eps);
+    return launch(norm_rows_kernel<T, ADD, LN, VPL, 1>, dim3((unsigned)grid),
+                  dim3(32 * kRowsPerSmallCta), 0, st, x, ri, ro, g, b, y, rows, hidden, eps);
 }
 
-template <typename T, bool ADD, int GW>
-cudaError_t launch_rows_gwn(const T* x, const T* ri, T* ro, const T* g, T* y, int64_t rows,
-                            int hidden, float eps, cudaStream_t st, int64_t cap)
+template <typename T, bool ADD, bool LN, int GW>
+cudaError_t launch_rows_gwn(const T* x, const T* ri, T* ro, const T* g, const T* b, T* y,
+                            int64_t rows, int hidden, float eps, cudaStream_t st, int64_t cap)
 {
     const int64_t grid = std::min<int64_t>(rows, cap);
-    return launch(norm_rows_kernel<T, ADD, 8, GW>, dim3((unsigned)grid), dim3(32 * GW), 0, st,
-                  x, ri, ro, g, y, rows, hidden, eps);
+    return launch(norm_rows_kernel<T, ADD, LN, 8, GW>, dim3((unsigned)grid), dim3(32 * GW), 0,
+                  st, x, ri, ro, g, b, y, rows, hidden, eps);
 }
 
-template <typename T, bool ADD>
-cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void* gv, void* yv,
-                          int64_t rows, int64_t hidden, float eps, cudaStream_t st)
+template <typename T, bool ADD, bool LN>
+cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void* gv,
+                          const void* bv, void* yv, int64_t rows, int64_t hidden, float eps,
+                          cudaStream_t st)
 {
     const T* x = static_cast<const T*>(xv);
     const T* ri = static_cast<const T*>(riv);
     T* ro = static_cast<T*>(rov);
     const T* g = static_cast<const T*>(gv);
+    const T* b = static_cast<const T*>(bv);
     T* y = static_cast<T*>(yv);
     constexpr int E = Vec<T>::N;
 
@@ -447,58 +563,69 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
     const int64_t cap = (int64_t)di.sm_count * 32;
 
     const bool vec = (hidden % E == 0) && aligned16(x) && aligned16(g) && aligned16(y) &&
-                     (!ADD || (aligned16(ri) && aligned16(ro)));
-    if (vec && streaming_enabled()) {
-        err = launch_norm_tma<T, ADD>(x, ri, ro, g, y, rows, (int)hidden, eps, st, di);
-        if (err != cudaErrorNotSupported)
-            return err;
+                     (!ADD || (aligned16(ri) && aligned16(ro))) && (!LN || aligned16(b));
+    if constexpr (!LN) {
+        if (vec && streaming_enabled()) {
+            err = launch_norm_tma<T, ADD>(x, ri, ro, g, y, rows, (int)hidden, eps, st, di);
+            if (err != cudaErrorNotSupported)
+                return err;
+        }
     }
     if (vec) {
         const int64_t nvec = hidden / E;
         const int h = (int)hidden;
         if (nvec <= 32)
-            return launch_rows_gw1<T, ADD, 1>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gw1<T, ADD, LN, 1>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 64)
-            return launch_rows_gw1<T, ADD, 2>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gw1<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 128)
-            return launch_rows_gw1<T, ADD, 4>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gw1<T, ADD, LN, 4>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 256)
-            return launch_rows_gw1<T, ADD, 8>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gw1<T, ADD, LN, 8>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 512)
-            return launch_rows_gwn<T, ADD, 2>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gwn<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 1024)
-            return launch_rows_gwn<T, ADD, 4>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gwn<T, ADD, LN, 4>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 2048)
-            return launch_rows_gwn<T, ADD, 8>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gwn<T, ADD, LN, 8>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 4096)
-            return launch_rows_gwn<T, ADD, 16>(x, ri, ro, g, y, rows, h, eps, st, cap);
+            return launch_rows_gwn<T, ADD, LN, 16>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
     }
     const int64_t grid = std::min<int64_t>(rows, cap);
     if (vec)
-        return launch(norm_looped_kernel<T, ADD, true>, dim3((unsigned)grid), dim3(kLoopThreads),
-                      0, st, x, ri, ro, g, y, rows, hidden, eps);
-    return launch(norm_looped_kernel<T, ADD, false>, dim3((unsigned)grid), dim3(kLoopThreads), 0,
-                  st, x, ri, ro, g, y, rows, hidden, eps);
+        return launch(norm_looped_kernel<T, ADD, LN, true>, dim3((unsigned)grid),
+                      dim3(kLoopThreads), 0, st, x, ri, ro, g, b, y, rows, hidden, eps);
+    return launch(norm_looped_kernel<T, ADD, LN, false>, dim3((unsigned)grid), dim3(kLoopThreads),
+                  0, st, x, ri, ro, g, b, y, rows, hidden, eps);
+}
+
+template <typename T>
+cudaError_t launch_norm_dt(const void* x, const void* ri, void* ro, const void* g, const void* b,
+                           void* y, int64_t rows, int64_t hidden, float eps, cudaStream_t st)
+{
+    const bool add = ri != nullptr;
+    const bool ln = b != nullptr;
+    if (add && ln)
+        return launch_norm_t<T, true, true>(x, ri, ro, g, b, y, rows, hidden, eps, st);
+    if (add)
+        return launch_norm_t<T, true, false>(x, ri, ro, g, nullptr, y, rows, hidden, eps, st);
+    if (ln)
+        return launch_norm_t<T, false, true>(x, nullptr, nullptr, g, b, y, rows, hidden, eps, st);
+    return launch_norm_t<T, false, false>(x, nullptr, nullptr, g, nullptr, y, rows, hidden, eps,
+                                          st);
 }
 
 }  // namespace
 
 cudaError_t launch_norm(const void* x, const void* residual_in, void* residual_out,
-                        const void* gamma, void* y, int64_t rows, int64_t hidden, float eps,
-                        arops_dtype dtype, cudaStream_t stream)
+                        const void* gamma, const void* beta, void* y, int64_t rows,
+                        int64_t hidden, float eps, arops_dtype dtype, cudaStream_t stream)
 {
-    const bool add = residual_in != nullptr;
-    if (dtype == AROPS_BF16) {
-        if (add)
-            return launch_norm_t<__nv_bfloat16, true>(x, residual_in, residual_out, gamma, y,
-                                                      rows, hidden, eps, stream);
-        return launch_norm_t<__nv_bfloat16, false>(x, nullptr, nullptr, gamma, y, rows, hidden,
-                                                   eps, stream);
-    }
-    if (add)
-        return launch_norm_t<float, true>(x, residual_in, residual_out, gamma, y, rows, hidden,
-                                          eps, stream);
-    return launch_norm_t<float, false>(x, nullptr, nullptr, gamma, y, rows, hidden, eps, stream);
+    if (dtype == AROPS_BF16)
+        return launch_norm_dt<__nv_bfloat16>(x, residual_in, residual_out, gamma, beta, y, rows,
+                                             hidden, eps, stream);
+    return launch_norm_dt<float>(x, residual_in, residual_out, gamma, beta, y, rows, hidden, eps,
+                                 stream);
 }
 
 }  // namespace arops

@@ -22,11 +22,13 @@ import statistics
 
 import torch
 
-from . import add_rmsnorm, mrope_qk, rmsnorm, set_pdl, set_streaming, swiglu
+from . import (add_layernorm, add_rmsnorm, layernorm, mrope_qk, rmsnorm, set_pdl, set_streaming,
+               swiglu)
 from . import inputs as I
 from .chain import DecodeChain
 
 OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
+EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln")
 
 
 CHAIN_PDL = True
@@ -58,12 +60,28 @@ def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
         nb = 2 * r * (I.N_Q_HEADS + I.N_K_HEADS) * I.HEAD_DIM * 2 + 3 * r * 4
         return ((lambda: mrope_qk(t["q"], t["k"], t["pos"], I.SECTIONS, I.THETA, q_out=qo, k_out=ko)),
                 nb, f"bf16 {r} tokens")
-    if op in ("decode5", "decode256"):
-        b = rows or (5 if op == "decode5" else 256)
-        c = DecodeChain(I.ChainShape(batch=b), device=dev, seed=seed, pdl=CHAIN_PDL)
+    if op == "layernorm":
+        r = rows or 4096
+        t = {k: v.to(dev) for k, v in I.rmsnorm_inputs(r, I.HIDDEN, "bf16", seed).items()}
+        beta = I.normal((I.HIDDEN,), seed + 9, std=0.1).to(dev)
+        y = torch.empty_like(t["x"])
+        return ((lambda: layernorm(t["x"], t["gamma"], beta, I.EPS, out=y)),
+                (2 * r * I.HIDDEN + 2 * I.HIDDEN) * 2, f"bf16 {r}x{I.HIDDEN}")
+    if op == "add_layernorm":
+        r = rows or 4096
+        t = {k: v.to(dev) for k, v in I.add_rmsnorm_inputs(r, I.HIDDEN, "bf16", seed).items()}
+        beta = I.normal((I.HIDDEN,), seed + 9, std=0.1).to(dev)
+        y, ro = torch.empty_like(t["x"]), torch.empty_like(t["x"])
+        return ((lambda: add_layernorm(t["x"], t["residual"], t["gamma"], beta, I.EPS, y=y,
+                                       residual_out=ro)),
+                (4 * r * I.HIDDEN + 2 * I.HIDDEN) * 2, f"bf16 {r}x{I.HIDDEN}")
+    if op.startswith("decode"):
+        b = rows or (5 if op.startswith("decode5") else 256)
+        norm = "layer" if op.endswith("_ln") else "rms"
+        c = DecodeChain(I.ChainShape(batch=b), device=dev, seed=seed, pdl=CHAIN_PDL, norm=norm)
         c.capture()
         c.set_position(7)
-        return (lambda: c._graph.replay()), c.bytes_per_step(), f"28 layers, batch {b}, graph"
+        return (lambda: c._graph.replay()), c.bytes_per_step(), f"28 layers, batch {b}, {norm}norm, graph"
     raise ValueError(op)
 
 
@@ -91,7 +109,7 @@ def time_op(fns, iters: int) -> list[float]:
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", default="all", choices=("all",) + OPS)
+    ap.add_argument("--op", default="all", choices=("all",) + OPS + EXTRA_OPS)
     ap.add_argument("--iters", type=int, default=50)
     ap.add_argument("--rows", type=int, default=None)
     ap.add_argument("--copies", type=int, default=None,

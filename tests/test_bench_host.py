@@ -92,3 +92,17 @@ def test_traffic_record_tracks_kernel_source(tmp_path):
 def test_hbm_peak_source():
     peak, kind = bench.measured_hbm_peak()
     assert kind in ("measured", "fallback") and peak > 1000
+
+
+@pytest.mark.parametrize("norm", ["rms", "layer"])
+def test_decode_calls_group_by_operator(norm):
+    """The bench's attribution groups a step's 112 launches as 56 norms, 28
+    M-RoPE, 28 SwiGLU (CPU buffers: only the grouping is exercised)."""
+    from swiglu_ar_tts_b200.inputs import decode_chain_inputs
+
+    shape = ChainShape(batch=5)
+    c = DecodeChain(shape, device="cpu", host_inputs=decode_chain_inputs(shape), norm=norm)
+    groups = bench.group_decode_calls(c)
+    norm_op = "add_layernorm" if norm == "layer" else "add_rmsnorm"
+    assert {k: len(v) for k, v in groups.items()} == {norm_op: 56, "mrope_qk": 28, "swiglu": 28}
+    assert all(bench.KERNEL_OF[k] for k in groups)

@@ -95,3 +95,28 @@ def test_launch_count_per_step():
     chain.step(0)
     torch.cuda.synchronize()
     assert ops.launch_count() - before == 12 == chain.launches_per_step
+
+
+def test_decode_chain_layernorm_variant():
+    """The LayerNorm decode chain (add + LayerNorm in place of add + RMSNorm):
+    residual bit-exact and every output within tolerance over 3 steps."""
+    chain = DecodeChain(ChainShape(batch=5, layers=6), norm="layer")
+    orc = oracle.get()
+    inp = _oracle_inputs(chain)
+    res = to_f64(chain.residual0.cpu())
+    for s in range(3):
+        chain.step(s)
+        res, outs = orc.decode_step(res, inp, s, chain.eps, chain.theta, chain.sections, "bf16",
+                                    norm="layer")
+        torch.cuda.synchronize()
+        assert np.array_equal(to_f64(chain.residual), res)
+        for l in range(chain.shape.layers):
+            check(chain.act[l], outs["act"][l], "bf16")
+            # y = (r - mean) * rstd * gamma + beta; cancellation scale
+            # (|r - mean| rstd + 1) |gamma| + |beta| = |y - beta| + |gamma| + |beta|
+            for name in ("y_attn", "y_mlp"):
+                key = "attn" if name == "y_attn" else "mlp"
+                beta, gamma = inp["beta_" + key][l], inp["gamma_" + key][l]
+                check(getattr(chain, name)[l], outs[name][l], "bf16",
+                      np.abs(outs[name][l] - beta) + np.abs(gamma) + np.abs(beta),
+                      what=f"{name}[{l}]")

@@ -160,3 +160,88 @@ def test_add_rmsnorm_x_zero_reduces_to_rmsnorm():
     y2 = ops.rmsnorm(r, g, EPS)
     torch.cuda.synchronize()
     assert torch.equal(r_out, r) and torch.equal(y, y2)
+
+
+# ---------------------------------------------------------------------------
+# LayerNorm and residual add + LayerNorm
+# ---------------------------------------------------------------------------
+
+
+def _ln_scale(xr: np.ndarray, gamma: np.ndarray, beta: np.ndarray, eps: float) -> np.ndarray:
+    """(|x - mean| r + 1) |gamma| + |beta|, r = 1/sqrt(var + eps): the size of the
+    operands of each output, used as its cancellation scale (tolerance.check).
+    The kernel sums the row shifted by its first element, so the fp32 error of
+    x - mean is of the order of the row's spread (the "+ 1", one standard
+    deviation times r), whatever the row's offset."""
+    mean = xr.mean(axis=-1, keepdims=True)
+    r = 1.0 / np.sqrt(((xr - mean) ** 2).mean(axis=-1, keepdims=True) + eps)
+    return (np.abs(xr - mean) * r + 1.0) * np.abs(gamma) + np.abs(beta)
+
+
+def _ln_inputs(rows, hidden, dtype, seed):
+    inp = inputs.add_rmsnorm_inputs(rows, hidden, dtype, seed)
+    inp["beta"] = inputs.normal((hidden,), seed + 3, std=0.1, dtype=dtype)
+    return inp
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", HIDDEN)
+def test_layernorm_shapes(dtype, hidden):
+    rows = 21 if hidden <= 16384 else 3
+    inp = _ln_inputs(rows, hidden, dtype, hidden + 7)
+    # a shifted input (mean far from 0) exercises the two-pass variance
+    x = (inp["x"].float() + 3.0).to(inp["x"].dtype)
+    y = ops.layernorm(dev(x), dev(inp["gamma"]), dev(inp["beta"]), EPS)
+    torch.cuda.synchronize()
+    exact = oracle.get().layernorm(x, inp["gamma"], inp["beta"], EPS)
+    scale = _ln_scale(to_f64(x), to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
+    check(y, exact, dtype, scale, what=f"layernorm {dtype} {rows}x{hidden}")
+
+
+@pytest.mark.parametrize("in_place", [False, True])
+def test_add_layernorm_bf16_4096x2048(in_place):
+    inp = _ln_inputs(4096, 2048, "bf16", 0)
+    x, r = dev(inp["x"]), dev(inp["residual"])
+    r_out = r if in_place else torch.empty_like(r)
+    y, r_out = ops.add_layernorm(x, r, dev(inp["gamma"]), dev(inp["beta"]), EPS, residual_out=r_out)
+    torch.cuda.synchronize()
+    y_exact, r_exact = oracle.get().add_layernorm(inp["x"], inp["residual"], inp["gamma"],
+                                                  inp["beta"], EPS, "bf16")
+    assert np.array_equal(to_f64(r_out), r_exact), "residual_out must be bit-exact"
+    scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
+    check(y, y_exact, "bf16", scale, what="add_layernorm 4096x2048")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", [8, 2048, 100, 40000, 16384])
+def test_add_layernorm_shapes(dtype, hidden):
+    rows = 9
+    inp = _ln_inputs(rows, hidden, dtype, hidden + 11)
+    y, r_out = ops.add_layernorm(dev(inp["x"]), dev(inp["residual"]), dev(inp["gamma"]),
+                                 dev(inp["beta"]), EPS, residual_out=torch.empty_like(dev(inp["x"])))
+    torch.cuda.synchronize()
+    y_exact, r_exact = oracle.get().add_layernorm(inp["x"], inp["residual"], inp["gamma"],
+                                                  inp["beta"], EPS, dtype)
+    assert np.array_equal(to_f64(r_out), r_exact)
+    scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
+    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}")
+
+
+def test_layernorm_constant_rows_give_beta_and_guarded():
+    """A constant row normalises to exactly beta (zero deviation)."""
+    hidden = 2048
+    beta = inputs.normal((hidden,), 5, std=0.1, dtype="bf16")
+    x = torch.full((6, hidden), 1.75, dtype=torch.bfloat16)
+    out = Guarded((6, hidden), torch.bfloat16, offset=1)
+    ops.layernorm(dev(x), dev(torch.ones(hidden, dtype=torch.bfloat16)), dev(beta), EPS, out=out.t)
+    torch.cuda.synchronize()
+    out.check()
+    assert torch.equal(out.t.cpu(), beta.expand(6, hidden))
+
+
+def test_layernorm_misaligned():
+    inp = _ln_inputs(5, 2048, "bf16", 31)
+    y = ops.layernorm(misaligned(dev(inp["x"])), dev(inp["gamma"]), misaligned(dev(inp["beta"])), EPS)
+    torch.cuda.synchronize()
+    exact = oracle.get().layernorm(inp["x"], inp["gamma"], inp["beta"], EPS)
+    check(y, exact, "bf16", _ln_scale(to_f64(inp["x"]), to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS))

@@ -93,6 +93,9 @@ class Oracle:
         L.oracle_add_layernorm.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_double_p,
                                            _c_double_p, _c_double_p, ctypes.c_int64,
                                            ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+        L.oracle_topk_sample.argtypes = [_c_double_p, ctypes.POINTER(ctypes.c_float), _c_i32_p,
+                                         _c_double_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_float, ctypes.c_void_p]
         L.oracle_mutant.restype = ctypes.c_int
         assert L.oracle_mutant() == mutant
 
@@ -208,6 +211,25 @@ class Oracle:
         self._lib.oracle_swiglu(_ptr(gate, _c_double_p), _ptr(up, _c_double_p),
                                 _ptr(out, _c_double_p), gate.size)
         return out
+
+    def topk_sample(self, logits, gumbel, top_k: int, temperature: float):
+        """Gumbel-max sample from softmax(logits / T) restricted to the top_k
+        logits.  logits [B, V]; gumbel [B, top_k] fp32 (draw j goes to the j-th
+        largest logit).  Returns (token int32 [B], probability fp64 [B])."""
+        logits = _f64(logits)
+        g = np.ascontiguousarray(gumbel.detach().cpu().numpy() if hasattr(gumbel, "detach")
+                                 else gumbel, dtype=np.float32)
+        rows, vocab = logits.shape
+        k = int(top_k)
+        assert g.shape == (rows, k) and 1 <= k <= vocab
+        tok = np.empty(rows, dtype=np.int32)
+        prob = np.empty(rows, dtype=np.float64)
+        scratch = ctypes.create_string_buffer(16 * k)
+        self._lib.oracle_topk_sample(_ptr(logits, _c_double_p),
+                                     g.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                     _ptr(tok, _c_i32_p), _ptr(prob, _c_double_p), rows, vocab, k,
+                                     float(temperature), ctypes.cast(scratch, ctypes.c_void_p))
+        return tok, prob
 
     # -- decode-step chain ---------------------------------------------------
     def decode_step(self, residual, layer_inputs: dict, step: int, eps: float = 1e-6,

@@ -323,6 +323,80 @@ void oracle_swiglu(const double* gate, const double* up, double* out, int64_t n)
     }
 }
 
+/* ------------------------------------------------------------------------- */
+/* Fused softmax + top-k sampling ("Optimising autoregressive speech models",  */
+/* "Custom Triton kernels", item 2: scale the logits by 1/temperature, softmax */
+/* them and sample from the top k).                                            */
+/*                                                                             */
+/* Per row: candidates are the k largest logits, ordered by (logit desc, index */
+/* asc), so ties go to the lower vocabulary index.  Rank j of that order gets  */
+/* the caller's Gumbel(0,1) draw gumbel[row*k + j]; the sampled candidate is   */
+/* the one with the largest score fl32(fl32(logit/T) + g) (ties to the lower   */
+/* rank) -- Gumbel-max sampling from the top-k softmax.  The score is formed   */
+/* with two correctly rounded fp32 operations, the precision the kernel takes  */
+/* this integer decision in.  prob_out is the probability of the sampled token */
+/* under softmax(logits/T) restricted to the k candidates, in fp64.            */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    double v;
+    int64_t idx;
+} cand_t;
+
+/* insertion into a list kept in (v desc, idx asc) order, at most k long */
+static void cand_insert(cand_t* list, int* n, int k, double v, int64_t idx)
+{
+    int pos = *n;
+    while (pos > 0 && (list[pos - 1].v < v || (list[pos - 1].v == v && list[pos - 1].idx > idx)))
+        --pos;
+    if (pos >= k)
+        return;
+    int last = (*n < k) ? *n : k - 1;
+    for (int i = last; i > pos; --i)
+        list[i] = list[i - 1];
+    list[pos].v = v;
+    list[pos].idx = idx;
+    if (*n < k)
+        ++*n;
+}
+
+void oracle_topk_sample(const double* logits, const float* gumbel, int32_t* token_out,
+                        double* prob_out, int64_t rows, int64_t vocab, int k, float temperature,
+                        cand_t* scratch /* k entries */)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* lr = logits + r * vocab;
+        int n = 0;
+        for (int64_t i = 0; i < vocab; ++i)
+            cand_insert(scratch, &n, k, lr[i], i);
+        /* decision in fp32, as fl(fl(l / T) + g) */
+        int best = 0;
+        float best_score = 0.0f;
+        for (int j = 0; j < n; ++j) {
+            volatile float q = (float)scratch[j].v / temperature;
+#if ORACLE_MUTANT == 15
+            volatile float score = q - gumbel[r * k + j]; /* planted: noise subtracted */
+#else
+            volatile float score = q + gumbel[r * k + j];
+#endif
+            if (j == 0 || score > best_score) {
+                best = j;
+                best_score = score;
+            }
+        }
+        /* probability under the top-k softmax, fp64 */
+        double zsum = 0.0;
+        for (int j = 0; j < n; ++j)
+            zsum += exp((scratch[j].v - scratch[0].v) / (double)temperature);
+#if ORACLE_MUTANT == 16
+        double p = exp(scratch[best].v - scratch[0].v) / zsum; /* planted: temperature dropped */
+#else
+        double p = exp((scratch[best].v - scratch[0].v) / (double)temperature) / zsum;
+#endif
+        token_out[r] = (int32_t)scratch[best].idx;
+        prob_out[r] = p;
+    }
+}
+
 /* Number of the planted mistake this build carries (0 = none). */
 int oracle_mutant(void)
 {

@@ -285,6 +285,69 @@ def pin_add_layernorm_is_add_then_norm(orc):
 
 
 # ---------------------------------------------------------------------------
+# fused softmax + top-k sampling
+# ---------------------------------------------------------------------------
+
+
+def pin_topk_greedy_cases(orc):
+    """k = 1, or zero noise, is greedy decoding: the (first) largest logit, with
+    probability 1 for k = 1; ties go to the lower index."""
+    rng = np.random.default_rng(70)
+    lg = rng.standard_normal((4, 300))
+    lg[2, 17] = lg[2, 200] = 9.0  # a tie for the maximum
+    g = rng.gumbel(size=(4, 1)).astype(np.float32)
+    tok, prob = orc.topk_sample(lg, g, 1, 0.7)
+    assert list(tok) == [int(np.argmax(r)) for r in lg] and tok[2] == 17
+    assert np.all(prob == 1.0)
+    tok, _ = orc.topk_sample(lg, np.zeros((4, 40), np.float32), 40, 1.3)
+    assert list(tok) == [int(np.argmax(r)) for r in lg]
+
+
+def pin_topk_probability_closed_form(orc):
+    """Logits (0, ln 2, ln 3, -inf-ish ...) with k = 3, T = 1: the top-3 softmax is
+    (3, 2, 1)/6 for indices (2, 1, 0); a dominant noise on rank j picks rank j."""
+    lg = np.array([[0.0, math.log(2.0), math.log(3.0), -50.0, -60.0]])
+    for j, (idx, p) in enumerate(((2, 0.5), (1, 1 / 3), (0, 1 / 6))):
+        g = np.zeros((1, 3), np.float32)
+        g[0, j] = 100.0
+        tok, prob = orc.topk_sample(lg, g, 3, 1.0)
+        assert tok[0] == idx
+        assert abs(prob[0] - p) < 1e-15
+    # temperature 2 on logits (0, ln 4): top-2 softmax of (0, ln 2) = (1/3, 2/3)
+    g = np.array([[0.0, 100.0]], np.float32)
+    tok, prob = orc.topk_sample(np.array([[0.0, math.log(4.0)]]), g, 2, 2.0)
+    assert tok[0] == 0 and abs(prob[0] - 1 / 3) < 1e-15
+
+
+def pin_topk_gumbel_max_distribution(orc):
+    """Gumbel-max with i.i.d. Gumbel(0,1) draws samples the top-k softmax: over
+    40,000 draws the token frequencies match the probabilities (chi-square)."""
+    rng = np.random.default_rng(71)
+    lg = np.array([[1.0, 0.2, 2.0, -1.0, 1.5, 0.0, -3.0, 0.7]])
+    k, T, n = 5, 0.8, 40_000
+    top = np.argsort(-lg[0], kind="stable")[:k]
+    p = np.exp(lg[0, top] / T - np.max(lg[0, top] / T))
+    p /= p.sum()
+    counts = np.zeros(k)
+    toks, _ = orc.topk_sample(np.repeat(lg, n, axis=0), rng.gumbel(size=(n, k)).astype(np.float32), k, T)
+    for i, t in enumerate(top):
+        counts[i] = np.count_nonzero(toks == t)
+    assert counts.sum() == n  # only top-k tokens are ever drawn
+    chi2 = np.sum((counts - n * p) ** 2 / (n * p))
+    assert chi2 < 20.0, (counts, n * p, chi2)  # 4 degrees of freedom: p(chi2 > 20) < 1e-3
+
+
+def pin_topk_candidate_set(orc):
+    """Only the k largest logits can be drawn, whatever the noise."""
+    rng = np.random.default_rng(72)
+    lg = rng.standard_normal((64, 1000))
+    k = 7
+    toks, _ = orc.topk_sample(lg, (rng.gumbel(size=(64, k)) * 5).astype(np.float32), k, 1.0)
+    for r in range(64):
+        assert lg[r, toks[r]] >= np.sort(lg[r])[-k]
+
+
+# ---------------------------------------------------------------------------
 # M-RoPE
 # ---------------------------------------------------------------------------
 SECTIONS = (24, 20, 20)

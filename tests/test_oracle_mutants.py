@@ -25,6 +25,8 @@ MUTANTS = {
     12: "sigmoid without the g factor",
     13: "LayerNorm with the unbiased variance",
     14: "LayerNorm without beta",
+    15: "Gumbel noise subtracted instead of added",
+    16: "sampling probability without the temperature",
 }
 
 

@@ -44,6 +44,7 @@
 #ifndef AROPS_H
 #define AROPS_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -157,6 +158,38 @@ AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out,
 AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
                                     int64_t rows, int64_t inter,
                                     arops_dtype dtype, void* stream);
+
+/*
+ * Fused softmax + top-k sampling ("Optimising autoregressive speech models",
+ * "Custom Triton kernels", item 2: scale logits by 1/temperature, softmax,
+ * sample from the top k; done in one pass over the logits).
+ *
+ * For each row: the candidates are the top_k largest logits, ordered by logit
+ * (descending) then index (ascending); candidate j (0 = largest) is given the
+ * caller's Gumbel(0,1) draw gumbel[row * top_k + j]; the sampled token is the
+ * candidate with the largest fl32(fl32(logit / temperature) + draw) (ties to
+ * the lower j).  That is Gumbel-max sampling from softmax(logits/temperature)
+ * restricted to the top_k candidates; the caller owns the randomness.
+ *   logits     [rows, vocab] dtype (no NaNs)
+ *   gumbel     [rows, top_k] float32 device array
+ *   token_out  [rows] int32: vocabulary index of the sampled token
+ *   prob_out   [rows] float32: its probability under the restricted softmax
+ *   1 <= top_k <= min(64, vocab), vocab <= 262144, rows <= 65535,
+ *   temperature > 0 and finite.
+ *   workspace  device scratch of at least arops_topk_sample_workspace() bytes
+ *              (8-byte aligned, caller-owned; contents need no initialisation
+ *              and are overwritten).  Two calls in flight at once must not
+ *              share one workspace.
+ * Two kernels are enqueued on `stream` (per-slice candidates, then the merge
+ * and the decision).
+ */
+AROPS_API arops_status arops_topk_sample_workspace(int64_t rows, int64_t vocab, int32_t top_k,
+                                                   size_t* bytes);
+AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel,
+                                         int32_t* token_out, float* prob_out, int64_t rows,
+                                         int64_t vocab, int32_t top_k, float temperature,
+                                         arops_dtype dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * Programmatic dependent launch.  When enabled (process-wide, default off),

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "swiglu", "set_pdl",
-    "set_streaming",
+    "set_streaming", "topk_sample", "topk_sample_workspace",
     "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
 ]
@@ -75,6 +75,11 @@ def lib() -> ctypes.CDLL:
         for fn in ("arops_rmsnorm", "arops_add_rmsnorm", "arops_mrope_qk", "arops_swiglu",
                    "arops_layernorm", "arops_add_layernorm"):
             getattr(L, fn).restype = ctypes.c_int
+        L.arops_topk_sample_workspace.argtypes = [_i64, _i64, _i32, ctypes.POINTER(ctypes.c_size_t)]
+        L.arops_topk_sample_workspace.restype = ctypes.c_int
+        L.arops_topk_sample.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i32, ctypes.c_float,
+                                        ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+        L.arops_topk_sample.restype = ctypes.c_int
         L.arops_set_pdl.argtypes = [ctypes.c_int]
         L.arops_set_pdl.restype = ctypes.c_int
         L.arops_set_streaming.argtypes = [ctypes.c_int]
@@ -249,6 +254,49 @@ def swiglu(gate: torch.Tensor, up: torch.Tensor, out: torch.Tensor | None = None
         _check(lib().arops_swiglu(gate.data_ptr(), up.data_ptr(), out.data_ptr(), rows, inter,
                                   code, _stream(gate)))
     return out
+
+
+def topk_sample_workspace(rows: int, vocab: int, top_k: int) -> int:
+    """Bytes of device workspace that topk_sample needs for this shape."""
+    n = ctypes.c_size_t(0)
+    _check(lib().arops_topk_sample_workspace(rows, vocab, top_k, ctypes.byref(n)))
+    return int(n.value)
+
+
+def topk_sample(logits: torch.Tensor, gumbel: torch.Tensor, top_k: int, temperature: float = 1.0,
+                workspace: torch.Tensor | None = None, token_out: torch.Tensor | None = None,
+                prob_out: torch.Tensor | None = None):
+    """Gumbel-max sample from softmax(logits / temperature) restricted to the
+    top_k logits of each row.  logits [rows, vocab] (bf16/f32); gumbel
+    [rows, top_k] float32 Gumbel(0,1) draws, draw j for the j-th largest logit.
+    Returns (token int32 [rows], probability float32 [rows]).  ``workspace`` is
+    a uint8 device tensor of at least topk_sample_workspace() bytes (allocated
+    here if omitted)."""
+    if logits.dim() != 2:
+        raise ValueError("logits must be [rows, vocab]")
+    rows, vocab = logits.shape
+    if token_out is None:
+        token_out = torch.empty(rows, dtype=torch.int32, device=logits.device)
+    if prob_out is None:
+        prob_out = torch.empty(rows, dtype=torch.float32, device=logits.device)
+    need = topk_sample_workspace(rows, vocab, top_k) if rows else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 8), dtype=torch.uint8, device=logits.device)
+    for n, t in (("logits", logits), ("gumbel", gumbel), ("token_out", token_out),
+                 ("prob_out", prob_out), ("workspace", workspace)):
+        _cuda_contig(n, t)
+    if gumbel.dtype != torch.float32 or tuple(gumbel.shape) != (rows, top_k):
+        raise ValueError("gumbel must be float32 [rows, top_k]")
+    if token_out.dtype != torch.int32 or prob_out.dtype != torch.float32:
+        raise ValueError("token_out must be int32 and prob_out float32")
+    code = _dtype_code(logits)
+    with torch.cuda.device(logits.device):
+        _check(lib().arops_topk_sample(logits.data_ptr(), gumbel.data_ptr(), token_out.data_ptr(),
+                                       prob_out.data_ptr(), rows, vocab, int(top_k),
+                                       float(temperature), code, workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(logits)))
+    return token_out, prob_out
 
 
 def set_pdl(enable: bool) -> bool:

@@ -244,6 +244,70 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
                      "arops_swiglu");
 }
 
+}  // extern "C"
+
+namespace {
+
+arops_status topk_check(const char* name, int64_t rows, int64_t vocab, int32_t top_k,
+                        float temperature)
+{
+    if (rows < 0 || vocab <= 0)
+        return fail(AROPS_ERR_INVALID, "%s: bad shape rows=%lld vocab=%lld", name,
+                    (long long)rows, (long long)vocab);
+    if (top_k < 1 || top_k > vocab)
+        return fail(AROPS_ERR_INVALID, "%s: top_k %d must be in [1, vocab]", name, (int)top_k);
+    if (top_k > topk_max_k() || vocab > (int64_t)topk_max_slices() * 4096 || rows > 65535)
+        return fail(AROPS_ERR_UNSUPPORTED,
+                    "%s: supported top_k <= %d, vocab <= %d, rows <= 65535", name, topk_max_k(),
+                    topk_max_slices() * 4096);
+    if (!(temperature > 0.0f) || isinf(temperature))
+        return fail(AROPS_ERR_INVALID, "%s: temperature must be finite and > 0", name);
+    return AROPS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+AROPS_API arops_status arops_topk_sample_workspace(int64_t rows, int64_t vocab, int32_t top_k,
+                                                   size_t* bytes)
+{
+    if (!bytes)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample_workspace: bytes is null");
+    const arops_status st = topk_check("arops_topk_sample_workspace", rows, vocab, top_k, 1.0f);
+    if (st != AROPS_OK)
+        return st;
+    *bytes = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * sizeof(uint64_t);
+    return ok();
+}
+
+AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel,
+                                         int32_t* token_out, float* prob_out, int64_t rows,
+                                         int64_t vocab, int32_t top_k, float temperature,
+                                         arops_dtype dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample: unknown dtype %d", (int)dtype);
+    const arops_status st = topk_check("arops_topk_sample", rows, vocab, top_k, temperature);
+    if (st != AROPS_OK)
+        return st;
+    if (rows == 0)
+        return ok();
+    if (!logits || !gumbel || !token_out || !prob_out || !workspace)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample: null pointer");
+    const size_t need = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * 8u;
+    if (workspace_bytes < need)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample: workspace of %zu bytes < %zu needed",
+                    workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 7u) != 0)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample: workspace not 8-byte aligned");
+    return from_cuda(launch_topk_sample(logits, gumbel, token_out, prob_out, rows, vocab, top_k,
+                                        temperature, dtype, static_cast<uint64_t*>(workspace),
+                                        static_cast<cudaStream_t>(stream)),
+                     "arops_topk_sample");
+}
+
 AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear)
 {
     if (!errors)

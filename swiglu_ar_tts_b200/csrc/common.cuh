@@ -231,4 +231,13 @@ struct MropeArgs {
 
 cudaError_t launch_mrope(const MropeArgs& a, arops_dtype dtype, cudaStream_t stream);
 
+// Fused softmax + top-k sampling (topk.cu).
+int topk_slices(int64_t vocab);
+int topk_max_k();
+int topk_max_slices();
+cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
+                               float* prob_out, int64_t rows, int64_t vocab, int k,
+                               float temperature, arops_dtype dtype, uint64_t* work,
+                               cudaStream_t stream);
+
 }  // namespace arops

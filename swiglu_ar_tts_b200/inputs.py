@@ -104,6 +104,17 @@ def mrope_inputs(tokens: int, n_q_heads: int = N_Q_HEADS, n_k_heads: int = N_K_H
     }
 
 
+def topk_inputs(rows: int, vocab: int, top_k: int, dtype: str = "bf16", seed: int = 0,
+                std: float = 3.0) -> dict:
+    """logits [rows, vocab] ~ N(0, std^2) (seed); gumbel [rows, top_k] float32
+    Gumbel(0,1) draws from default_rng(seed + 1)."""
+    rng = np.random.default_rng(seed + 1)
+    return {
+        "logits": normal((rows, vocab), seed, std=std, dtype=dtype),
+        "gumbel": torch.from_numpy(rng.gumbel(size=(rows, top_k)).astype(np.float32)),
+    }
+
+
 @dataclass
 class ChainShape:
     """Shape of the decode-step chain: per layer add+RMSNorm, M-RoPE on q/k,

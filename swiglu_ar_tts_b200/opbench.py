@@ -23,12 +23,12 @@ import statistics
 import torch
 
 from . import (add_layernorm, add_rmsnorm, layernorm, mrope_qk, rmsnorm, set_pdl, set_streaming,
-               swiglu)
+               swiglu, topk_sample, topk_sample_workspace)
 from . import inputs as I
 from .chain import DecodeChain
 
 OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
-EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln")
+EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln", "topk_sample")
 
 
 CHAIN_PDL = True
@@ -75,6 +75,15 @@ def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
         return ((lambda: add_layernorm(t["x"], t["residual"], t["gamma"], beta, I.EPS, y=y,
                                        residual_out=ro)),
                 (4 * r * I.HIDDEN + 2 * I.HIDDEN) * 2, f"bf16 {r}x{I.HIDDEN}")
+    if op == "topk_sample":
+        r = rows or 5
+        t = {k: v.to(dev) for k, v in I.topk_inputs(r, 151936, 50, "bf16", seed).items()}
+        ws = torch.empty(topk_sample_workspace(r, 151936, 50), dtype=torch.uint8, device=dev)
+        tok = torch.empty(r, dtype=torch.int32, device=dev)
+        prob = torch.empty(r, dtype=torch.float32, device=dev)
+        return ((lambda: topk_sample(t["logits"], t["gumbel"], 50, 0.8, workspace=ws,
+                                     token_out=tok, prob_out=prob)),
+                r * 151936 * 2 + r * 50 * 4 + r * 8, f"bf16 {r}x151936, top-50")
     if op.startswith("decode"):
         b = rows or (5 if op.startswith("decode5") else 256)
         norm = "layer" if op.endswith("_ln") else "rms"

@@ -92,3 +92,23 @@ def test_python_binding_rejects_cpu_tensors():
     x = torch.zeros(2, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.rmsnorm(x, torch.ones(8, dtype=torch.bfloat16))
+
+
+def test_topk_sample_argument_errors(L):
+    import ctypes as C
+
+    n = C.c_size_t(0)
+    assert L.arops_topk_sample_workspace(5, 151936, 50, C.byref(n)) == 0
+    assert n.value == 5 * 38 * 50 * 8
+    assert L.arops_topk_sample_workspace(5, 100, 0, C.byref(n)) == 1
+    assert L.arops_topk_sample_workspace(5, 100, 101, C.byref(n)) == 1
+    assert L.arops_topk_sample_workspace(5, 1000, 65, C.byref(n)) == 2
+    assert L.arops_topk_sample_workspace(5, 262145, 5, C.byref(n)) == 2
+    before = L.arops_launch_count()
+    # workspace too small, null pointers, bad temperature: nothing launched
+    assert L.arops_topk_sample(1, 1, 1, 1, 5, 1000, 5, 1.0, 1, 8, 16, None) == 1
+    assert L.arops_topk_sample(None, 1, 1, 1, 5, 1000, 5, 1.0, 1, 8, 1 << 20, None) == 1
+    assert L.arops_topk_sample(1, 1, 1, 1, 5, 1000, 5, 0.0, 1, 8, 1 << 20, None) == 1
+    assert L.arops_topk_sample(1, 1, 1, 1, 5, 1000, 5, 1.0, 1, 9, 1 << 20, None) == 1  # misaligned
+    assert L.arops_topk_sample(None, None, None, None, 0, 1000, 5, 1.0, 1, None, 0, None) == 0
+    assert L.arops_launch_count() == before

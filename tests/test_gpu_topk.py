@@ -1,0 +1,106 @@
+"""Fused softmax + top-k sampling on the GPU against the oracle: the sampled
+token bit for bit (the decision is taken in fp32 on both sides), its
+probability within the fp32 bound."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import swiglu_ar_tts_b200 as ops
+from swiglu_ar_tts_b200 import inputs
+from gpu_util import Guarded, dev
+from tolerance import to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, k, temp):
+    tok, prob = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, temp)
+    torch.cuda.synchronize()
+    return tok.cpu().numpy(), to_f64(prob)
+
+
+def _check(inp, k, temp, what=""):
+    tok, prob = _run(inp, k, temp)
+    t_ref, p_ref = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, temp)
+    assert np.array_equal(tok, t_ref), f"{what}: tokens differ at {np.flatnonzero(tok != t_ref)[:5]}"
+    np.testing.assert_allclose(prob, p_ref, rtol=1e-5, atol=0, err_msg=what)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("vocab,k", [(1, 1), (63, 5), (4096, 50), (4097, 64), (3072, 1),
+                                     (151936, 50), (262144, 64), (10000, 20)])
+def test_topk_sample_shapes(dtype, vocab, k):
+    inp = inputs.topk_inputs(5, vocab, k, dtype, seed=vocab + k)
+    _check(inp, k, 0.8, f"{dtype} V={vocab} k={k}")
+
+
+@pytest.mark.parametrize("temp", [0.3, 1.0, 1.7])
+def test_topk_sample_temperatures_many_rows(temp):
+    inp = inputs.topk_inputs(257, 20000, 40, "bf16", seed=int(temp * 10))
+    _check(inp, 40, temp, f"T={temp}")
+
+
+def test_topk_sample_ties_go_to_lower_index():
+    """Coarse logits (multiples of 0.5) tie constantly; the candidates and ranks
+    must follow (logit desc, index asc) exactly."""
+    rng = np.random.default_rng(3)
+    lg = torch.from_numpy(np.round(rng.standard_normal((16, 30000)) * 2) / 2).float()
+    for dt in (torch.bfloat16, torch.float32):
+        inp = {"logits": lg.to(dt), "gumbel": torch.from_numpy(rng.gumbel(size=(16, 64)).astype(np.float32))}
+        _check(inp, 64, 1.0, f"ties {dt}")
+        inp["gumbel"] = torch.zeros(16, 64)
+        tok, _ = _run(inp, 64, 1.0)  # no noise: greedy, first index of the maximum
+        assert np.array_equal(tok, np.argmax(lg.to(dt).float().numpy(), axis=1))
+
+
+def test_topk_sample_winner_in_last_slice_and_greedy():
+    inp = inputs.topk_inputs(4, 151936, 8, "bf16", seed=9)
+    lg = inp["logits"].clone()
+    lg[0, -1] = 40.0
+    lg[1, 4095] = 40.0
+    lg[2, 4096] = 40.0
+    lg[3, 0] = 40.0
+    inp["logits"] = lg
+    tok, prob = _run({"logits": lg, "gumbel": torch.zeros(4, 1)}, 1, 1.0)
+    assert list(tok) == [151935, 4095, 4096, 0] and np.all(prob == 1.0)
+    _check(inp, 8, 1.0, "winners at slice edges")
+
+
+def test_topk_sample_distribution():
+    """Over 20,000 rows of one logit vector with fresh draws, the GPU's token
+    frequencies match the top-k softmax (chi-square)."""
+    rng = np.random.default_rng(11)
+    base = rng.standard_normal(1000) * 2
+    n, k, temp = 20000, 6, 0.9
+    lg = torch.from_numpy(np.tile(base, (n, 1))).float()
+    g = torch.from_numpy(rng.gumbel(size=(n, k)).astype(np.float32))
+    tok, _ = _run({"logits": lg, "gumbel": g}, k, temp)
+    top = np.argsort(-base.astype(np.float32), kind="stable")[:k]
+    p = np.exp(base[top] / temp - base[top].max() / temp)
+    p /= p.sum()
+    counts = np.array([np.count_nonzero(tok == t) for t in top])
+    assert counts.sum() == n
+    chi2 = np.sum((counts - n * p) ** 2 / (n * p))
+    assert chi2 < 25.0, (counts, n * p)
+
+
+def test_topk_sample_workspace_is_exact_and_guarded():
+    rows, vocab, k = 5, 50000, 32
+    need = ops.topk_sample_workspace(rows, vocab, k)
+    assert need == rows * ((vocab + 4095) // 4096) * k * 8
+    ws = Guarded((need // 4,), torch.float32)  # canaries on both sides of the workspace
+    inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=12)
+    tok, prob = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.1,
+                                workspace=ws.t.view(torch.uint8))
+    torch.cuda.synchronize()
+    ws.check()
+    t_ref, p_ref = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 1.1)
+    assert np.array_equal(tok.cpu().numpy(), t_ref)
+
+
+def test_topk_sample_empty_rows():
+    lg = torch.empty(0, 100, dtype=torch.bfloat16, device="cuda")
+    tok, prob = ops.topk_sample(lg, torch.empty(0, 4, device="cuda"), 4, 1.0)
+    torch.cuda.synchronize()
+    assert tok.numel() == 0

@@ -192,6 +192,36 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
                                          size_t workspace_bytes, void* stream);
 
 /*
+ * arops_topk_sample without a workspace argument: the same computation and
+ * results, with the scratch taken from a 1 MiB array that the library itself
+ * holds in device memory (a file-scope __device__ array; every GPU that loads
+ * the library keeps it until the process exits).  The paper has no
+ * counterpart: it is here for callers that cannot allocate device memory,
+ * such as code running inside a host application's real-time audio or
+ * streaming callback, where cudaMalloc is not allowed because it can block
+ * and synchronise the device, or a plugin that only receives buffers from a
+ * host that owns all device memory.  This entry point itself allocates
+ * nothing and calls no allocating routine.
+ *   - Limit: rows * ceil(vocab / 4096) * top_k * 8 bytes must not exceed 1 MiB
+ *     (e.g. vocab 151936, top_k 50: up to 68 rows); larger shapes return
+ *     AROPS_ERR_UNSUPPORTED with the numbers in arops_last_error(), before
+ *     anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on the device.
+ *   - All calls share the one array and it keeps the previous call's contents;
+ *     no part of it needs to start at zero, since every slot a call reads is
+ *     written earlier in that same call.  Calls whose kernels overlap on the
+ *     GPU (different streams, different host threads) race on the array:
+ *     serialise them, e.g. by issuing them on one stream.
+ */
+AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float* gumbel,
+                                                 int32_t* token_out, float* prob_out,
+                                                 int64_t rows, int64_t vocab, int32_t top_k,
+                                                 float temperature, arops_dtype dtype,
+                                                 void* stream);
+
+/*
  * Programmatic dependent launch.  When enabled (process-wide, default off),
  * every kernel is launched with the programmatic-stream-serialisation attribute
  * so that it can be scheduled while the previous kernel on the stream drains;

@@ -308,6 +308,39 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
                      "arops_topk_sample");
 }
 
+AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float* gumbel,
+                                                 int32_t* token_out, float* prob_out,
+                                                 int64_t rows, int64_t vocab, int32_t top_k,
+                                                 float temperature, arops_dtype dtype,
+                                                 void* stream)
+{
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample_noalloc: unknown dtype %d", (int)dtype);
+    const arops_status st =
+        topk_check("arops_topk_sample_noalloc", rows, vocab, top_k, temperature);
+    if (st != AROPS_OK)
+        return st;
+    if (rows == 0)
+        return ok();
+    if (!logits || !gumbel || !token_out || !prob_out)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample_noalloc: null pointer");
+    const size_t need = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * 8u;
+    if (need > topk_noalloc_scratch_bytes())
+        return fail(AROPS_ERR_UNSUPPORTED,
+                    "arops_topk_sample_noalloc: this shape needs %zu bytes of scratch "
+                    "(rows x ceil(vocab/4096) x top_k x 8) but the built-in array holds %zu; "
+                    "use arops_topk_sample with a caller workspace",
+                    need, topk_noalloc_scratch_bytes());
+    uint64_t* scratch = nullptr;
+    cudaError_t err = topk_noalloc_scratch(&scratch);
+    if (err != cudaSuccess)
+        return from_cuda(err, "arops_topk_sample_noalloc (scratch address)");
+    return from_cuda(launch_topk_sample(logits, gumbel, token_out, prob_out, rows, vocab, top_k,
+                                        temperature, dtype, scratch,
+                                        static_cast<cudaStream_t>(stream)),
+                     "arops_topk_sample_noalloc");
+}
+
 AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear)
 {
     if (!errors)

@@ -22,6 +22,8 @@
 // is read, so it needs no clearing.
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace arops {
@@ -182,6 +184,51 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
         return err;
     return launch(topk_sample_kernel, dim3((unsigned)rows), dim3(kMergeThreads), 0, stream,
                   (const uint64_t*)work, slices, k, gumbel, temperature, token_out, prob_out);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the workspace lives in this file-scope device
+// array instead of caller memory.  It exists for callers that cannot allocate
+// device memory themselves, e.g. code running inside a host application's
+// real-time audio or streaming callback, where cudaMalloc is off limits
+// because it can block and synchronise the device, or a plugin that is handed
+// buffers by a host application that owns all device memory.  Every GPU that
+// loads the library holds this array until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+
+static __device__ __align__(256) uint64_t g_topk_scratch[kNoAllocScratchBytes / sizeof(uint64_t)];
+
+namespace {
+constexpr int kScratchDevices = 64;
+std::atomic<uint64_t*> g_topk_scratch_addr[kScratchDevices];
+}  // namespace
+
+size_t topk_noalloc_scratch_bytes()
+{
+    return kNoAllocScratchBytes;
+}
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+cudaError_t topk_noalloc_scratch(uint64_t** ptr)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= kScratchDevices)
+        return cudaErrorInvalidDevice;
+    uint64_t* p = g_topk_scratch_addr[dev].load();
+    if (p == nullptr) {
+        err = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_topk_scratch);
+        if (err != cudaSuccess)
+            return err;
+        g_topk_scratch_addr[dev].store(p);
+    }
+    *ptr = p;
+    return cudaSuccess;
 }
 
 }  // namespace arops

@@ -96,6 +96,10 @@ class Oracle:
         L.oracle_topk_sample.argtypes = [_c_double_p, ctypes.POINTER(ctypes.c_float), _c_i32_p,
                                          _c_double_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                          ctypes.c_float, ctypes.c_void_p]
+        L.oracle_mrope_kv_append.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+            _c_i32_p, _c_i32_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int64, _c_i32_p, ctypes.c_double, _c_double_p]
         L.oracle_mutant.restype = ctypes.c_int
         assert L.oracle_mutant() == mutant
 
@@ -202,6 +206,35 @@ class Oracle:
                                        _ptr(y, _c_double_p), _ptr(res_out, _c_double_p), rows,
                                        hidden, float(eps), code)
         return y, res_out
+
+    def mrope_kv_append(self, q, k, v, pos, cache_loc, k_cache, v_cache, sections=(24, 20, 20),
+                        theta: float = 1e6):
+        """q [T, Hq, D], k/v [T, Hkv, D], pos [3, T], cache_loc [2, T] int32
+        (cache row, position); k_cache/v_cache [rows, Hkv, max_seq, D] (their
+        current contents).  Returns (q_out, k_cache', v_cache') in fp64."""
+        q = _f64(q)
+        k = _f64(k)
+        v = _f64(v)
+        kc = _f64(k_cache).copy()
+        vc = _f64(v_cache).copy()
+        pos = np.ascontiguousarray(pos.detach().cpu().numpy() if hasattr(pos, "detach") else pos,
+                                   dtype=np.int32)
+        loc = np.ascontiguousarray(cache_loc.detach().cpu().numpy()
+                                   if hasattr(cache_loc, "detach") else cache_loc, dtype=np.int32)
+        sec = np.ascontiguousarray(sections, dtype=np.int32)
+        tokens, hq, d = q.shape
+        hk = k.shape[1]
+        rows, hk2, max_seq, d2 = kc.shape
+        assert hk2 == hk and d2 == d and v.shape == k.shape and vc.shape == kc.shape
+        assert pos.shape == (3, tokens) and loc.shape == (2, tokens)
+        q_out = np.empty_like(q)
+        k_rot = np.empty_like(k)
+        self._lib.oracle_mrope_kv_append(
+            _ptr(q, _c_double_p), _ptr(k, _c_double_p), _ptr(v, _c_double_p),
+            _ptr(q_out, _c_double_p), _ptr(kc, _c_double_p), _ptr(vc, _c_double_p),
+            _ptr(pos, _c_i32_p), _ptr(loc, _c_i32_p), tokens, hq, hk, d, rows, max_seq,
+            _ptr(sec, _c_i32_p), float(theta), _ptr(k_rot, _c_double_p))
+        return q_out, kc, vc
 
     def swiglu(self, gate, up) -> np.ndarray:
         gate = _f64(gate)

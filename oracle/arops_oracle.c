@@ -305,6 +305,49 @@ void oracle_mrope_qk(const double* q, const double* k, double* q_out, double* k_
 }
 
 /* ------------------------------------------------------------------------- */
+/* M-RoPE fused with the KV-cache append ("Optimising autoregressive speech    */
+/* models", "Custom Triton kernels", item 3: write the new K, V of a token into */
+/* cache[head, position, :]).  q is rotated into q_out; k is rotated and        */
+/* written, and v copied, into slot (cache_loc[0][t], cache_loc[1][t]) = (cache */
+/* row b, position s) of caches laid out [cache_rows][n_kv_heads][max_seq][D].  */
+/* Tokens whose (b, s) fall outside the cache leave it untouched.               */
+/* ------------------------------------------------------------------------- */
+void oracle_mrope_kv_append(const double* q, const double* k, const double* v, double* q_out,
+                            double* k_cache, double* v_cache, const int32_t* pos,
+                            const int32_t* cache_loc, int64_t tokens, int n_q_heads,
+                            int n_kv_heads, int head_dim, int64_t cache_rows, int64_t max_seq,
+                            const int32_t sections[3], double theta, double* k_rot /* T*Hk*D */)
+{
+    for (int64_t t = 0; t < tokens; ++t) {
+        rotate_heads(q, q_out, pos, tokens, t, n_q_heads, head_dim, sections, theta);
+        rotate_heads(k, k_rot, pos, tokens, t, n_kv_heads, head_dim, sections, theta);
+    }
+    for (int64_t t = 0; t < tokens; ++t) {
+        int64_t b = cache_loc[t];
+        int64_t slot = cache_loc[tokens + t];
+#if ORACLE_MUTANT == 17
+        int64_t tmp = b; /* planted: row and position swapped */
+        b = slot;
+        slot = tmp;
+#endif
+        if (b < 0 || b >= cache_rows || slot < 0 || slot >= max_seq)
+            continue;
+        for (int h = 0; h < n_kv_heads; ++h) {
+            int64_t dst = ((b * n_kv_heads + h) * max_seq + slot) * head_dim;
+            int64_t src = (t * n_kv_heads + h) * (int64_t)head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                k_cache[dst + d] = k_rot[src + d];
+#if ORACLE_MUTANT == 18
+                v_cache[dst + d] = k[src + d]; /* planted: k stored as v */
+#else
+                v_cache[dst + d] = v[src + d];
+#endif
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
 /* SwiGLU (section 3 of the Triton fusion post, by name): out = silu(g) * u,   */
 /* silu(g) = g * sigmoid(g) = g / (1 + e^-g).                                  */
 /* ------------------------------------------------------------------------- */

@@ -455,6 +455,57 @@ def pin_mrope_relative_position(orc):
     assert abs(dot((11, 3, 5), (4, 1, 2)) - base) > 1e-6
 
 
+def _kv_case(seed, tokens=4, hq=3, hk=2, rows=3, max_seq=8):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((tokens, hq, D))
+    k = rng.standard_normal((tokens, hk, D))
+    v = rng.standard_normal((tokens, hk, D))
+    kc = rng.standard_normal((rows, hk, max_seq, D))
+    vc = rng.standard_normal((rows, hk, max_seq, D))
+    return q, k, v, kc, vc
+
+
+def pin_kv_append_is_plain_append_at_position_zero(orc):
+    """With every position 0 the rotation is the identity and the operation is
+    the pages' KV-cache append: cache[row][head][slot][:] = new k / v, bit for
+    bit; q passes through; every other slot keeps its contents."""
+    q, k, v, kc, vc = _kv_case(80)
+    pos = np.zeros((3, 4), np.int32)
+    loc = np.array([[0, 2, 1, 2], [5, 0, 7, 3]], np.int32)
+    qo, kc2, vc2 = orc.mrope_kv_append(q, k, v, pos, loc, kc, vc, SECTIONS, THETA)
+    assert np.array_equal(qo, q)
+    want_k, want_v = kc.copy(), vc.copy()
+    for t in range(4):
+        want_k[loc[0, t], :, loc[1, t], :] = k[t]
+        want_v[loc[0, t], :, loc[1, t], :] = v[t]
+    assert np.array_equal(kc2, want_k) and np.array_equal(vc2, want_v)
+
+
+def pin_kv_append_rotates_k_like_q(orc):
+    """The cached k is the rotation M-RoPE gives k at the token's positions (the
+    same rotation q gets); v is copied unrotated; out-of-range slots are skipped."""
+    q, k, v, kc, vc = _kv_case(81)
+    pos = np.array([[3, 100, 7, 0], [1, 2, 3, 4], [9, 9, 9, 9]], np.int32)
+    loc = np.array([[1, 0, 3, 2], [2, 6, 0, -1]], np.int32)  # tokens 2, 3 out of range
+    qo, kc2, vc2 = orc.mrope_kv_append(q, k, v, pos, loc, kc, vc, SECTIONS, THETA)
+    q_ref, k_ref = orc.mrope_qk(q, k, pos, SECTIONS, THETA)
+    assert np.array_equal(qo, q_ref)
+    assert np.array_equal(kc2[1, :, 2], k_ref[0]) and np.array_equal(kc2[0, :, 6], k_ref[1])
+    assert np.array_equal(vc2[1, :, 2], v[0]) and np.array_equal(vc2[0, :, 6], v[1])
+    kc2[1, :, 2] = kc[1, :, 2]
+    kc2[0, :, 6] = kc[0, :, 6]
+    vc2[1, :, 2] = vc[1, :, 2]
+    vc2[0, :, 6] = vc[0, :, 6]
+    assert np.array_equal(kc2, kc) and np.array_equal(vc2, vc)
+    # the cached k of token 1 is k rotated: its pair norms are those of k
+    half = D // 2
+    n_in = k[1, :, :half] ** 2 + k[1, :, half:] ** 2
+    n_out = kc[0, :, 6, :half] ** 2 + kc[0, :, 6, half:] ** 2
+    assert not np.allclose(n_in, n_out)  # the old slot contents differ ...
+    c = orc.mrope_kv_append(q, k, v, pos, loc, kc, vc, SECTIONS, THETA)[1]
+    np.testing.assert_allclose(c[0, :, 6, :half] ** 2 + c[0, :, 6, half:] ** 2, n_in, rtol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # SwiGLU
 # ---------------------------------------------------------------------------

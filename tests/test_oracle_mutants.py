@@ -27,6 +27,8 @@ MUTANTS = {
     14: "LayerNorm without beta",
     15: "Gumbel noise subtracted instead of added",
     16: "sampling probability without the temperature",
+    17: "KV cache row and position swapped",
+    18: "k written into the V cache",
 }
 
 

@@ -151,6 +151,33 @@ AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out,
                                       arops_dtype dtype, void* stream);
 
 /*
+ * M-RoPE fused with the KV-cache append ("Optimising autoregressive speech
+ * models", "Custom Triton kernels", item 3: insert the new K, V of a token at
+ * its position in a cache laid out [head, position, head_dim] per sequence).
+ * In one pass: q is rotated into q_out exactly as arops_mrope_qk does; k is
+ * rotated the same way and written straight into its cache slot; v is copied
+ * into its slot.  Token t's slot is (cache_loc[t], cache_loc[tokens + t]) =
+ * (cache row, position).
+ *   q, q_out      [tokens, n_q_heads, head_dim] dtype
+ *   k, v          [tokens, n_kv_heads, head_dim] dtype
+ *   k_cache, v_cache [cache_rows, n_kv_heads, max_seq, head_dim] dtype
+ *   pos           [3, tokens] int32 (rows t, h, w); cache_loc [2, tokens] int32
+ *   sections/theta/head_dim as for arops_mrope_qk.
+ * A token whose cache row or position is out of range writes no cache slot
+ * (its q is still rotated) and sets AROPS_DEVICE_ERR_BAD_INDEX in the device
+ * error word.  Slots not named by cache_loc are left untouched.  Two tokens
+ * naming one slot race.
+ */
+#define AROPS_DEVICE_ERR_BAD_INDEX 2u
+AROPS_API arops_status arops_mrope_kv_append(const void* q, const void* k, const void* v,
+                                             void* q_out, void* k_cache, void* v_cache,
+                                             const int32_t* pos, const int32_t* cache_loc,
+                                             int64_t tokens, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, int64_t cache_rows, int64_t max_seq,
+                                             const int32_t* sections, float theta,
+                                             arops_dtype dtype, void* stream);
+
+/*
  * SwiGLU activation ("SwiGLU" in the Triton kernel-fusion post, section 3):
  *   out = silu(gate) * up,  silu(g) = g / (1 + e^-g), computed in fp32.
  *   gate, up, out: [rows, inter] dtype, separate tensors (out may be gate or up).

@@ -18,7 +18,8 @@ import threading
 import torch
 
 __all__ = [
-    "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "swiglu", "set_pdl",
+    "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "mrope_kv_append",
+    "swiglu", "set_pdl",
     "set_streaming", "topk_sample", "topk_sample_workspace",
     "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
@@ -68,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.arops_mrope_qk.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32,
                                      ctypes.POINTER(_i32), ctypes.c_float, ctypes.c_int, _vp]
         L.arops_swiglu.argtypes = [_vp, _vp, _vp, _i64, _i64, ctypes.c_int, _vp]
+        L.arops_mrope_kv_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32,
+                                            _i32, _i32, _i64, _i64, ctypes.POINTER(_i32),
+                                            ctypes.c_float, ctypes.c_int, _vp]
+        L.arops_mrope_kv_append.restype = ctypes.c_int
         L.arops_layernorm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.c_float,
                                       ctypes.c_int, _vp]
         L.arops_add_layernorm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
@@ -237,6 +242,39 @@ def mrope_qk(q: torch.Tensor, k: torch.Tensor, pos: torch.Tensor, sections=(24, 
                                     pos.data_ptr(), tokens, hq, k.shape[1], d, sec, float(theta),
                                     code, _stream(q)))
     return q_out, k_out
+
+
+def mrope_kv_append(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+                    cache_loc: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    sections=(24, 20, 20), theta: float = 1e6,
+                    q_out: torch.Tensor | None = None) -> torch.Tensor:
+    """Rotate q (into ``q_out``, default in place) and k with M-RoPE and write
+    the rotated k and the unrotated v of token t into slot
+    (cache_loc[0, t], cache_loc[1, t]) of k_cache / v_cache
+    [cache_rows, n_kv_heads, max_seq, head_dim].  Returns ``q_out``."""
+    if q_out is None:
+        q_out = q
+    for n, t in (("q", q), ("k", k), ("v", v), ("pos", pos), ("cache_loc", cache_loc),
+                 ("k_cache", k_cache), ("v_cache", v_cache), ("q_out", q_out)):
+        _cuda_contig(n, t)
+    tokens, hq, d = q.shape
+    hk = k.shape[1]
+    if (k.shape != (tokens, hk, d) or v.shape != k.shape or q_out.shape != q.shape
+            or k_cache.dim() != 4 or k_cache.shape[1] != hk or k_cache.shape[3] != d
+            or v_cache.shape != k_cache.shape):
+        raise ValueError("shape mismatch")
+    if pos.dtype != torch.int32 or tuple(pos.shape) != (3, tokens):
+        raise ValueError("pos must be int32 [3, tokens]")
+    if cache_loc.dtype != torch.int32 or tuple(cache_loc.shape) != (2, tokens):
+        raise ValueError("cache_loc must be int32 [2, tokens]")
+    code = _dtype_code(q, k, v, q_out, k_cache, v_cache)
+    sec = (_i32 * 3)(*[int(s) for s in sections])
+    with torch.cuda.device(q.device):
+        _check(lib().arops_mrope_kv_append(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), q_out.data_ptr(), k_cache.data_ptr(),
+            v_cache.data_ptr(), pos.data_ptr(), cache_loc.data_ptr(), tokens, hq, hk, d,
+            k_cache.shape[0], k_cache.shape[2], sec, float(theta), code, _stream(q)))
+    return q_out
 
 
 def swiglu(gate: torch.Tensor, up: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:

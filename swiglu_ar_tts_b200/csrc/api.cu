@@ -227,6 +227,63 @@ AROPS_API arops_status arops_mrope_qk(const void* q, const void* k, void* q_out,
     return from_cuda(launch_mrope(a, dtype, static_cast<cudaStream_t>(stream)), "arops_mrope_qk");
 }
 
+AROPS_API arops_status arops_mrope_kv_append(const void* q, const void* k, const void* v,
+                                             void* q_out, void* k_cache, void* v_cache,
+                                             const int32_t* pos, const int32_t* cache_loc,
+                                             int64_t tokens, int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, int64_t cache_rows, int64_t max_seq,
+                                             const int32_t* sections, float theta,
+                                             arops_dtype dtype, void* stream)
+{
+    const char* name = "arops_mrope_kv_append";
+    if (!valid_dtype(dtype))
+        return fail(AROPS_ERR_INVALID, "%s: unknown dtype %d", name, (int)dtype);
+    if (tokens < 0 || n_q_heads < 0 || n_kv_heads < 0 || cache_rows < 0 || max_seq < 0)
+        return fail(AROPS_ERR_INVALID, "%s: negative size", name);
+    if (head_dim <= 0 || head_dim % 2 != 0)
+        return fail(AROPS_ERR_INVALID, "%s: head_dim must be even and > 0 (got %d)", name,
+                    (int)head_dim);
+    if (head_dim > 512)
+        return fail(AROPS_ERR_UNSUPPORTED, "%s: head_dim %d > 512", name, (int)head_dim);
+    if (!sections)
+        return fail(AROPS_ERR_INVALID, "%s: sections is null", name);
+    if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
+        (int64_t)sections[0] + sections[1] + sections[2] != head_dim / 2)
+        return fail(AROPS_ERR_INVALID, "%s: sections [%d,%d,%d] must be >= 0 and sum to %d", name,
+                    (int)sections[0], (int)sections[1], (int)sections[2], (int)head_dim / 2);
+    if (!(theta > 0.0f) || isinf(theta))
+        return fail(AROPS_ERR_INVALID, "%s: theta must be finite and > 0", name);
+    if (tokens == 0 || n_q_heads + n_kv_heads == 0)
+        return ok();
+    if (!pos || (n_q_heads > 0 && (!q || !q_out)) ||
+        (n_kv_heads > 0 && (!k || !v || !k_cache || !v_cache || !cache_loc)))
+        return fail(AROPS_ERR_INVALID, "%s: null pointer", name);
+    if (k_cache == v_cache && n_kv_heads > 0)
+        return fail(AROPS_ERR_INVALID, "%s: k_cache and v_cache are one buffer", name);
+    MropeArgs a;
+    a.q = q;
+    a.k = k;
+    a.q_out = q_out;
+    a.k_out = nullptr;
+    a.pos = pos;
+    a.tokens = tokens;
+    a.n_q_heads = n_q_heads;
+    a.n_k_heads = n_kv_heads;
+    a.head_dim = head_dim;
+    a.sections[0] = sections[0];
+    a.sections[1] = sections[1];
+    a.sections[2] = sections[2];
+    a.theta = theta;
+    AppendArgs x;
+    x.v = v;
+    x.k_cache = k_cache;
+    x.v_cache = v_cache;
+    x.cache_loc = cache_loc;
+    x.cache_rows = cache_rows;
+    x.max_seq = max_seq;
+    return from_cuda(launch_mrope_append(a, x, dtype, static_cast<cudaStream_t>(stream)), name);
+}
+
 AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out, int64_t rows,
                                     int64_t inter, arops_dtype dtype, void* stream)
 {

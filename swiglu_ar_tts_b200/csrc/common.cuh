@@ -231,6 +231,18 @@ struct MropeArgs {
 
 cudaError_t launch_mrope(const MropeArgs& a, arops_dtype dtype, cudaStream_t stream);
 
+// M-RoPE fused with the KV-cache append (mrope.cu).
+struct AppendArgs {
+    const void* v;
+    void* k_cache;  // [cache_rows, n_k_heads, max_seq, head_dim]
+    void* v_cache;
+    const int32_t* cache_loc;  // [2, tokens]: cache row, position
+    int64_t cache_rows;
+    int64_t max_seq;
+};
+cudaError_t launch_mrope_append(const MropeArgs& a, const AppendArgs& x, arops_dtype dtype,
+                                cudaStream_t stream);
+
 // Fused softmax + top-k sampling (topk.cu).
 int topk_slices(int64_t vocab);
 int topk_max_k();

@@ -324,6 +324,202 @@ mrope_scalar_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* _
     }
 }
 
+// ---------------------------------------------------------------------------
+// M-RoPE fused with the KV-cache append ("Custom Triton kernels", item 3:
+// new K, V of a token written into cache[head, position, :]).  One warp per
+// token as in mrope_vec_kernel, over hq + 2*hkv "heads": q heads are rotated
+// into q_out, k heads are rotated straight into their cache slot, v heads are
+// copied into theirs; the rotated k never makes a round trip through memory.
+// A token whose (cache row, position) lies outside the cache writes no cache
+// slot and sets kDeviceErrBadIndex in the library's error word.
+// ---------------------------------------------------------------------------
+constexpr unsigned kDeviceErrBadIndex = 2u;
+
+struct CacheArgs {
+    const int32_t* loc;  // [2, tokens]: cache row, position
+    int64_t rows;
+    int64_t max_seq;
+};
+
+template <typename T, int P, int U>
+__global__ void __launch_bounds__(32 * kWarpsPerCta)
+mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T* v_cache,
+                    const int32_t* __restrict__ pos, int64_t tokens, int hq, int hk,
+                    const __grid_constant__ MropeParams prm, const __grid_constant__ CacheArgs ca,
+                    unsigned* err_word)
+{
+    constexpr int E = Vec<T>::N;
+    constexpr int G = 32 / P;
+    constexpr int HALF = P * E;
+    constexpr int D = 2 * HALF;
+    constexpr int F = (E >= G) ? E / G : 1;
+    const int lane = threadIdx.x & 31;
+    const int pv = lane % P;
+    const int hg = lane / P;
+    const int j0 = pv * E;
+    const int nh = hq + 2 * hk;
+    __shared__ double inv_freq[HALF];
+
+    {
+        const int64_t t0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+        if (lane == 0 && t0 < tokens) {
+            if (hq > 0)
+                prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
+            if (hk > 0) {
+                prefetch_l2(k + (size_t)t0 * hk * D, (uint32_t)(hk * D * sizeof(T)));
+                prefetch_l2(v + (size_t)t0 * hk * D, (uint32_t)(hk * D * sizeof(T)));
+                prefetch_l2_line(ca.loc + t0);
+                prefetch_l2_line(ca.loc + tokens + t0);
+            }
+            prefetch_l2_line(pos + t0);
+            prefetch_l2_line(pos + tokens + t0);
+            prefetch_l2_line(pos + 2 * tokens + t0);
+        }
+    }
+    fill_inv_freq(inv_freq, HALF, prm);
+    pdl_wait();
+    pdl_allow_dependents();
+
+    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < tokens;
+         t += (int64_t)gridDim.x * kWarpsPerCta) {
+        const int32_t pt = __ldg(pos + t);
+        const int32_t ph = __ldg(pos + tokens + t);
+        const int32_t pw = __ldg(pos + 2 * tokens + t);
+        int64_t cb = -1, cs = -1;
+        if (hk > 0) {
+            cb = __ldg(ca.loc + t);
+            cs = __ldg(ca.loc + tokens + t);
+        }
+        const bool in_cache = cb >= 0 && cb < ca.rows && cs >= 0 && cs < ca.max_seq;
+        if (hk > 0 && !in_cache && lane == 0)
+            record_device_error(err_word, kDeviceErrBadIndex);
+
+        uint4 lo[U], hi[U];
+        auto src_of = [&](int h) -> const T* {
+            if (h < hq)
+                return q + ((size_t)t * hq + h) * D;
+            if (h < hq + hk)
+                return k + ((size_t)t * hk + (h - hq)) * D;
+            return v + ((size_t)t * hk + (h - hq - hk)) * D;
+        };
+        auto load_batch = [&](int h0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int h = h0 + u * G;
+                if (h < nh) {
+                    const T* src = src_of(h);
+                    lo[u] = ld_stream(src + j0);
+                    hi[u] = ld_stream(src + HALF + j0);
+                }
+            }
+        };
+        load_batch(hg);
+
+        float cs_[F], sn_[F];
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            const int j = j0 + ((hg * F + f) % E);
+            rope_cos_sin(inv_freq[j], position_of(j, prm, pt, ph, pw), &cs_[f], &sn_[f]);
+        }
+        float c[E], s[E];
+#pragma unroll
+        for (int m = 0; m < E; ++m) {
+            const int src = pv + P * ((m / F) % G);
+            c[m] = __shfl_sync(0xFFFFFFFFu, cs_[m % F], src);
+            s[m] = __shfl_sync(0xFFFFFFFFu, sn_[m % F], src);
+        }
+
+        for (int h0 = hg; h0 < nh; h0 += G * U) {
+            if (h0 != hg)
+                load_batch(h0);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int h = h0 + u * G;
+                if (h >= nh)
+                    continue;
+                if (h >= hq + hk) {  // v: copied unrotated into its cache slot
+                    if (in_cache) {
+                        T* dst = v_cache + (((size_t)cb * hk + (h - hq - hk)) * ca.max_seq + cs) * D;
+                        st_stream(dst + j0, lo[u]);
+                        st_stream(dst + HALF + j0, hi[u]);
+                    }
+                    continue;
+                }
+                float a[E], b[E], oa[E], ob[E];
+                Vec<T>::unpack(lo[u], a);
+                Vec<T>::unpack(hi[u], b);
+#pragma unroll
+                for (int m = 0; m < E; ++m) {
+                    oa[m] = a[m] * c[m] - b[m] * s[m];
+                    ob[m] = b[m] * c[m] + a[m] * s[m];
+                }
+                T* dst;
+                if (h < hq) {
+                    dst = q_out + ((size_t)t * hq + h) * D;
+                } else {
+                    if (!in_cache)
+                        continue;
+                    dst = k_cache + (((size_t)cb * hk + (h - hq)) * ca.max_seq + cs) * D;
+                }
+                st_stream(dst + j0, Vec<T>::pack(oa));
+                st_stream(dst + HALF + j0, Vec<T>::pack(ob));
+            }
+        }
+    }
+}
+
+// Any even head_dim, any alignment: one thread per (token, head, pair).
+template <typename T>
+__global__ void __launch_bounds__(256)
+mrope_append_scalar_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T* v_cache,
+                           const int32_t* __restrict__ pos, int64_t tokens, int hq, int hk,
+                           int half, const __grid_constant__ MropeParams prm,
+                           const __grid_constant__ CacheArgs ca, unsigned* err_word)
+{
+    pdl_wait();
+    pdl_allow_dependents();
+    const int nh = hq + 2 * hk;
+    const int64_t total = tokens * nh * half;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int j = (int)(idx % half);
+        const int h = (int)((idx / half) % nh);
+        const int64_t t = idx / ((int64_t)half * nh);
+        const int64_t d2 = 2 * (int64_t)half;
+        if (h < hq + hk) {
+            const int32_t p = position_of(j, prm, __ldg(pos + t), __ldg(pos + tokens + t),
+                                          __ldg(pos + 2 * tokens + t));
+            float c, s;
+            rope_cos_sin(inv_freq_of(j, prm), p, &c, &s);
+            const T* src = (h < hq) ? q + ((size_t)t * hq + h) * d2 : k + ((size_t)t * hk + (h - hq)) * d2;
+            const float a = load_elem(src + j);
+            const float b = load_elem(src + half + j);
+            T* dst;
+            if (h < hq) {
+                dst = q_out + ((size_t)t * hq + h) * d2;
+            } else {
+                const int64_t cb = __ldg(ca.loc + t), cs = __ldg(ca.loc + tokens + t);
+                if (cb < 0 || cb >= ca.rows || cs < 0 || cs >= ca.max_seq) {
+                    if (j == 0)
+                        record_device_error(err_word, kDeviceErrBadIndex);
+                    continue;
+                }
+                dst = k_cache + (((size_t)cb * hk + (h - hq)) * ca.max_seq + cs) * d2;
+            }
+            store_elem(dst + j, a * c - b * s);
+            store_elem(dst + half + j, b * c + a * s);
+        } else {
+            const int64_t cb = __ldg(ca.loc + t), cs = __ldg(ca.loc + tokens + t);
+            if (cb < 0 || cb >= ca.rows || cs < 0 || cs >= ca.max_seq)
+                continue;
+            const T* src = v + ((size_t)t * hk + (h - hq - hk)) * d2;
+            T* dst = v_cache + (((size_t)cb * hk + (h - hq - hk)) * ca.max_seq + cs) * d2;
+            dst[j] = src[j];
+            dst[half + j] = src[half + j];
+        }
+    }
+}
+
 constexpr int kHeadUnroll = 8;
 
 template <typename T, int P, int U>
@@ -435,7 +631,88 @@ cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStrea
                   (int)a.n_q_heads, (int)a.n_k_heads, half, prm);
 }
 
+template <typename T, int P, int U>
+cudaError_t launch_append_u(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
+                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens, kWarpsPerCta), cap);
+    return launch(mrope_append_kernel<T, P, U>, dim3((unsigned)grid), dim3(32 * kWarpsPerCta), 0,
+                  st, static_cast<const T*>(a.q), static_cast<const T*>(a.k),
+                  static_cast<const T*>(x.v), static_cast<T*>(a.q_out),
+                  static_cast<T*>(x.k_cache), static_cast<T*>(x.v_cache), a.pos, a.tokens,
+                  (int)a.n_q_heads, (int)a.n_k_heads, prm, ca, word);
+}
+
+template <typename T, int P>
+cudaError_t launch_append_p(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
+                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap)
+{
+    constexpr int G = 32 / P;
+    const int passes = (int)ceil_div(a.n_q_heads + 2 * a.n_k_heads, G);
+    if (passes <= 2)
+        return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap);
+    if (passes <= 4)
+        return launch_append_u<T, P, 4>(a, x, prm, ca, word, st, cap);
+    if (passes <= 6)
+        return launch_append_u<T, P, 6>(a, x, prm, ca, word, st, cap);
+    return launch_append_u<T, P, kHeadUnroll>(a, x, prm, ca, word, st, cap);
+}
+
+template <typename T>
+cudaError_t launch_append_t(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
+                            cudaStream_t st)
+{
+    DeviceInfo di;
+    cudaError_t err = current_device_info(&di);
+    if (err != cudaSuccess)
+        return err;
+    unsigned* word = nullptr;
+    err = device_error_word(&word);
+    if (err != cudaSuccess)
+        return err;
+    CacheArgs ca;
+    ca.loc = x.cache_loc;
+    ca.rows = x.cache_rows;
+    ca.max_seq = x.max_seq;
+    constexpr int E = Vec<T>::N;
+    const int half = a.head_dim / 2;
+    const bool aligned = aligned16(a.q) && aligned16(a.q_out) &&
+                         (a.n_k_heads == 0 || (aligned16(a.k) && aligned16(x.v) &&
+                                               aligned16(x.k_cache) && aligned16(x.v_cache)));
+    const int64_t cap = (int64_t)di.sm_count * 64;
+    if (aligned && half % E == 0) {
+        switch (half / E) {
+        case 1: return launch_append_p<T, 1>(a, x, prm, ca, word, st, cap);
+        case 2: return launch_append_p<T, 2>(a, x, prm, ca, word, st, cap);
+        case 4: return launch_append_p<T, 4>(a, x, prm, ca, word, st, cap);
+        case 8: return launch_append_p<T, 8>(a, x, prm, ca, word, st, cap);
+        case 16: return launch_append_p<T, 16>(a, x, prm, ca, word, st, cap);
+        case 32: return launch_append_p<T, 32>(a, x, prm, ca, word, st, cap);
+        default: break;
+        }
+    }
+    const int64_t total = a.tokens * (int64_t)(a.n_q_heads + 2 * a.n_k_heads) * half;
+    const int64_t grid = std::min<int64_t>(ceil_div(total, 256), (int64_t)di.sm_count * 16);
+    return launch(mrope_append_scalar_kernel<T>, dim3((unsigned)grid), dim3(256), 0, st,
+                  static_cast<const T*>(a.q), static_cast<const T*>(a.k),
+                  static_cast<const T*>(x.v), static_cast<T*>(a.q_out),
+                  static_cast<T*>(x.k_cache), static_cast<T*>(x.v_cache), a.pos, a.tokens,
+                  (int)a.n_q_heads, (int)a.n_k_heads, half, prm, ca, word);
+}
+
 }  // namespace
+
+cudaError_t launch_mrope_append(const MropeArgs& a, const AppendArgs& x, arops_dtype dtype,
+                                cudaStream_t stream)
+{
+    MropeParams prm;
+    prm.sec0 = a.sections[0];
+    prm.sec01 = a.sections[0] + a.sections[1];
+    prm.freq_scale = 2.0 * log2((double)a.theta) / (double)a.head_dim;
+    if (dtype == AROPS_BF16)
+        return launch_append_t<__nv_bfloat16>(a, x, prm, stream);
+    return launch_append_t<float>(a, x, prm, stream);
+}
 
 cudaError_t launch_mrope(const MropeArgs& a, arops_dtype dtype, cudaStream_t stream)
 {

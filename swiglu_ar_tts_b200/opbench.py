@@ -23,12 +23,13 @@ import statistics
 import torch
 
 from . import (add_layernorm, add_rmsnorm, layernorm, mrope_qk, rmsnorm, set_pdl, set_streaming,
-               swiglu, topk_sample, topk_sample_workspace)
+               mrope_kv_append, swiglu, topk_sample, topk_sample_workspace)
 from . import inputs as I
 from .chain import DecodeChain
 
 OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
-EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln", "topk_sample")
+EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln", "topk_sample",
+             "mrope_kv_append")
 
 
 CHAIN_PDL = True
@@ -75,6 +76,23 @@ def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
         return ((lambda: add_layernorm(t["x"], t["residual"], t["gamma"], beta, I.EPS, y=y,
                                        residual_out=ro)),
                 (4 * r * I.HIDDEN + 2 * I.HIDDEN) * 2, f"bf16 {r}x{I.HIDDEN}")
+    if op == "mrope_kv_append":
+        r = rows or 4096
+        hq, hk, d = I.N_Q_HEADS, I.N_K_HEADS, I.HEAD_DIM
+        q = I.normal((r, hq, d), seed).to(dev)
+        k = I.normal((r, hk, d), seed + 1).to(dev)
+        v = I.normal((r, hk, d), seed + 2).to(dev)
+        qo = torch.empty_like(q)
+        cache_rows, max_seq = (r, 512) if r <= 256 else (1, r)
+        kc = torch.zeros(cache_rows, hk, max_seq, d, dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        t = torch.arange(r, dtype=torch.int32)
+        loc = (torch.stack([t, torch.full_like(t, 7)]) if r <= 256
+               else torch.stack([torch.zeros_like(t), t])).to(dev)
+        pos = I.mrope_positions(r).to(dev)
+        nb = (2 * r * hq * d + 4 * r * hk * d) * 2 + 3 * r * 4 + 2 * r * 4
+        return ((lambda: mrope_kv_append(q, k, v, pos, loc, kc, vc, I.SECTIONS, I.THETA, q_out=qo)),
+                nb, f"bf16 {r} tokens, cache [{cache_rows},{hk},{max_seq},{d}]")
     if op == "topk_sample":
         r = rows or 5
         t = {k: v.to(dev) for k, v in I.topk_inputs(r, 151936, 50, "bf16", seed).items()}

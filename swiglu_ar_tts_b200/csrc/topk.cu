@@ -10,13 +10,16 @@
 //
 // Two kernels:
 //   topk_slice_kernel   grid (slices, rows): a CTA turns its 4096-logit slice
-//                       into 64-bit keys (order-preserving bits of the value,
-//                       then the inverted index, so that larger keys are larger
-//                       logits and, among equal logits, lower indices), sorts
-//                       them in shared memory (bitonic network) and writes its
-//                       k best keys to the workspace.
-//   topk_sample_kernel  grid (rows): merges the slices' candidates the same
-//                       way, then takes the sampling decision and the
+//                       into keys (order-preserving bits of the value, then the
+//                       inverted position, so that larger keys are larger logits
+//                       and, among equal logits, lower indices: every key is
+//                       distinct; 32 bits for bf16, 48 for fp32), finds its k
+//                       largest with a block-wide radix select in registers and
+//                       shared memory, and writes them to the workspace as
+//                       (value bits, inverted 24-bit vocabulary index) keys.
+//   topk_sample_kernel  grid (rows): selects the row's k largest among the
+//                       slices' candidates the same way, ranks those k by
+//                       counting, then takes the sampling decision and the
 //                       probability for its row.
 // The workspace holds rows x slices x k keys; every slot is written before it
 // is read, so it needs no clearing.
@@ -42,101 +45,257 @@ __device__ __forceinline__ uint32_t order_bits(float v)
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ float value_of(uint64_t key)
+__device__ __forceinline__ float from_order_bits(uint32_t o)
 {
-    const uint32_t o = (uint32_t)(key >> 32);
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 
-__device__ __forceinline__ int64_t index_of(uint64_t key)
+// Keys of the storage type T: the value's order bits, of which a bf16 needs
+// only the top 16 (its low 16 are 0 for positive and 1 for negative values).
+template <typename T>
+struct KeyBits;
+template <>
+struct KeyBits<float> {
+    static constexpr int V = 32;
+    __device__ static uint32_t of(float v) { return order_bits(v); }
+    __device__ static float value(uint32_t k) { return from_order_bits(k); }
+};
+template <>
+struct KeyBits<__nv_bfloat16> {
+    static constexpr int V = 16;
+    __device__ static uint32_t of(float v) { return order_bits(v) >> 16; }
+    __device__ static float value(uint32_t k)
+    {
+        return from_order_bits((k << 16) | ((k & 0x8000u) ? 0u : 0xFFFFu));
+    }
+};
+
+// Candidate keys: value bits above the inverted vocabulary index (24 bits:
+// vocab <= 2^18 < 2^24), so larger keys are larger logits and, among equal
+// logits, lower indices; every key is distinct and 0 is below every logit.
+constexpr int kIndexBits = 24;
+template <typename T>
+__device__ __forceinline__ uint64_t cand_key(float v, int64_t idx)
 {
-    return (int64_t)(uint32_t)~(uint32_t)key;
+    return ((uint64_t)KeyBits<T>::of(v) << kIndexBits) |
+           (uint64_t)((1u << kIndexBits) - 1u - (uint32_t)idx);
+}
+template <typename T>
+__device__ __forceinline__ float cand_value(uint64_t key)
+{
+    return KeyBits<T>::value((uint32_t)(key >> kIndexBits));
+}
+__device__ __forceinline__ int64_t cand_index(uint64_t key)
+{
+    return (int64_t)((1u << kIndexBits) - 1u - (uint32_t)(key & ((1u << kIndexBits) - 1u)));
 }
 
-__device__ __forceinline__ uint64_t make_key(float v, int64_t idx)
-{
-    return ((uint64_t)order_bits(v) << 32) | (uint64_t)(uint32_t)~(uint32_t)idx;
-}
+// Shared state of one block-wide radix select.
+struct SelectState {
+    uint32_t hist[256];
+    uint64_t tau;   // digits of the k-th largest key found so far
+    int need;       // how many keys still to take from the current bin
+    int shift;      // the select ends at this digit: keys with (key >> shift) >= (tau >> shift)
+    int done;
+    int count;      // output slots handed out
+};
 
-// Bitonic sort of n (a power of two) keys in shared memory, descending.
-__device__ void sort_desc(uint64_t* keys, int n)
+// Radix select (most significant 8-bit digit first) of the k largest among
+// the block's BITS-bit keys, all distinct: every thread passes its M keys
+// (`valid` marks real ones).  On return every thread can test a key with selected().
+// A round histograms the digit of the keys that share the digits fixed so
+// far; the bin holding the k-th largest key becomes the next prefix; the
+// select stops once that bin is taken whole, which always happens by the last
+// digit because keys are distinct.  Histogram updates are aggregated across
+// the lanes of a warp that share a digit.
+template <int BITS, int M>
+__device__ void select_top_k(const uint64_t (&key)[M], const bool (&valid)[M], int k,
+                             SelectState& st)
 {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
-                // the pair (lo, hi) of comparator i at this stage
-                const int lo = 2 * i - (i & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = ((lo & size) == 0);
-                const uint64_t a = keys[lo], b = keys[hi];
-                if ((a < b) == desc) {
-                    keys[lo] = b;
-                    keys[hi] = a;
+    static_assert(BITS % 8 == 0 && BITS <= 64, "keys are a whole number of 8-bit digits");
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        st.tau = 0;
+        st.need = k;
+        st.done = 0;
+        st.shift = 0;
+    }
+    for (int shift = BITS - 8; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x)
+            st.hist[i] = 0;
+        __syncthreads();
+        const uint64_t high_mask = (shift + 8 >= 64) ? 0ull : (~0ull << (shift + 8));
+        const uint64_t prefix = st.tau & high_mask;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const bool active = valid[m] && ((key[m] & high_mask) == prefix);
+            const unsigned am = __ballot_sync(0xFFFFFFFFu, active);
+            if (active) {
+                const uint32_t digit = (uint32_t)(key[m] >> shift) & 255u;
+                const unsigned peers = __match_any_sync(am, digit);
+                if (lane == __ffs(peers) - 1)
+                    atomicAdd(&st.hist[digit], (uint32_t)__popc(peers));
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            // bins [8 lane, 8 lane + 8); counts from the top down
+            uint32_t local = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                local += st.hist[8 * lane + b];
+            uint32_t above = local;  // keys in this lane's bins and every higher bin
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, above, o);
+                if (lane + o < 32)
+                    above += v;
+            }
+            const uint32_t higher = above - local;  // keys in higher lanes' bins
+            const int need = st.need;
+            if (higher < (uint32_t)need && above >= (uint32_t)need) {
+                uint32_t run = higher;
+                for (int b = 7; b >= 0; --b) {
+                    const uint32_t h = st.hist[8 * lane + b];
+                    if (run + h >= (uint32_t)need) {
+                        const int rest = need - (int)run;
+                        st.tau |= (uint64_t)(8 * lane + b) << shift;
+                        st.need = rest;
+                        if ((uint32_t)rest == h) {  // the whole bin is taken
+                            st.done = 1;
+                            st.shift = shift;
+                        }
+                        break;
+                    }
+                    run += h;
                 }
             }
         }
+        __syncthreads();
+        if (st.done)
+            break;
     }
-    __syncthreads();
 }
+
+__device__ __forceinline__ bool selected(uint64_t key, const SelectState& st)
+{
+    return (key >> st.shift) >= (st.tau >> st.shift);
+}
+
+constexpr int kPerThread = kSlice / kSliceThreads;  // 16
 
 template <typename T>
 __global__ void __launch_bounds__(kSliceThreads)
 topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices,
                   uint64_t* __restrict__ work)
 {
-    __shared__ uint64_t keys[kSlice];
+    __shared__ SelectState st;
     const int64_t row = blockIdx.y;
     const int64_t first = (int64_t)blockIdx.x * kSlice;
     const T* lr = logits + row * vocab;
+    const int64_t n = (vocab - first < kSlice) ? vocab - first : kSlice;
     // the slice into L2 while the previous kernel drains, one line per thread
     {
         constexpr int kPerLine = 128 / sizeof(T);
-        const int64_t n = (vocab - first < kSlice) ? vocab - first : kSlice;
         if ((int64_t)threadIdx.x * kPerLine < n)
             prefetch_l2_line(lr + first + (int64_t)threadIdx.x * kPerLine);
     }
     pdl_wait();
     pdl_allow_dependents();
-    for (int i = threadIdx.x; i < kSlice; i += kSliceThreads) {
-        const int64_t idx = first + i;
-        keys[i] = (idx < vocab) ? make_key(load_elem(lr + idx), idx) : 0ull;  // 0: below any logit
+    // in-slice keys: value bits above the inverted 16-bit position in the slice
+    constexpr int kLocalBits = KeyBits<T>::V + 16;
+    uint64_t key[kPerThread];
+    float val[kPerThread];
+    bool valid[kPerThread];
+#pragma unroll
+    for (int m = 0; m < kPerThread; ++m) {
+        const int i = threadIdx.x + m * kSliceThreads;
+        valid[m] = i < n;
+        val[m] = valid[m] ? load_elem(lr + first + i) : 0.f;
+        key[m] = valid[m] ? (((uint64_t)KeyBits<T>::of(val[m]) << 16) | (uint64_t)(0xFFFFu - i)) : 0ull;
     }
-    sort_desc(keys, kSlice);
     uint64_t* out = work + (row * slices + blockIdx.x) * (int64_t)k;
-    for (int j = threadIdx.x; j < k; j += kSliceThreads)
-        out[j] = keys[j];
+    if (n <= k) {
+        // the whole slice is a candidate; the unused slots get keys below any logit
+#pragma unroll
+        for (int m = 0; m < kPerThread; ++m) {
+            const int i = threadIdx.x + m * kSliceThreads;
+            if (i < k)
+                out[i] = valid[m] ? cand_key<T>(val[m], first + i) : 0ull;
+        }
+        return;
+    }
+    select_top_k<kLocalBits>(key, valid, k, st);
+    if (threadIdx.x == 0)
+        st.count = 0;
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kPerThread; ++m)
+        if (valid[m] && selected(key[m], st)) {
+            const int slot = atomicAdd(&st.count, 1);
+            if (slot < k)  // exactly k are selected; the test only guards the bound
+                out[slot] = cand_key<T>(val[m], first + threadIdx.x + m * kSliceThreads);
+        }
 }
 
+constexpr int kMergePerThread = kMaxSlices * kMaxTopK / kMergeThreads;  // 8
+
+template <typename T>
 __global__ void __launch_bounds__(kMergeThreads)
 topk_sample_kernel(const uint64_t* __restrict__ work, int slices, int k,
                    const float* __restrict__ gumbel, float temperature,
                    int32_t* __restrict__ token_out, float* __restrict__ prob_out)
 {
-    __shared__ uint64_t keys[kMaxSlices * kMaxTopK];
+    __shared__ SelectState st;
+    __shared__ uint64_t sel[kMaxTopK];
+    __shared__ uint64_t ranked[kMaxTopK];
     __shared__ float e[kMaxTopK];
     const int64_t row = blockIdx.x;
     const int n = slices * k;
-    int np2 = 1;
-    while (np2 < n)
-        np2 <<= 1;
     pdl_wait();
     pdl_allow_dependents();
-    for (int i = threadIdx.x; i < np2; i += kMergeThreads)
-        keys[i] = (i < n) ? work[row * n + i] : 0ull;
-    sort_desc(keys, np2);
+    uint64_t key[kMergePerThread];
+    bool valid[kMergePerThread];
+#pragma unroll
+    for (int m = 0; m < kMergePerThread; ++m) {
+        const int i = threadIdx.x + m * kMergeThreads;
+        // padding keys (0) of short slices are not candidates
+        key[m] = (i < n) ? work[row * n + i] : 0ull;
+        valid[m] = key[m] != 0ull;
+    }
+    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
+    if (threadIdx.x == 0)
+        st.count = 0;
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kMergePerThread; ++m)
+        if (valid[m] && selected(key[m], st)) {
+            const int slot = atomicAdd(&st.count, 1);
+            if (slot < k)
+                sel[slot] = key[m];
+        }
+    __syncthreads();
+    // order the k candidates by counting: rank = number of larger keys
+    if (threadIdx.x < k) {
+        const uint64_t mine = sel[threadIdx.x];
+        int rank = 0;
+        for (int j = 0; j < k; ++j)
+            rank += sel[j] > mine;
+        ranked[rank] = mine;
+    }
+    __syncthreads();
 
     // exp((l_j - l_0) / T) for the k candidates
-    const float l0 = value_of(keys[0]);
+    const float l0 = cand_value<T>(ranked[0]);
     for (int j = threadIdx.x; j < k; j += kMergeThreads)
-        e[j] = expf((value_of(keys[j]) - l0) / temperature);
+        e[j] = expf((cand_value<T>(ranked[j]) - l0) / temperature);
     __syncthreads();
     if (threadIdx.x == 0) {
         int best = 0;
         float best_score = 0.f, z = 0.f;
         for (int j = 0; j < k; ++j) {
             // fl(fl(l / T) + g), two correctly rounded operations
-            const float score = __fadd_rn(__fdiv_rn(value_of(keys[j]), temperature),
+            const float score = __fadd_rn(__fdiv_rn(cand_value<T>(ranked[j]), temperature),
                                           gumbel[row * k + j]);
             if (j == 0 || score > best_score) {
                 best = j;
@@ -144,7 +303,7 @@ topk_sample_kernel(const uint64_t* __restrict__ work, int slices, int k,
             }
             z += e[j];
         }
-        token_out[row] = (int32_t)index_of(keys[best]);
+        token_out[row] = (int32_t)cand_index(ranked[best]);
         prob_out[row] = e[best] / z;
     }
 }
@@ -182,7 +341,11 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
                      static_cast<const float*>(logits), vocab, k, slices, work);
     if (err != cudaSuccess)
         return err;
-    return launch(topk_sample_kernel, dim3((unsigned)rows), dim3(kMergeThreads), 0, stream,
+    if (dtype == AROPS_BF16)
+        return launch(topk_sample_kernel<__nv_bfloat16>, dim3((unsigned)rows), dim3(kMergeThreads),
+                      0, stream, (const uint64_t*)work, slices, k, gumbel, temperature, token_out,
+                      prob_out);
+    return launch(topk_sample_kernel<float>, dim3((unsigned)rows), dim3(kMergeThreads), 0, stream,
                   (const uint64_t*)work, slices, k, gumbel, temperature, token_out, prob_out);
 }
 

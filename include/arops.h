@@ -281,6 +281,16 @@ AROPS_API int arops_set_streaming(int enable);
 #define AROPS_DEVICE_ERR_TIMEOUT 1u
 AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear);
 
+/*
+ * Self-test of the bounded waits used by the streaming kernels: launches one
+ * thread that waits, with limit `timeout_ns` (at most 2 s), for 16 bytes of a
+ * bulk copy that is never issued.  The wait must run out: the kernel writes 1
+ * to *waited_out (a device int32), sets AROPS_DEVICE_ERR_TIMEOUT and returns,
+ * and the context stays usable.  Nothing else is launched or touched.
+ */
+AROPS_API arops_status arops_selftest_wait_timeout(uint64_t timeout_ns, int32_t* waited_out,
+                                                   void* stream);
+
 /* Number of kernels this library has launched in this process (all devices). */
 AROPS_API uint64_t arops_launch_count(void);
 

@@ -414,6 +414,18 @@ AROPS_API arops_status arops_device_errors(uint32_t* errors, int clear)
     return ok();
 }
 
+AROPS_API arops_status arops_selftest_wait_timeout(uint64_t timeout_ns, int32_t* waited_out,
+                                                   void* stream)
+{
+    if (!waited_out)
+        return fail(AROPS_ERR_INVALID, "arops_selftest_wait_timeout: waited_out is null");
+    if (timeout_ns == 0 || timeout_ns > 2000000000ull)
+        return fail(AROPS_ERR_INVALID, "arops_selftest_wait_timeout: timeout must be in (0, 2 s]");
+    return from_cuda(launch_wait_timeout_selftest(timeout_ns, waited_out,
+                                                  static_cast<cudaStream_t>(stream)),
+                     "arops_selftest_wait_timeout");
+}
+
 AROPS_API int arops_set_pdl(int enable)
 {
     return g_pdl.exchange(enable ? 1 : 0);

@@ -251,6 +251,10 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
                                float* prob_out, int64_t rows, int64_t vocab, int k,
                                float temperature, arops_dtype dtype, uint64_t* work,
                                cudaStream_t stream);
+// Self-test of the bounded mbarrier wait (selftest.cu).
+cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* waited_out,
+                                         cudaStream_t stream);
+
 // The allocation-free variant's built-in scratch array: its size, and its
 // device address on the current device.
 size_t topk_noalloc_scratch_bytes();

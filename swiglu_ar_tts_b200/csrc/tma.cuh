@@ -72,14 +72,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Waits for phase `parity` of `bar` to complete; false if it has not after
-// kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+// `timeout_ns` (kWaitTimeoutNs unless given).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t timeout_ns = kWaitTimeoutNs)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitTimeoutNs)
+        if (global_timer_ns() - t0 > timeout_ns)
             return false;
     }
     return true;

@@ -13,7 +13,10 @@
 // `pv` of a head owns the 16-byte vector x[pv*E .. pv*E+E) of the first half
 // and its partner vector of the second half; G = 32/P heads are covered per
 // warp pass and up to U passes are loaded before any math, so each lane keeps
-// 2*U 16-byte loads in flight.  The angle is formed in fp64 and reduced modulo
+// 2*U 16-byte loads in flight.  A token's passes may be shared by `splits`
+// warps (warp s of the token takes passes s, s + splits, ...): few tokens, as
+// in a decode step, then spread over many warps instead of queueing every pass
+// of a token behind one warp.  The angle is formed in fp64 and reduced modulo
 // 2*pi (|k * 2pi rounding| <= 1e-13 rad for the positions used here) before the
 // fp32 sincosf, so cos/sin carry ~1e-7 absolute error at any position.
 #include <math.h>
@@ -68,7 +71,7 @@ constexpr int kWarpsPerCta = 4;
 template <typename T, int P, int U>
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __restrict__ pos,
-                 int64_t tokens, int hq, int hk, const __grid_constant__ MropeParams prm)
+                 int64_t tokens, int hq, int hk, int splits, const __grid_constant__ MropeParams prm)
 {
     constexpr int E = Vec<T>::N;
     constexpr int G = 32 / P;                // heads per warp pass
@@ -83,10 +86,12 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     __shared__ double inv_freq[HALF];
 
     // this warp's first token (q and k heads, positions) into L2 while the
-    // previous kernel drains
+    // previous kernel drains; of the warps that share a token, the first asks
+    const int64_t units = tokens * splits;
+    const int64_t unit0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     {
-        const int64_t t0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-        if (lane == 0 && t0 < tokens) {
+        const int64_t t0 = unit0 / splits;
+        if (lane == 0 && unit0 < units && unit0 % splits == 0) {
             if (hq > 0)
                 prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
             if (hk > 0)
@@ -100,8 +105,9 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     pdl_wait();
     pdl_allow_dependents();
 
-    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < tokens;
-         t += (int64_t)gridDim.x * kWarpsPerCta) {
+    for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
+        const int64_t t = unit / splits;
+        const int h_first = hg + (int)(unit % splits) * G * U;
         const int32_t pt = __ldg(pos + t);
         const int32_t ph = __ldg(pos + tokens + t);
         const int32_t pw = __ldg(pos + 2 * tokens + t);
@@ -121,7 +127,7 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
                 }
             }
         };
-        load_batch(hg);
+        load_batch(h_first);
 
         // this lane's share of the E angles of block pv ...
         float cs[F], sn[F];
@@ -139,8 +145,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
             s[m] = __shfl_sync(0xFFFFFFFFu, sn[m % F], src);
         }
 
-        for (int h0 = hg; h0 < nh; h0 += G * U) {
-            if (h0 != hg)
+        for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
+            if (h0 != h_first)
                 load_batch(h0);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -344,7 +350,7 @@ struct CacheArgs {
 template <typename T, int P, int U>
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T* v_cache,
-                    const int32_t* __restrict__ pos, int64_t tokens, int hq, int hk,
+                    const int32_t* __restrict__ pos, int64_t tokens, int hq, int hk, int splits,
                     const __grid_constant__ MropeParams prm, const __grid_constant__ CacheArgs ca,
                     unsigned* err_word)
 {
@@ -360,9 +366,11 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     const int nh = hq + 2 * hk;
     __shared__ double inv_freq[HALF];
 
+    const int64_t units = tokens * splits;
+    const int64_t unit0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     {
-        const int64_t t0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-        if (lane == 0 && t0 < tokens) {
+        const int64_t t0 = unit0 / splits;
+        if (lane == 0 && unit0 < units && unit0 % splits == 0) {
             if (hq > 0)
                 prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
             if (hk > 0) {
@@ -380,8 +388,9 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     pdl_wait();
     pdl_allow_dependents();
 
-    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < tokens;
-         t += (int64_t)gridDim.x * kWarpsPerCta) {
+    for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
+        const int64_t t = unit / splits;
+        const int h_first = hg + (int)(unit % splits) * G * U;
         const int32_t pt = __ldg(pos + t);
         const int32_t ph = __ldg(pos + tokens + t);
         const int32_t pw = __ldg(pos + 2 * tokens + t);
@@ -413,7 +422,7 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
                 }
             }
         };
-        load_batch(hg);
+        load_batch(h_first);
 
         float cs_[F], sn_[F];
 #pragma unroll
@@ -429,8 +438,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
             s[m] = __shfl_sync(0xFFFFFFFFu, sn_[m % F], src);
         }
 
-        for (int h0 = hg; h0 < nh; h0 += G * U) {
-            if (h0 != hg)
+        for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
+            if (h0 != h_first)
                 load_batch(h0);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -523,22 +532,33 @@ mrope_append_scalar_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_ca
 constexpr int kHeadUnroll = 8;
 
 template <typename T, int P, int U>
-cudaError_t launch_vec_u(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
+cudaError_t launch_vec_u(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap,
+                         int splits = 1)
 {
-    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens, kWarpsPerCta), cap);
+    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens * splits, kWarpsPerCta), cap);
     return launch(mrope_vec_kernel<T, P, U>, dim3((unsigned)grid), dim3(32 * kWarpsPerCta), 0, st,
                   static_cast<const T*>(a.q), static_cast<const T*>(a.k),
                   static_cast<T*>(a.q_out), static_cast<T*>(a.k_out), a.pos, a.tokens,
-                  (int)a.n_q_heads, (int)a.n_k_heads, prm);
+                  (int)a.n_q_heads, (int)a.n_k_heads, splits, prm);
 }
 
-// Heads per lane per pass: just enough passes to cover every head at once (6
-// for 16 + 8 heads of 128), so no registers are held for absent heads.
+// A problem with at most one pass for every warp the GPU holds at once (a
+// decode step: a few tokens) is latency-bound: one pass per warp, the token's
+// passes spread over as many warps.
+inline bool one_pass_per_warp(int64_t tokens, int passes, int64_t cap)
+{
+    return tokens * passes <= cap;
+}
+
+// Otherwise heads per lane per pass: just enough passes to cover every head at
+// once (6 for 16 + 8 heads of 128), so no registers are held for absent heads.
 template <typename T, int P>
 cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
 {
     constexpr int G = 32 / P;
     const int passes = (int)ceil_div(a.n_q_heads + a.n_k_heads, G);
+    if (one_pass_per_warp(a.tokens, passes, cap))
+        return launch_vec_u<T, P, 1>(a, prm, st, cap, passes);
     if (passes <= 2)
         return launch_vec_u<T, P, 2>(a, prm, st, cap);
     if (passes <= 4)
@@ -633,14 +653,15 @@ cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStrea
 
 template <typename T, int P, int U>
 cudaError_t launch_append_u(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
-                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap)
+                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap,
+                            int splits = 1)
 {
-    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens, kWarpsPerCta), cap);
+    const int64_t grid = std::min<int64_t>(ceil_div(a.tokens * splits, kWarpsPerCta), cap);
     return launch(mrope_append_kernel<T, P, U>, dim3((unsigned)grid), dim3(32 * kWarpsPerCta), 0,
                   st, static_cast<const T*>(a.q), static_cast<const T*>(a.k),
                   static_cast<const T*>(x.v), static_cast<T*>(a.q_out),
                   static_cast<T*>(x.k_cache), static_cast<T*>(x.v_cache), a.pos, a.tokens,
-                  (int)a.n_q_heads, (int)a.n_k_heads, prm, ca, word);
+                  (int)a.n_q_heads, (int)a.n_k_heads, splits, prm, ca, word);
 }
 
 template <typename T, int P>
@@ -649,6 +670,8 @@ cudaError_t launch_append_p(const MropeArgs& a, const AppendArgs& x, const Mrope
 {
     constexpr int G = 32 / P;
     const int passes = (int)ceil_div(a.n_q_heads + 2 * a.n_k_heads, G);
+    if (one_pass_per_warp(a.tokens, passes, cap))
+        return launch_append_u<T, P, 1>(a, x, prm, ca, word, st, cap, passes);
     if (passes <= 2)
         return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap);
     if (passes <= 4)

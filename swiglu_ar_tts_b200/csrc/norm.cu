@@ -40,7 +40,8 @@ namespace {
 template <typename T, bool ADD, int THREADS>
 __global__ void __launch_bounds__(THREADS)
 norm_tma_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
-                T* y, int64_t rows, int hidden, float eps, int stages, unsigned* err_word)
+                T* y, int64_t rows, int hidden, float eps, float inv_hidden, int stages,
+                unsigned* err_word)
 {
     constexpr int E = Vec<T>::N;
     constexpr int W = THREADS / 32;
@@ -141,7 +142,7 @@ norm_tma_kernel(const T* x, const T* residual_in, T* residual_out, const T* __re
 #pragma unroll
         for (int w = 0; w < W; ++w)
             ss += red[w];
-        const float r = rsqrtf(ss / (float)hidden + eps);
+        const float r = rsqrtf(ss * inv_hidden + eps);
 
         for (int v = tid; v < nvec; v += THREADS) {
             float a[E], g[E];
@@ -196,6 +197,10 @@ __device__ __forceinline__ float row_broadcast(float v, float& slot, int tid)
     }
 }
 
+// The mean of a sum is taken as sum * inv_hidden, inv_hidden = fl(1/hidden)
+// computed by the host: a division at that point would sit between the
+// reduction and the output on every row's critical path.
+//
 // LN = false: RMSNorm, y = x * rsqrt(mean(x^2) + eps) * gamma.
 // LN = true:  LayerNorm, y = (x - mean) * rsqrt(mean((x - mean)^2) + eps) * gamma + beta,
 //             the variance taken from the row held in registers (two reductions),
@@ -203,7 +208,8 @@ __device__ __forceinline__ float row_broadcast(float v, float& slot, int tid)
 template <typename T, bool ADD, bool LN, int VPL, int GW>
 __global__ void __launch_bounds__(GW == 1 ? 32 * kRowsPerSmallCta : 32 * GW)
 norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
-                 const T* __restrict__ beta, T* y, int64_t rows, int hidden, float eps)
+                 const T* __restrict__ beta, T* y, int64_t rows, int hidden, float eps,
+                 float inv_hidden)
 {
     constexpr int E = Vec<T>::N;
     constexpr int G = 32 * GW;  // threads per row
@@ -305,7 +311,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
 
         float mean = 0.f, r;  // for LayerNorm: the mean of the shifted row
         if constexpr (LN) {
-            mean = s1 / (float)hidden;
+            mean = s1 * inv_hidden;
             float s2 = 0.f;
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
@@ -321,9 +327,9 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
                 }
             }
             s2 = group_sum<GW>(s2, red, parity, tid);
-            r = rsqrtf(s2 / (float)hidden + eps);
+            r = rsqrtf(s2 * inv_hidden + eps);
         } else {
-            r = rsqrtf(s1 / (float)hidden + eps);
+            r = rsqrtf(s1 * inv_hidden + eps);
         }
 
 #pragma unroll
@@ -360,7 +366,8 @@ constexpr int kLoopThreads = 256;
 template <typename T, bool ADD, bool LN, bool VEC>
 __global__ void __launch_bounds__(kLoopThreads)
 norm_looped_kernel(const T* x, const T* residual_in, T* residual_out, const T* __restrict__ gamma,
-                   const T* __restrict__ beta, T* y, int64_t rows, int64_t hidden, float eps)
+                   const T* __restrict__ beta, T* y, int64_t rows, int64_t hidden, float eps,
+                   float inv_hidden)
 {
     constexpr int E = Vec<T>::N;
     constexpr int W = kLoopThreads / 32;
@@ -424,7 +431,7 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out, const T* _
         const T* src = ADD ? residual_out : x;
         float mean = 0.f, r;
         if constexpr (LN) {
-            mean = s1 / (float)hidden;
+            mean = s1 * inv_hidden;
             float s2 = 0.f;
             if constexpr (VEC) {
                 const int64_t nvec = hidden / E;
@@ -444,9 +451,9 @@ norm_looped_kernel(const T* x, const T* residual_in, T* residual_out, const T* _
                 }
             }
             s2 = group_sum<W>(s2, red, parity, tid);
-            r = rsqrtf(s2 / (float)hidden + eps);
+            r = rsqrtf(s2 * inv_hidden + eps);
         } else {
-            r = rsqrtf(s1 / (float)hidden + eps);
+            r = rsqrtf(s1 * inv_hidden + eps);
         }
 
         if constexpr (VEC) {
@@ -510,7 +517,7 @@ cudaError_t launch_norm_tma_t(const T* x, const T* ri, T* ro, const T* g, T* y, 
         return err;
     const int64_t grid = std::min<int64_t>(rows, (int64_t)di.sm_count * per_sm);
     return launch(kernel, dim3((unsigned)grid), dim3(THREADS), smem, st, x, ri, ro, g, y, rows,
-                  hidden, eps, stages, word);
+                  hidden, eps, 1.0f / (float)hidden, stages, word);
 }
 
 template <typename T, bool ADD>
@@ -531,7 +538,18 @@ cudaError_t launch_rows_gw1(const T* x, const T* ri, T* ro, const T* g, const T*
 {
     const int64_t grid = std::min<int64_t>(ceil_div(rows, kRowsPerSmallCta), cap);
     return launch(norm_rows_kernel<T, ADD, LN, VPL, 1>, dim3((unsigned)grid),
-                  dim3(32 * kRowsPerSmallCta), 0, st, x, ri, ro, g, b, y, rows, hidden, eps);
+                  dim3(32 * kRowsPerSmallCta), 0, st, x, ri, ro, g, b, y, rows, hidden, eps,
+                  1.0f / (float)hidden);
+}
+
+// One 16-byte vector per lane, GW warps per row, one row per CTA.
+template <typename T, bool ADD, bool LN, int GW>
+cudaError_t launch_rows_wide(const T* x, const T* ri, T* ro, const T* g, const T* b, T* y,
+                             int64_t rows, int hidden, float eps, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(rows, cap);
+    return launch(norm_rows_kernel<T, ADD, LN, 1, GW>, dim3((unsigned)grid), dim3(32 * GW), 0,
+                  st, x, ri, ro, g, b, y, rows, hidden, eps, 1.0f / (float)hidden);
 }
 
 template <typename T, bool ADD, bool LN, int GW>
@@ -540,7 +558,7 @@ cudaError_t launch_rows_gwn(const T* x, const T* ri, T* ro, const T* g, const T*
 {
     const int64_t grid = std::min<int64_t>(rows, cap);
     return launch(norm_rows_kernel<T, ADD, LN, 8, GW>, dim3((unsigned)grid), dim3(32 * GW), 0,
-                  st, x, ri, ro, g, b, y, rows, hidden, eps);
+                  st, x, ri, ro, g, b, y, rows, hidden, eps, 1.0f / (float)hidden);
 }
 
 template <typename T, bool ADD, bool LN>
@@ -574,6 +592,20 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
     if (vec) {
         const int64_t nvec = hidden / E;
         const int h = (int)hidden;
+        // A problem that fits one wave at one vector per thread (a decode step's
+        // few rows) is latency-bound: after the dependency wait each warp then
+        // has one load, a few flops and one store per tensor, and the row's
+        // reduction runs across warps, instead of one warp walking the whole row.
+        if (rows * nvec <= (int64_t)di.sm_count * 2048 && nvec > 32) {
+            if (nvec <= 64)
+                return launch_rows_wide<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            if (nvec <= 128)
+                return launch_rows_wide<T, ADD, LN, 4>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            if (nvec <= 256)
+                return launch_rows_wide<T, ADD, LN, 8>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            if (nvec <= 512)
+                return launch_rows_wide<T, ADD, LN, 16>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+        }
         if (nvec <= 32)
             return launch_rows_gw1<T, ADD, LN, 1>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 64)
@@ -594,9 +626,10 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
     const int64_t grid = std::min<int64_t>(rows, cap);
     if (vec)
         return launch(norm_looped_kernel<T, ADD, LN, true>, dim3((unsigned)grid),
-                      dim3(kLoopThreads), 0, st, x, ri, ro, g, b, y, rows, hidden, eps);
+                      dim3(kLoopThreads), 0, st, x, ri, ro, g, b, y, rows, hidden, eps,
+                      1.0f / (float)hidden);
     return launch(norm_looped_kernel<T, ADD, LN, false>, dim3((unsigned)grid), dim3(kLoopThreads),
-                  0, st, x, ri, ro, g, b, y, rows, hidden, eps);
+                  0, st, x, ri, ro, g, b, y, rows, hidden, eps, 1.0f / (float)hidden);
 }
 
 template <typename T>

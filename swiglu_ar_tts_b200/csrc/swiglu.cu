@@ -24,23 +24,50 @@ constexpr int kThreads = 256;
 // below half a bf16 ulp); fp32 storage uses expf and an IEEE divide so that its
 // error stays well inside the 1e-5 relative bound.
 template <typename T>
-__device__ __forceinline__ float silu(float g)
+__device__ __forceinline__ float silu_quotient(float g)
 {
-    if (g < -80.0f)
-        return -expf(g + logf(-g));
     if constexpr (sizeof(T) == 2)
         return __fdividef(g, 1.0f + __expf(-g));
     else
         return g / (1.0f + expf(-g));
 }
 
-template <typename T, int U>
-__global__ void __launch_bounds__(kThreads)
+template <typename T>
+__device__ __forceinline__ float silu(float g)
+{
+    if (g < -80.0f)
+        return -expf(g + logf(-g));
+    return silu_quotient<T>(g);
+}
+
+// out = silu(gate) * up over one vector.  The g < -80 form is taken only by a
+// vector that holds such a g: evaluated element by element, its exp and log
+// would otherwise be paid for every element.
+template <typename T, int E>
+__device__ __forceinline__ void silu_mul(float (&a)[E], const float (&b)[E])
+{
+    float lo = a[0];
+#pragma unroll
+    for (int e = 1; e < E; ++e)
+        lo = fminf(lo, a[e]);
+    if (lo < -80.0f) {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            a[e] = silu<T>(a[e]) * b[e];
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            a[e] = silu_quotient<T>(a[e]) * b[e];
+    }
+}
+
+template <typename T, int U, int THREADS>
+__global__ void __launch_bounds__(THREADS)
 swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
 {
     constexpr int E = Vec<T>::N;
     const int64_t nvec = n / E;
-    const int64_t chunk = (int64_t)kThreads * U;
+    const int64_t chunk = (int64_t)THREADS * U;
 
     // the CTA's first chunk of gate and up into L2 while the previous kernel drains
     if (threadIdx.x == 0) {
@@ -59,7 +86,7 @@ swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
         uint4 g[U], u[U];
 #pragma unroll
         for (int i = 0; i < U; ++i) {
-            const int64_t vi = base + (int64_t)i * kThreads;
+            const int64_t vi = base + (int64_t)i * THREADS;
             if (vi < nvec) {
                 g[i] = ld_stream(gate + vi * E);
                 u[i] = ld_stream(up + vi * E);
@@ -67,14 +94,12 @@ swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
         }
 #pragma unroll
         for (int i = 0; i < U; ++i) {
-            const int64_t vi = base + (int64_t)i * kThreads;
+            const int64_t vi = base + (int64_t)i * THREADS;
             if (vi < nvec) {
                 float a[E], b[E];
                 Vec<T>::unpack(g[i], a);
                 Vec<T>::unpack(u[i], b);
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    a[e] = silu<T>(a[e]) * b[e];
+                silu_mul<T>(a, b);
                 st_stream(out + vi * E, Vec<T>::pack(a));
             }
         }
@@ -163,9 +188,7 @@ swiglu_tma_kernel(const T* gate, const T* up, T* out, int64_t n, int slots, unsi
             float a[E], b[E];
             Vec<T>::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), a);
             Vec<T>::unpack(*reinterpret_cast<const uint4*>(sg + kBytes + (size_t)v * 16), b);
-#pragma unroll
-            for (int e = 0; e < E; ++e)
-                a[e] = silu<T>(a[e]) * b[e];
+            silu_mul<T>(a, b);
             st_stream(out + base + (int64_t)v * E, Vec<T>::pack(a));
         }
         __syncwarp();  // the slot has been read; it can take the next copy
@@ -228,16 +251,23 @@ cudaError_t launch_swiglu_t(const void* gv, const void* uv, void* ov, int64_t n,
     if (aligned) {
         const int64_t nvec = n / E;
         // a problem that fits one wave at one vector per thread (decode batches)
-        // is latency-bound: spread it over as many threads as possible
+        // is latency-bound: one vector per thread.  CTAs of 128 threads (a few
+        // CTAs' worth of vectors per SM at most) or else 512 measured fastest
+        // on B200 for 5 x 6144 and 256 x 6144 in chains of dependent launches.
         if (nvec <= (int64_t)di.sm_count * 2048) {
-            const int64_t grid = std::max<int64_t>(1, ceil_div(nvec, kThreads));
-            return launch(swiglu_vec_kernel<T, 1>, dim3((unsigned)grid), dim3(kThreads), 0, st, g,
+            if (nvec <= (int64_t)di.sm_count * 256) {
+                const int64_t grid = std::max<int64_t>(1, ceil_div(nvec, 128));
+                return launch(swiglu_vec_kernel<T, 1, 128>, dim3((unsigned)grid), dim3(128), 0,
+                              st, g, u, o, n);
+            }
+            const int64_t grid = ceil_div(nvec, 512);
+            return launch(swiglu_vec_kernel<T, 1, 512>, dim3((unsigned)grid), dim3(512), 0, st, g,
                           u, o, n);
         }
         const int64_t want = ceil_div(nvec, (int64_t)kThreads * kUnroll);
         const int64_t grid = std::min<int64_t>(want, (int64_t)INT32_MAX);
-        return launch(swiglu_vec_kernel<T, kUnroll>, dim3((unsigned)grid), dim3(kThreads), 0, st,
-                      g, u, o, n);
+        return launch(swiglu_vec_kernel<T, kUnroll, kThreads>, dim3((unsigned)grid),
+                      dim3(kThreads), 0, st, g, u, o, n);
     }
     const int64_t grid = std::min<int64_t>(ceil_div(n, kThreads), (int64_t)di.sm_count * 8);
     return launch(swiglu_scalar_kernel<T>, dim3((unsigned)grid), dim3(kThreads), 0, st, g, u, o, n);

@@ -48,3 +48,11 @@ def misaligned(t: torch.Tensor, by: int = 1) -> torch.Tensor:
     out.copy_(t)
     assert out.data_ptr() % 16 != 0
     return out
+
+
+def resident_threads() -> int:
+    """Threads the device holds at once (2048 per SM).  The launchers treat a
+    problem of at most one vector (norm, SwiGLU) or one head pass (M-RoPE) per
+    resident thread or warp as latency-bound and lay it out differently; tests
+    size cases on both sides of that line."""
+    return torch.cuda.get_device_properties(0).multi_processor_count * 2048

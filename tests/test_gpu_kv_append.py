@@ -57,7 +57,10 @@ def _run_and_check(q, k, v, kc, vc, pos, loc, dtype, sections=(24, 20, 20), what
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("tokens,rows,max_seq", [(5, 5, 300), (256, 256, 4), (1000, 4, 512), (1, 1, 1)])
+# 2400 tokens hold more (token, head-pass) units than warps resident at once,
+# the others fewer: both layouts of the launcher
+@pytest.mark.parametrize("tokens,rows,max_seq", [(5, 5, 300), (256, 256, 4), (1000, 4, 512), (1, 1, 1),
+                                                 (2400, 8, 512)])
 def test_kv_append_shapes(dtype, tokens, rows, max_seq):
     case = _case(tokens, 16, 8, 128, rows, max_seq, dtype, seed=tokens + rows)
     _run_and_check(*case, dtype, what=f"{dtype} T={tokens}")

@@ -6,7 +6,7 @@ import torch
 import oracle
 import swiglu_ar_tts_b200 as ops
 from swiglu_ar_tts_b200 import inputs
-from gpu_util import Guarded, dev, misaligned
+from gpu_util import Guarded, dev, misaligned, resident_threads
 from tolerance import check, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -106,6 +106,19 @@ def test_mrope_head_counts(hq, hk, family):
     ops.mrope_qk(q, k, pos, SECTIONS, THETA, q_out=qo, k_out=ko)
     torch.cuda.synchronize()
     _compare(qo, ko, inp, what=f"hq={hq} hk={hk}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hq,hk", [(1, 1), (7, 5), (16, 8), (40, 40)])
+def test_mrope_head_counts_past_one_wave(dtype, hq, hk):
+    """More (token, head-pass) units than warps resident at once: each warp then
+    takes whole tokens, U head passes at a time, instead of one pass each."""
+    heads_per_pass = 4 if dtype == "bf16" else 2  # head_dim 128: 32 lanes / (64 / E)
+    passes = -(-(hq + hk) // heads_per_pass)
+    tokens = (resident_threads() // 32) // passes + 5
+    inp = inputs.mrope_inputs(tokens, n_q_heads=hq, n_k_heads=hk, dtype=dtype, seed=hq + 100 * hk)
+    qo, ko = _run(inp)
+    _compare(qo, ko, inp, dtype=dtype, what=f"{dtype} {tokens} tokens hq={hq} hk={hk}")
 
 
 def test_mrope_theta_values():

@@ -6,7 +6,7 @@ import torch
 import oracle
 import swiglu_ar_tts_b200 as ops
 from swiglu_ar_tts_b200 import inputs
-from gpu_util import Guarded, dev, misaligned
+from gpu_util import Guarded, dev, misaligned, resident_threads
 from tolerance import check, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -32,8 +32,21 @@ def test_rmsnorm_f32_64x1024(family):
 
 # hidden sizes cover every kernel variant: 1/2/4/8 vectors per lane with one
 # warp per row, 2/4/8/16 warps per row, the looped vector kernel (> 4096
-# vectors) and the element-wise kernel (hidden not a multiple of the vector)
-HIDDEN = [8, 16, 24, 40, 256, 512, 1000, 1024, 2048, 4104, 8192, 16384, 32768, 40000, 100, 2050, 40001]
+# vectors) and the element-wise kernel (hidden not a multiple of the vector).
+# With few rows (as here) rows of 33 to 512 vectors take one vector per lane
+# over 2 to 16 warps, some lanes idle for 264, 1000 and 4000.
+HIDDEN = [8, 16, 24, 40, 256, 264, 512, 1000, 1024, 2048, 4000, 4104, 8192, 16384, 32768, 40000,
+          100, 2050, 40001]
+
+# Row widths whose layout depends on the row count, run with just more rows
+# than one wave of one vector per thread holds: 8 / 4 vectors per lane, one warp
+# per row, or 2 warps per row for 512 vectors.
+HIDDEN_WIDE = [264, 512, 1000, 1024, 2048, 4000]
+
+
+def rows_past_one_wave(hidden: int, dtype: str) -> int:
+    nvec = hidden // (8 if dtype == "bf16" else 4)
+    return resident_threads() // nvec + 3
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -41,6 +54,14 @@ HIDDEN = [8, 16, 24, 40, 256, 512, 1000, 1024, 2048, 4104, 8192, 16384, 32768, 4
 def test_rmsnorm_shapes(dtype, hidden, family):
     rows = 37 if hidden <= 16384 else 5
     y, exact = _run_rmsnorm(rows, hidden, dtype, seed=hidden)
+    check(y, exact, dtype, what=f"rmsnorm {dtype} {rows}x{hidden}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", HIDDEN_WIDE)
+def test_rmsnorm_shapes_past_one_wave(dtype, hidden):
+    rows = rows_past_one_wave(hidden, dtype)
+    y, exact = _run_rmsnorm(rows, hidden, dtype, seed=hidden + 2)
     check(y, exact, dtype, what=f"rmsnorm {dtype} {rows}x{hidden}")
 
 
@@ -127,6 +148,15 @@ def test_add_rmsnorm_shapes(dtype, hidden, family):
     check(y, y_exact, dtype, what=f"add_rmsnorm {dtype} {rows}x{hidden}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", HIDDEN_WIDE)
+def test_add_rmsnorm_shapes_past_one_wave(dtype, hidden):
+    rows = rows_past_one_wave(hidden, dtype)
+    y, r_out, y_exact, r_exact = _run_add(rows, hidden, dtype, seed=hidden + 4)
+    assert np.array_equal(to_f64(r_out), r_exact)
+    check(y, y_exact, dtype, what=f"add_rmsnorm {dtype} {rows}x{hidden}")
+
+
 def test_add_rmsnorm_is_add_then_norm_on_gpu(family):
     """The fused kernel equals the add written back, then RMSNorm of it, both on
     the GPU (bit for bit: the norm sees exactly the written residual)."""
@@ -198,6 +228,22 @@ def test_layernorm_shapes(dtype, hidden):
     check(y, exact, dtype, scale, what=f"layernorm {dtype} {rows}x{hidden}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", HIDDEN_WIDE)
+def test_add_layernorm_shapes_past_one_wave(dtype, hidden):
+    rows = rows_past_one_wave(hidden, dtype)
+    inp = _ln_inputs(rows, hidden, dtype, hidden + 13)
+    x = (inp["x"].float() + 3.0).to(inp["x"].dtype)
+    y, r_out = ops.add_layernorm(dev(x), dev(inp["residual"]), dev(inp["gamma"]),
+                                 dev(inp["beta"]), EPS, residual_out=torch.empty_like(dev(x)))
+    torch.cuda.synchronize()
+    y_exact, r_exact = oracle.get().add_layernorm(x, inp["residual"], inp["gamma"],
+                                                  inp["beta"], EPS, dtype)
+    assert np.array_equal(to_f64(r_out), r_exact)
+    scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
+    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}")
+
+
 @pytest.mark.parametrize("in_place", [False, True])
 def test_add_layernorm_bf16_4096x2048(in_place):
     inp = _ln_inputs(4096, 2048, "bf16", 0)
@@ -213,7 +259,7 @@ def test_add_layernorm_bf16_4096x2048(in_place):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("hidden", [8, 2048, 100, 40000, 16384])
+@pytest.mark.parametrize("hidden", [8, 264, 1000, 2048, 4000, 100, 40000, 16384])
 def test_add_layernorm_shapes(dtype, hidden):
     rows = 9
     inp = _ln_inputs(rows, hidden, dtype, hidden + 11)

@@ -120,6 +120,19 @@ __device__ __forceinline__ void st_stream(void* p, const uint4& v)
     __stcs(reinterpret_cast<uint4*>(p), v);
 }
 
+// Output store of a kernel that streams (STREAM) or of a latency-bound launch
+// of a few KB to a few MB whose output the next kernel reads at once: there a
+// plain write-back store measured ~3% less time per launch on B200 than the
+// evict-first one in chains of dependent decode-size launches.
+template <bool STREAM>
+__device__ __forceinline__ void st_out(void* p, const uint4& v)
+{
+    if constexpr (STREAM)
+        __stcs(reinterpret_cast<uint4*>(p), v);
+    else
+        *reinterpret_cast<uint4*>(p) = v;
+}
+
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------

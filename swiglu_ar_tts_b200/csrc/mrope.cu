@@ -68,6 +68,20 @@ __device__ __forceinline__ int32_t position_of(int j, const MropeParams& prm, in
 
 constexpr int kWarpsPerCta = 4;
 
+// Token of warp unit `unit` and which of the token's `splits` warps it is.
+// splits > 1 only for launches of at most one head pass per resident warp, so
+// the unit index fits 32 bits there and the division stays a 32-bit one.
+__device__ __forceinline__ int64_t unit_token(int64_t unit, int splits, int& part)
+{
+    if (splits == 1) {
+        part = 0;
+        return unit;
+    }
+    const uint32_t u = (uint32_t)unit;
+    part = (int)(u % (uint32_t)splits);
+    return (int64_t)(u / (uint32_t)splits);
+}
+
 template <typename T, int P, int U>
 __global__ void __launch_bounds__(32 * kWarpsPerCta)
 mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __restrict__ pos,
@@ -77,7 +91,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     constexpr int G = 32 / P;                // heads per warp pass
     constexpr int HALF = P * E;              // head_dim / 2
     constexpr int D = 2 * HALF;
-    constexpr int F = (E >= G) ? E / G : 1;  // angles evaluated per lane
+    constexpr int F = (E >= G) ? E / G : 1;
+    constexpr bool kStream = U > 1;  // one pass per warp: decode-size launches  // angles evaluated per lane
     const int lane = threadIdx.x & 31;
     const int pv = lane % P;
     const int hg = lane / P;
@@ -90,8 +105,9 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     const int64_t units = tokens * splits;
     const int64_t unit0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     {
-        const int64_t t0 = unit0 / splits;
-        if (lane == 0 && unit0 < units && unit0 % splits == 0) {
+        int part0 = 0;
+        const int64_t t0 = unit_token(unit0, splits, part0);
+        if (lane == 0 && unit0 < units && part0 == 0) {
             if (hq > 0)
                 prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
             if (hk > 0)
@@ -106,8 +122,9 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     pdl_allow_dependents();
 
     for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
-        const int64_t t = unit / splits;
-        const int h_first = hg + (int)(unit % splits) * G * U;
+        int part = 0;
+        const int64_t t = unit_token(unit, splits, part);
+        const int h_first = hg + part * G * U;
         const int32_t pt = __ldg(pos + t);
         const int32_t ph = __ldg(pos + tokens + t);
         const int32_t pw = __ldg(pos + 2 * tokens + t);
@@ -162,8 +179,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
                     }
                     T* dst = (h < hq) ? q_out + ((size_t)t * hq + h) * D
                                       : k_out + ((size_t)t * hk + (h - hq)) * D;
-                    st_stream(dst + j0, Vec<T>::pack(oa));
-                    st_stream(dst + HALF + j0, Vec<T>::pack(ob));
+                    st_out<kStream>(dst + j0, Vec<T>::pack(oa));
+                    st_out<kStream>(dst + HALF + j0, Vec<T>::pack(ob));
                 }
             }
         }
@@ -359,6 +376,7 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     constexpr int HALF = P * E;
     constexpr int D = 2 * HALF;
     constexpr int F = (E >= G) ? E / G : 1;
+    constexpr bool kStream = U > 1;  // one pass per warp: decode-size launches
     const int lane = threadIdx.x & 31;
     const int pv = lane % P;
     const int hg = lane / P;
@@ -369,8 +387,9 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     const int64_t units = tokens * splits;
     const int64_t unit0 = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     {
-        const int64_t t0 = unit0 / splits;
-        if (lane == 0 && unit0 < units && unit0 % splits == 0) {
+        int part0 = 0;
+        const int64_t t0 = unit_token(unit0, splits, part0);
+        if (lane == 0 && unit0 < units && part0 == 0) {
             if (hq > 0)
                 prefetch_l2(q + (size_t)t0 * hq * D, (uint32_t)(hq * D * sizeof(T)));
             if (hk > 0) {
@@ -389,8 +408,9 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     pdl_allow_dependents();
 
     for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
-        const int64_t t = unit / splits;
-        const int h_first = hg + (int)(unit % splits) * G * U;
+        int part = 0;
+        const int64_t t = unit_token(unit, splits, part);
+        const int h_first = hg + part * G * U;
         const int32_t pt = __ldg(pos + t);
         const int32_t ph = __ldg(pos + tokens + t);
         const int32_t pw = __ldg(pos + 2 * tokens + t);
@@ -449,8 +469,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
                 if (h >= hq + hk) {  // v: copied unrotated into its cache slot
                     if (in_cache) {
                         T* dst = v_cache + (((size_t)cb * hk + (h - hq - hk)) * ca.max_seq + cs) * D;
-                        st_stream(dst + j0, lo[u]);
-                        st_stream(dst + HALF + j0, hi[u]);
+                        st_out<kStream>(dst + j0, lo[u]);
+                        st_out<kStream>(dst + HALF + j0, hi[u]);
                     }
                     continue;
                 }
@@ -470,8 +490,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
                         continue;
                     dst = k_cache + (((size_t)cb * hk + (h - hq)) * ca.max_seq + cs) * D;
                 }
-                st_stream(dst + j0, Vec<T>::pack(oa));
-                st_stream(dst + HALF + j0, Vec<T>::pack(ob));
+                st_out<kStream>(dst + j0, Vec<T>::pack(oa));
+                st_out<kStream>(dst + HALF + j0, Vec<T>::pack(ob));
             }
         }
     }

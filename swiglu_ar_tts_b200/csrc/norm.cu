@@ -214,6 +214,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
     constexpr int E = Vec<T>::N;
     constexpr int G = 32 * GW;  // threads per row
     constexpr int ROWS_PER_CTA = (GW == 1) ? kRowsPerSmallCta : 1;
+    constexpr bool kStream = VPL > 1;  // one vector per lane: decode-size launches
     const int nvec = hidden / E;
     const int tid = threadIdx.x;
     const int gt = (GW == 1) ? (tid & 31) : tid;
@@ -277,7 +278,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
                     for (int e = 0; e < E; ++e)
                         a[e] = a[e] + b[e];
                     v[i] = Vec<T>::pack(a);  // the residual, rounded to T
-                    st_stream(residual_out + base + (size_t)vi * E, v[i]);
+                    st_out<kStream>(residual_out + base + (size_t)vi * E, v[i]);
                 }
             }
         } else {
@@ -350,7 +351,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
                     for (int e = 0; e < E; ++e)
                         a[e] = a[e] * r * g[e];
                 }
-                st_stream(y + base + (size_t)vi * E, Vec<T>::pack(a));
+                st_out<kStream>(y + base + (size_t)vi * E, Vec<T>::pack(a));
             }
         }
     }

@@ -61,6 +61,7 @@ __device__ __forceinline__ void silu_mul(float (&a)[E], const float (&b)[E])
     }
 }
 
+// U = 1 only for decode-size launches, whose output takes a plain store.
 template <typename T, int U, int THREADS>
 __global__ void __launch_bounds__(THREADS)
 swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
@@ -100,7 +101,7 @@ swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
                 Vec<T>::unpack(g[i], a);
                 Vec<T>::unpack(u[i], b);
                 silu_mul<T>(a, b);
-                st_stream(out + vi * E, Vec<T>::pack(a));
+                st_out<(U > 1)>(out + vi * E, Vec<T>::pack(a));
             }
         }
     }

@@ -26,6 +26,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -90,51 +91,168 @@ __device__ __forceinline__ int64_t cand_index(uint64_t key)
     return (int64_t)((1u << kIndexBits) - 1u - (uint32_t)(key & ((1u << kIndexBits) - 1u)));
 }
 
-// Shared state of one block-wide radix select.
+// Shared state of one block-wide select.
+constexpr int kSmallBin = 64;  // boundary bins up to this size are ranked directly
+
 struct SelectState {
     uint32_t hist[256];
+    uint32_t warp_top[32];
+    uint64_t bin_keys[kSmallBin];
+    uint32_t bin_top;  // leading 16 bits of the boundary bin's keys
+    int bin_size;
+    int bin_filled;
     uint64_t tau;   // digits of the k-th largest key found so far
     int need;       // how many keys still to take from the current bin
     int shift;      // the select ends at this digit: keys with (key >> shift) >= (tau >> shift)
     int done;
+    int window;     // the first round found the bin of the k-th largest key
     int count;      // output slots handed out
 };
 
-// Radix select (most significant 8-bit digit first) of the k largest among
-// the block's BITS-bit keys, all distinct: every thread passes its M keys
-// (`valid` marks real ones).  On return every thread can test a key with selected().
-// A round histograms the digit of the keys that share the digits fixed so
-// far; the bin holding the k-th largest key becomes the next prefix; the
-// select stops once that bin is taken whole, which always happens by the last
-// digit because keys are distinct.  Histogram updates are plain shared-memory
-// atomics: lanes of a warp that hit one bin serialise, which costs less than
-// aggregating them with warp match instructions (measured), and after the
-// first digit few keys are still active.
-template <int BITS, int M>
-__device__ void select_top_k(const uint64_t (&key)[M], const bool (&valid)[M], int k,
-                             SelectState& st)
+// Select of the k largest among the block's BITS-bit keys, all distinct: every
+// thread passes its M keys (`valid` marks real ones).  On return every thread
+// can test a key with selected().
+//
+// First round: the keys' leading 16 bits (the value's sign, exponent and
+// leading mantissa bits) are measured as a distance d below the block's
+// largest, and keys with d < 256 are histogrammed by d.  The k largest keys of
+// a row of logits lie within that window (within two binades of the largest
+// value) unless the row is flatter than any logit distribution, so this round
+// usually finds the bin of the k-th largest key at once, and only the keys
+// near the top touch the histogram.  An 8-bit digit of the raw bits instead
+// puts most values into a handful of exponent bins, where shared-memory
+// atomics on one address serialise.  When the window holds fewer than k keys,
+// the select starts over on the raw bits.
+// Further rounds (most significant 8-bit digit first) histogram the digit of
+// the keys that share the bits fixed so far; the bin holding the k-th largest
+// key becomes the next prefix; the select stops once that bin is taken whole,
+// which always happens by the last digit because keys are distinct.  They are
+// needed only for a boundary bin of more than kSmallBin keys (or after a
+// window that held fewer than k): a smaller one is gathered into shared
+// memory and its keys ranked by counting, and the key of rank `need` becomes
+// the threshold.
+template <int BITS, typename K, int M>
+__device__ void select_top_k(const K (&key)[M], const bool (&valid)[M], int k, SelectState& st)
 {
-    static_assert(BITS % 8 == 0 && BITS <= 64, "keys are a whole number of 8-bit digits");
+    static_assert(BITS % 8 == 0 && BITS >= 32 && BITS <= 8 * (int)sizeof(K),
+                  "keys are whole 8-bit digits that fit the key type");
+    constexpr int VS = BITS - 16;  // shift of the leading 16 bits
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int warps = (int)(blockDim.x >> 5);
+
+    // largest leading 16 bits in the block
+    uint32_t top = 0;
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+        if (valid[m])
+            top = max(top, (uint32_t)(key[m] >> VS));
+    top = __reduce_max_sync(0xFFFFFFFFu, top);
+    if (lane == 0)
+        st.warp_top[warp] = top;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        st.hist[i] = 0;
     if (threadIdx.x == 0) {
-        st.tau = 0;
-        st.need = k;
         st.done = 0;
+        st.window = 0;
         st.shift = 0;
     }
-    for (int shift = BITS - 8; shift >= 0; shift -= 8) {
+    __syncthreads();
+    top = 0;
+    for (int w = 0; w < warps; ++w)
+        top = max(top, st.warp_top[w]);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        if (valid[m]) {
+            const uint32_t d = top - (uint32_t)(key[m] >> VS);
+            if (d < 256u)
+                atomicAdd(&st.hist[d], 1u);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // bins [8 lane, 8 lane + 8), nearest the top first
+        uint32_t local = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+            local += st.hist[8 * lane + b];
+        uint32_t upto = local;  // keys in this lane's bins and every nearer bin
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, upto, o);
+            if (lane >= o)
+                upto += v;
+        }
+        const uint32_t nearer = upto - local;
+        if (nearer < (uint32_t)k && upto >= (uint32_t)k) {
+            uint32_t run = nearer;
+            for (int b = 0; b < 8; ++b) {
+                const uint32_t h = st.hist[8 * lane + b];
+                if (run + h >= (uint32_t)k) {
+                    const int rest = k - (int)run;
+                    st.tau = (uint64_t)(top - (uint32_t)(8 * lane + b)) << VS;
+                    st.need = rest;
+                    st.window = 1;
+                    st.bin_top = top - (uint32_t)(8 * lane + b);
+                    st.bin_size = (int)h;
+                    st.bin_filled = 0;
+                    if ((uint32_t)rest == h) {  // the whole bin is taken
+                        st.done = 1;
+                        st.shift = VS;
+                    }
+                    break;
+                }
+                run += h;
+            }
+        }
+    }
+    __syncthreads();
+    if (st.done)
+        return;
+    if (st.window && st.bin_size <= kSmallBin) {
+        const uint32_t bin_top = st.bin_top;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (valid[m] && (uint32_t)(key[m] >> VS) == bin_top)
+                st.bin_keys[atomicAdd(&st.bin_filled, 1)] = (uint64_t)key[m];
+        }
+        __syncthreads();
+        const int size = st.bin_size;
+        if ((int)threadIdx.x < size) {
+            const uint64_t mine = st.bin_keys[threadIdx.x];
+            int larger = 0;
+            for (int j = 0; j < size; ++j)
+                larger += st.bin_keys[j] > mine;
+            if (larger == st.need - 1) {  // keys are distinct: exactly one thread
+                st.tau = mine;
+                st.shift = 0;
+                st.done = 1;
+            }
+        }
+        __syncthreads();
+        return;
+    }
+    int first = VS - 8;  // the bin's leading 16 bits are fixed
+    if (!st.window) {
+        first = BITS - 8;
+        if (threadIdx.x == 0) {
+            st.tau = 0;
+            st.need = k;
+        }
+    }
+    for (int shift = first; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x)
             st.hist[i] = 0;
         __syncthreads();
-        const uint64_t high_mask = (shift + 8 >= 64) ? 0ull : (~0ull << (shift + 8));
-        const uint64_t prefix = st.tau & high_mask;
+        const K high_mask = (shift + 8 >= BITS) ? K(0) : (K(~K(0)) << (shift + 8));
+        const K prefix = (K)st.tau & high_mask;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
             if (valid[m] && ((key[m] & high_mask) == prefix))
                 atomicAdd(&st.hist[(uint32_t)(key[m] >> shift) & 255u], 1u);
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
+        if (warp == 0) {
             // bins [8 lane, 8 lane + 8); counts from the top down
             uint32_t local = 0;
 #pragma unroll
@@ -173,55 +291,94 @@ __device__ void select_top_k(const uint64_t (&key)[M], const bool (&valid)[M], i
     }
 }
 
-__device__ __forceinline__ bool selected(uint64_t key, const SelectState& st)
+template <typename K>
+__device__ __forceinline__ bool selected(K key, const SelectState& st)
 {
-    return (key >> st.shift) >= (st.tau >> st.shift);
+    return (key >> st.shift) >= ((K)st.tau >> st.shift);
 }
 
 constexpr int kPerThread = kSlice / kSliceThreads;  // 16
 
+// In-slice keys: value bits above the inverted 16-bit position in the slice
+// (32 bits in all for bf16, 48 for fp32).
 template <typename T>
-__global__ void __launch_bounds__(kSliceThreads)
+struct LocalKey {
+    using type = typename std::conditional<KeyBits<T>::V + 16 <= 32, uint32_t, uint64_t>::type;
+    static constexpr int BITS = KeyBits<T>::V + 16;
+};
+
+// VEC: rows start on 16-byte boundaries, so a thread loads its 16 logits as
+// 16-byte vectors (positions (v * 256 + thread) * E + e); otherwise one
+// element at a time (positions thread + 256 m).  Either way every position of
+// the slice is read exactly once.
+// bf16: three CTAs per SM (<= 85 registers), which many-row calls need as they
+// run several waves; fp32's 48-bit keys would spill there, so two.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSliceThreads, sizeof(T) == 2 ? 3 : 2)
 topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices,
                   uint64_t* __restrict__ work)
 {
+    using K = typename LocalKey<T>::type;
+    constexpr int E = Vec<T>::N;
     __shared__ SelectState st;
     const int64_t row = blockIdx.y;
     const int64_t first = (int64_t)blockIdx.x * kSlice;
     const T* lr = logits + row * vocab;
-    const int64_t n = (vocab - first < kSlice) ? vocab - first : kSlice;
+    const int n = (int)((vocab - first < kSlice) ? vocab - first : kSlice);
     // the slice into L2 while the previous kernel drains, one line per thread
     {
         constexpr int kPerLine = 128 / sizeof(T);
-        if ((int64_t)threadIdx.x * kPerLine < n)
-            prefetch_l2_line(lr + first + (int64_t)threadIdx.x * kPerLine);
+        if (threadIdx.x * kPerLine < n)
+            prefetch_l2_line(lr + first + threadIdx.x * kPerLine);
     }
     pdl_wait();
     pdl_allow_dependents();
-    // in-slice keys: value bits above the inverted 16-bit position in the slice
-    constexpr int kLocalBits = KeyBits<T>::V + 16;
-    uint64_t key[kPerThread];
+    K key[kPerThread];
     float val[kPerThread];
     bool valid[kPerThread];
+    int pos[kPerThread];
+    if constexpr (VEC) {
+#pragma unroll
+        for (int v = 0; v < kPerThread / E; ++v) {
+            const int p0 = (v * kSliceThreads + (int)threadIdx.x) * E;
+            float f[E];
+            if (p0 + E <= n) {
+                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(lr + first + p0)), f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < E; ++j)
+                    f[j] = (p0 + j < n) ? load_elem(lr + first + p0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+                val[v * E + j] = f[j];
+                pos[v * E + j] = p0 + j;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < kPerThread; ++m) {
+            pos[m] = (int)threadIdx.x + m * kSliceThreads;
+            val[m] = (pos[m] < n) ? load_elem(lr + first + pos[m]) : 0.f;
+        }
+    }
 #pragma unroll
     for (int m = 0; m < kPerThread; ++m) {
-        const int i = threadIdx.x + m * kSliceThreads;
-        valid[m] = i < n;
-        val[m] = valid[m] ? load_elem(lr + first + i) : 0.f;
-        key[m] = valid[m] ? (((uint64_t)KeyBits<T>::of(val[m]) << 16) | (uint64_t)(0xFFFFu - i)) : 0ull;
+        valid[m] = pos[m] < n;
+        key[m] = valid[m] ? (((K)KeyBits<T>::of(val[m]) << 16) | (K)(0xFFFFu - (uint32_t)pos[m]))
+                          : K(0);
     }
     uint64_t* out = work + (row * slices + blockIdx.x) * (int64_t)k;
     if (n <= k) {
         // the whole slice is a candidate; the unused slots get keys below any logit
 #pragma unroll
         for (int m = 0; m < kPerThread; ++m) {
-            const int i = threadIdx.x + m * kSliceThreads;
-            if (i < k)
-                out[i] = valid[m] ? cand_key<T>(val[m], first + i) : 0ull;
+            if (pos[m] < k)
+                out[pos[m]] = valid[m] ? cand_key<T>(val[m], first + pos[m]) : 0ull;
         }
         return;
     }
-    select_top_k<kLocalBits>(key, valid, k, st);
+    select_top_k<LocalKey<T>::BITS>(key, valid, k, st);
     if (threadIdx.x == 0)
         st.count = 0;
     __syncthreads();
@@ -230,7 +387,7 @@ topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices
         if (valid[m] && selected(key[m], st)) {
             const int slot = atomicAdd(&st.count, 1);
             if (slot < k)  // exactly k are selected; the test only guards the bound
-                out[slot] = cand_key<T>(val[m], first + threadIdx.x + m * kSliceThreads);
+                out[slot] = cand_key<T>(val[m], first + pos[m]);
         }
 }
 
@@ -245,7 +402,6 @@ topk_sample_kernel(const uint64_t* __restrict__ work, int slices, int k,
     __shared__ SelectState st;
     __shared__ uint64_t sel[kMaxTopK];
     __shared__ uint64_t ranked[kMaxTopK];
-    __shared__ float e[kMaxTopK];
     const int64_t row = blockIdx.x;
     const int n = slices * k;
     pdl_wait();
@@ -281,26 +437,52 @@ topk_sample_kernel(const uint64_t* __restrict__ work, int slices, int k,
     }
     __syncthreads();
 
-    // exp((l_j - l_0) / T) for the k candidates
+    // Warp 0 takes the decision, two ranks per lane (k <= 64).  Per rank j:
+    // e_j = exp((l_j - l_0) / T) and the score fl(fl(l_j / T) + g_j), two
+    // correctly rounded operations.  The token is the first rank with the
+    // largest score, as a scan in rank order that moves on only to a strictly
+    // larger score finds it: NaN scores after rank 0 never win, a NaN at rank 0
+    // always does.
+    if (threadIdx.x >= 32)
+        return;
+    const int lane = threadIdx.x;
     const float l0 = cand_value<T>(ranked[0]);
-    for (int j = threadIdx.x; j < k; j += kMergeThreads)
-        e[j] = expf((cand_value<T>(ranked[j]) - l0) / temperature);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int best = 0;
-        float best_score = 0.f, z = 0.f;
-        for (int j = 0; j < k; ++j) {
-            // fl(fl(l / T) + g), two correctly rounded operations
-            const float score = __fadd_rn(__fdiv_rn(cand_value<T>(ranked[j]), temperature),
-                                          gumbel[row * k + j]);
-            if (j == 0 || score > best_score) {
-                best = j;
-                best_score = score;
+    float ej[2], bs = 0.f, z = 0.f;
+    int bj = k;  // none yet
+    float s0 = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = lane + 32 * r;
+        ej[r] = 0.f;
+        if (j < k) {
+            const float l = cand_value<T>(ranked[j]);
+            ej[r] = expf((l - l0) / temperature);
+            const float sc = __fadd_rn(__fdiv_rn(l, temperature), gumbel[row * k + j]);
+            if (j == 0)
+                s0 = sc;
+            if (!isnan(sc) && (bj == k || sc > bs)) {
+                bs = sc;
+                bj = j;
             }
-            z += e[j];
+            z += ej[r];
         }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
+        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, o);
+        if (oj < k && (bj == k || os > bs || (os == bs && oj < bj))) {
+            bs = os;
+            bj = oj;
+        }
+        z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    }
+    s0 = __shfl_sync(0xFFFFFFFFu, s0, 0);
+    const int best = isnan(s0) ? 0 : bj;
+    const float eb = __shfl_sync(0xFFFFFFFFu, best < 32 ? ej[0] : ej[1], best & 31);
+    if (lane == 0) {
         token_out[row] = (int32_t)cand_index(ranked[best]);
-        prob_out[row] = e[best] / z;
+        prob_out[row] = eb / z;
     }
 }
 
@@ -328,13 +510,22 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
 {
     const int slices = topk_slices(vocab);
     const dim3 grid1((unsigned)slices, (unsigned)rows);
+    const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
+    const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
     cudaError_t err;
-    if (dtype == AROPS_BF16)
-        err = launch(topk_slice_kernel<__nv_bfloat16>, grid1, dim3(kSliceThreads), 0, stream,
-                     static_cast<const __nv_bfloat16*>(logits), vocab, k, slices, work);
-    else
-        err = launch(topk_slice_kernel<float>, grid1, dim3(kSliceThreads), 0, stream,
-                     static_cast<const float*>(logits), vocab, k, slices, work);
+    if (dtype == AROPS_BF16) {
+        const auto* lg = static_cast<const __nv_bfloat16*>(logits);
+        err = vec ? launch(topk_slice_kernel<__nv_bfloat16, true>, grid1, dim3(kSliceThreads), 0,
+                           stream, lg, vocab, k, slices, work)
+                  : launch(topk_slice_kernel<__nv_bfloat16, false>, grid1, dim3(kSliceThreads), 0,
+                           stream, lg, vocab, k, slices, work);
+    } else {
+        const auto* lg = static_cast<const float*>(logits);
+        err = vec ? launch(topk_slice_kernel<float, true>, grid1, dim3(kSliceThreads), 0, stream,
+                           lg, vocab, k, slices, work)
+                  : launch(topk_slice_kernel<float, false>, grid1, dim3(kSliceThreads), 0, stream,
+                           lg, vocab, k, slices, work);
+    }
     if (err != cudaSuccess)
         return err;
     if (dtype == AROPS_BF16)

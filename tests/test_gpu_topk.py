@@ -54,6 +54,27 @@ def test_topk_sample_ties_go_to_lower_index():
         assert np.array_equal(tok, np.argmax(lg.to(dt).float().numpy(), axis=1))
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_topk_sample_flat_spread_and_outlier_rows(dtype):
+    """Rows whose k largest values are not all near the largest one, and rows
+    where one value repeats everywhere: constant logits (the k lowest indices
+    win), three outliers far above N(0,1) noise (fewer than k values within
+    two binades of the largest), magnitudes spread over 2^-60 .. 2^60 of both
+    signs, and all-negative logits."""
+    rng = np.random.default_rng(17)
+    v, k = 20000, 50
+    lg = np.empty((5, v))
+    lg[0] = 1.25
+    lg[1] = rng.standard_normal(v)
+    lg[1, [7, 5000, 19999]] = [9000.0, 8000.0, 7000.0]
+    lg[2] = rng.choice([-1.0, 1.0], v) * np.exp2(rng.uniform(-60, 60, v))
+    lg[3] = -np.abs(rng.standard_normal(v)) * 4 - 1.0
+    lg[4] = np.round(rng.standard_normal(v) * 3)
+    inp = {"logits": torch.from_numpy(lg).float().to(dtype),
+           "gumbel": torch.from_numpy(rng.gumbel(size=(5, k)).astype(np.float32))}
+    _check(inp, k, 1.0, f"flat/spread/outliers {dtype}")
+
+
 def test_topk_sample_winner_in_last_slice_and_greedy():
     inp = inputs.topk_inputs(4, 151936, 8, "bf16", seed=9)
     lg = inp["logits"].clone()

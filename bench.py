@@ -60,6 +60,11 @@ FALLBACK_HBM_GBS = 6650.0
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
+# B200 HBM3e specification (DGX figure); fractions of it are reported beside
+# the fractions of the measured copy peak
+SPEC_HBM_GBS = 8000.0
+
+
 def measured_hbm_peak() -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -567,7 +572,8 @@ def main() -> None:
         us = 1e3 * per_op_ms[i]
         gbs = step.bytes[name] / (us * 1e-6) / 1e9
         ops_report[name] = {"us": round(us, 3), "bytes": step.bytes[name], "gbs": round(gbs, 1),
-                            "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4)}
+                            "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
+                            "frac_of_spec_hbm": round(gbs / SPEC_HBM_GBS, 4)}
     # time per kernel type in the step: prefill operators are timed directly;
     # each decode graph is split across its operators' kernels (decode_split)
     kernels: dict[str, dict] = {}
@@ -634,6 +640,28 @@ def main() -> None:
                                  "rmsnorm_saves": round(1 - t["rmsnorm"] / t["layernorm"], 4)}
         del ln
 
+    # a decoding run: 300 consecutive steps (positions 0..299, as the 300 decode
+    # steps of an utterance), replaying the captured step graph and launching
+    # the 112 operators one by one from the host loop, outside the timed steps
+    run300 = {}
+    for batch, chain in ((5, step.chain5), (256, step.chain256)):
+        saved = chain.residual.clone()
+        t = {}
+        for mode in ("graph", "eager"):
+            go = chain.replay if mode == "graph" else chain.step
+            for s in range(3):
+                go(s)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for s in range(300):
+                go(s)
+            e1.record()
+            torch.cuda.synchronize()
+            t[mode] = 1e3 * e0.elapsed_time(e1) / 300
+        chain.residual.copy_(saved)
+        run300[f"batch{batch}"] = {"graph_us_per_step": round(t["graph"], 2),
+                                   "eager_us_per_step": round(t["eager"], 2)}
+
     # end to end: pinned host buffers in and out, through the same public calls
     step.setup_e2e()
     torch.cuda.synchronize()
@@ -688,6 +716,7 @@ def main() -> None:
         "roofline_swiglu": roofline_swiglu,
         "kernels": kernels,
         "layernorm_to_rmsnorm": swap,
+        "decode_300_steps": run300,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": eager_launches + args.steps * (step.kernels_per_step - 4),

@@ -596,12 +596,21 @@ def main() -> None:
         k["us"] = round(k["us"], 2)
     dominant = max(kernels, key=lambda k: kernels[k]["us"])
     dk = kernels[dominant]
+    # traffic: DRAM bytes per launch averaged over the step's launches of the
+    # kernel, from one ncu capture per launch size (profiles/traffic.json)
+    dom_traffic = None
+    if dominant == "norm_rows_kernel":
+        dom_traffic = ncu_traffic("norm_rows_kernel", ("swiglu_ar_tts_b200/csrc/norm.cu",
+                                                       "swiglu_ar_tts_b200/csrc/common.cuh"))
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": dk["gbs"], "peak": peak,
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dk["gbs"] / peak, 4),
-                "traffic": None, "launches_per_step": dk["launches"],
+                "traffic": dom_traffic, "launches_per_step": dk["launches"],
                 "algorithmic_bytes_per_step": dk["bytes"],
-                "note": "dominant by share of step time; its launches span prefill and decode "
-                        "sizes, so no single ncu capture gives their DRAM traffic"}
+                "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
+                "note": "dominant by share of step time; achieved = its algorithmic bytes per "
+                        "step / its time per step; traffic = DRAM bytes per launch, averaged "
+                        "over the step's prefill and decode launches (reads = operands, "
+                        "outputs still in L2 at kernel end)"}
     sw_us = ops_report["swiglu"]["us"]
     sw_gbs = step.bytes["swiglu"] / (sw_us * 1e-6) / 1e9
     roofline_swiglu = {"kernel": "swiglu_vec_kernel<bf16> 8192x6144 (largest single launch)",

@@ -278,6 +278,8 @@ class Step:
         self.h2d_bytes = (sum(nbytes(v.values()) for k, v in self.h_in.items() if isinstance(v, dict))
                           + nbytes(self.h_in["c5"]) + nbytes(self.h_in["c256"]))
         self.d2h_bytes = sum(nbytes(v) for v in self.h_out.values())
+        self.s_h2d = torch.cuda.Stream(self.device)
+        self.s_d2h = torch.cuda.Stream(self.device)
 
     @staticmethod
     def _chain_inputs(c):
@@ -290,34 +292,57 @@ class Step:
     def _chain_outputs(c):
         return [c.residual] + c.y_attn + c.q_out + c.k_out + c.y_mlp + c.act
 
+    # operators with the most output first: their copies back overlap the
+    # later operators' copies in, and the pipeline ends on small copies
+    E2E_GROUPS = (("c256", "decode_b256"), ("sw", "swiglu"), ("an", "add_rmsnorm"),
+                  ("mr", "mrope_qk"), ("c5", "decode_b5"), ("rn", "rmsnorm"))
+
+    def _e2e_in(self, g: str) -> list:
+        """(device input, pinned host source) pairs of operator group ``g``."""
+        if g in ("c5", "c256"):
+            c = self.chain5 if g == "c5" else self.chain256
+            return list(zip(self._chain_inputs(c), self.h_in[g]))
+        dev = {"rn": self.rn, "an": self.an, "sw": self.sw, "mr": self.mr}[g]
+        return [(dev[k], v) for k, v in self.h_in[g].items()]
+
+    def _e2e_out(self, g: str) -> list:
+        """(pinned host destination, device output) pairs of operator group ``g``."""
+        dev = {"rn": [self.rn["y"]], "an": [self.an["y"], self.an["residual_out"]],
+               "sw": [self.sw["out"]], "mr": [self.mr["q_out"], self.mr["k_out"]]}
+        if g in ("c5", "c256"):
+            srcs = self._chain_outputs(self.chain5 if g == "c5" else self.chain256)
+        else:
+            srcs = dev[g]
+        return list(zip(self.h_out[g], srcs))
+
     def run_e2e(self) -> None:
         """Host->device copies of every input, the step, device->host copies of
-        every output, all on the current stream."""
+        every output.  Three streams form a pipeline over the operators: the
+        inputs of operator i+1 cross PCIe while operator i computes and the
+        results of operator i-1 cross back (the two copy directions run at the
+        same time).  Events order each operator's copy-in, compute and
+        copy-out; the step starts after the previous step's copy-outs."""
         nb = dict(non_blocking=True)
-        for k, v in self.h_in["rn"].items():
-            self.rn[k].copy_(v, **nb)
-        for k, v in self.h_in["an"].items():
-            self.an[k].copy_(v, **nb)
-        for k, v in self.h_in["sw"].items():
-            self.sw[k].copy_(v, **nb)
-        for k, v in self.h_in["mr"].items():
-            self.mr[k].copy_(v, **nb)
-        for dst, src in zip(self._chain_inputs(self.chain5), self.h_in["c5"]):
-            dst.copy_(src, **nb)
-        for dst, src in zip(self._chain_inputs(self.chain256), self.h_in["c256"]):
-            dst.copy_(src, **nb)
-        self.run()
-        self.h_out["rn"][0].copy_(self.rn["y"], **nb)
-        self.h_out["an"][0].copy_(self.an["y"], **nb)
-        self.h_out["an"][1].copy_(self.an["residual_out"], **nb)
-        self.h_out["sw"][0].copy_(self.sw["out"], **nb)
-        self.h_out["mr"][0].copy_(self.mr["q_out"], **nb)
-        self.h_out["mr"][1].copy_(self.mr["k_out"], **nb)
-        for dst, src in zip(self.h_out["c5"], self._chain_outputs(self.chain5)):
-            dst.copy_(src, **nb)
-        for dst, src in zip(self.h_out["c256"], self._chain_outputs(self.chain256)):
-            dst.copy_(src, **nb)
-
+        cur = torch.cuda.current_stream()
+        h2d, d2h = self.s_h2d, self.s_d2h
+        h2d.wait_stream(cur)
+        for g, name in self.E2E_GROUPS:
+            with torch.cuda.stream(h2d):
+                for dst, src in self._e2e_in(g):
+                    dst.copy_(src, **nb)
+            arrived = torch.cuda.Event()
+            arrived.record(h2d)
+            cur.wait_event(arrived)
+            self.prepare_op(name)
+            self.run_op(name)
+            done = torch.cuda.Event()
+            done.record(cur)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                for dst, src in self._e2e_out(g):
+                    dst.copy_(src, **nb)
+        cur.wait_stream(d2h)
+        self.decode_step_index += 1
 
 def reduce_max(x: float, pg=None, device=None) -> float:
     """Max of ``x`` over the ranks of process group ``pg`` (identity without one).
@@ -686,6 +711,11 @@ def main() -> None:
     e1.record()
     torch.cuda.synchronize()
     barrier()
+    # the pipelined copies hand back exactly what the device holds
+    for g, _ in step.E2E_GROUPS:
+        for dst, src in step._e2e_out(g):
+            if not torch.equal(dst, src.cpu()):
+                raise SystemExit(f"e2e: host copy of {g} differs from the device result")
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
     e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
            "ms_per_step": e2e_ms, "h2d_bytes_per_step": step.h2d_bytes,

@@ -213,6 +213,9 @@ class Step:
             "decode_b5": self.chain5.bytes_per_step(),
             "decode_b256": self.chain256.bytes_per_step(),
         }
+        # rows (tokens) one launch of each operator processes
+        self.rows = {"rmsnorm": 64, "add_rmsnorm": 4096, "swiglu": 8192, "mrope_qk": 4096,
+                     "decode_b5": 5, "decode_b256": 256}
         # kernels of this library launched per step (graph replays bypass the
         # launch counter, so their kernels are counted from the capture)
         self.kernels_per_step = 4 + self.chain5.launches_per_step + self.chain256.launches_per_step
@@ -598,7 +601,8 @@ def main() -> None:
         gbs = step.bytes[name] / (us * 1e-6) / 1e9
         ops_report[name] = {"us": round(us, 3), "bytes": step.bytes[name], "gbs": round(gbs, 1),
                             "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
-                            "frac_of_spec_hbm": round(gbs / SPEC_HBM_GBS, 4)}
+                            "frac_of_spec_hbm": round(gbs / SPEC_HBM_GBS, 4),
+                            "rows_per_s": round(step.rows[name] / (us * 1e-6))}
     # time per kernel type in the step: prefill operators are timed directly;
     # each decode graph is split across its operators' kernels (decode_split)
     kernels: dict[str, dict] = {}

@@ -14,9 +14,10 @@
 //                       inverted position, so that larger keys are larger logits
 //                       and, among equal logits, lower indices: every key is
 //                       distinct; 32 bits for bf16, 48 for fp32), finds its k
-//                       largest with a block-wide radix select in registers and
-//                       shared memory, and writes them to the workspace as
-//                       (value bits, inverted 24-bit vocabulary index) keys.
+//                       largest with a block-wide select in registers and
+//                       shared memory (select_top_k below), and writes them to
+//                       the workspace as (value bits, inverted 24-bit
+//                       vocabulary index) keys.
 //   topk_sample_kernel  grid (rows): selects the row's k largest among the
 //                       slices' candidates the same way, ranks those k by
 //                       counting, then takes the sampling decision and the

@@ -615,9 +615,12 @@ def main() -> None:
 
     for name in ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk"):
         add_time(KERNEL_OF[name], ops_report[name]["us"], 1, step.bytes[name])
+    decode_launch_us: dict[str, dict] = {}  # µs per decode launch, per kernel and batch
     for name, chain in (("decode_b5", step.chain5), ("decode_b256", step.chain256)):
         for op, (frac, launches, nbytes) in decode_split(chain).items():
             add_time(KERNEL_OF[op], frac * ops_report[name]["us"], launches, nbytes)
+            decode_launch_us.setdefault(KERNEL_OF[op], {})[name] = round(
+                frac * ops_report[name]["us"] / launches, 3)
     step_us = 1e3 * ms_per_step
     for k in kernels.values():
         k["share"] = round(k["us"] / step_us, 4)
@@ -636,10 +639,13 @@ def main() -> None:
                 "traffic": dom_traffic, "launches_per_step": dk["launches"],
                 "algorithmic_bytes_per_step": dk["bytes"],
                 "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
+                "us_per_decode_launch": decode_launch_us.get(dominant, {}),
                 "note": "dominant by share of step time; achieved = its algorithmic bytes per "
                         "step / its time per step; traffic = DRAM bytes per launch, averaged "
                         "over the step's prefill and decode launches (reads = operands, "
-                        "outputs still in L2 at kernel end)"}
+                        "outputs still in L2 at kernel end); all but 2 of its launches are "
+                        "decode launches of 45 KB to 4.2 MB, bound by the latency of a "
+                        "dependent launch (us_per_decode_launch) rather than by bandwidth"}
     sw_us = ops_report["swiglu"]["us"]
     sw_gbs = step.bytes["swiglu"] / (sw_us * 1e-6) / 1e9
     roofline_swiglu = {"kernel": "swiglu_vec_kernel<bf16> 8192x6144 (largest single launch)",

@@ -121,11 +121,19 @@ def _dtype_code(*ts: torch.Tensor) -> int:
     return DTYPES[dt]
 
 
-def _cuda_contig(name: str, t: torch.Tensor) -> None:
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+def _check_tensors(named) -> None:
+    """Every (name, tensor) is a contiguous CUDA tensor on the first one's device:
+    the kernels receive raw pointers and run on that device."""
+    dev = None
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
 
 
 def rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
@@ -134,8 +142,7 @@ def rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
     hidden = x.shape[-1]
     if out is None:
         out = torch.empty_like(x)
-    for n, t in (("x", x), ("gamma", gamma), ("out", out)):
-        _cuda_contig(n, t)
+    _check_tensors((("x", x), ("gamma", gamma), ("out", out)))
     if gamma.shape != (hidden,) or out.shape != x.shape:
         raise ValueError("shape mismatch")
     code = _dtype_code(x, gamma, out)
@@ -157,9 +164,8 @@ def add_rmsnorm(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor, ep
         y = torch.empty_like(x)
     if residual_out is None:
         residual_out = residual
-    for n, t in (("x", x), ("residual", residual), ("gamma", gamma), ("y", y),
-                 ("residual_out", residual_out)):
-        _cuda_contig(n, t)
+    _check_tensors((("x", x), ("residual", residual), ("gamma", gamma), ("y", y),
+                    ("residual_out", residual_out)))
     if (residual.shape != x.shape or y.shape != x.shape or residual_out.shape != x.shape
             or gamma.shape != (hidden,)):
         raise ValueError("shape mismatch")
@@ -178,8 +184,7 @@ def layernorm(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, eps: flo
     hidden = x.shape[-1]
     if out is None:
         out = torch.empty_like(x)
-    for n, t in (("x", x), ("gamma", gamma), ("beta", beta), ("out", out)):
-        _cuda_contig(n, t)
+    _check_tensors((("x", x), ("gamma", gamma), ("beta", beta), ("out", out)))
     if gamma.shape != (hidden,) or beta.shape != (hidden,) or out.shape != x.shape:
         raise ValueError("shape mismatch")
     code = _dtype_code(x, gamma, beta, out)
@@ -200,9 +205,8 @@ def add_layernorm(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
         y = torch.empty_like(x)
     if residual_out is None:
         residual_out = residual
-    for n, t in (("x", x), ("residual", residual), ("gamma", gamma), ("beta", beta), ("y", y),
-                 ("residual_out", residual_out)):
-        _cuda_contig(n, t)
+    _check_tensors((("x", x), ("residual", residual), ("gamma", gamma), ("beta", beta), ("y", y),
+                    ("residual_out", residual_out)))
     if (residual.shape != x.shape or y.shape != x.shape or residual_out.shape != x.shape
             or gamma.shape != (hidden,) or beta.shape != (hidden,)):
         raise ValueError("shape mismatch")
@@ -226,8 +230,7 @@ def mrope_qk(q: torch.Tensor, k: torch.Tensor, pos: torch.Tensor, sections=(24, 
         q_out = q
     if k_out is None:
         k_out = k
-    for n, t in (("q", q), ("k", k), ("pos", pos), ("q_out", q_out), ("k_out", k_out)):
-        _cuda_contig(n, t)
+    _check_tensors((("q", q), ("k", k), ("pos", pos), ("q_out", q_out), ("k_out", k_out)))
     if q.dim() != 3 or k.dim() != 3:
         raise ValueError("q and k must be [tokens, heads, head_dim]")
     tokens, hq, d = q.shape
@@ -254,9 +257,8 @@ def mrope_kv_append(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torc
     [cache_rows, n_kv_heads, max_seq, head_dim].  Returns ``q_out``."""
     if q_out is None:
         q_out = q
-    for n, t in (("q", q), ("k", k), ("v", v), ("pos", pos), ("cache_loc", cache_loc),
-                 ("k_cache", k_cache), ("v_cache", v_cache), ("q_out", q_out)):
-        _cuda_contig(n, t)
+    _check_tensors((("q", q), ("k", k), ("v", v), ("pos", pos), ("cache_loc", cache_loc),
+                    ("k_cache", k_cache), ("v_cache", v_cache), ("q_out", q_out)))
     tokens, hq, d = q.shape
     hk = k.shape[1]
     if (k.shape != (tokens, hk, d) or v.shape != k.shape or q_out.shape != q.shape
@@ -281,8 +283,7 @@ def swiglu(gate: torch.Tensor, up: torch.Tensor, out: torch.Tensor | None = None
     """out = silu(gate) * up (fp32 math); ``out`` may be ``gate`` or ``up``."""
     if out is None:
         out = torch.empty_like(gate)
-    for n, t in (("gate", gate), ("up", up), ("out", out)):
-        _cuda_contig(n, t)
+    _check_tensors((("gate", gate), ("up", up), ("out", out)))
     if up.shape != gate.shape or out.shape != gate.shape:
         raise ValueError("shape mismatch")
     code = _dtype_code(gate, up, out)
@@ -320,9 +321,8 @@ def topk_sample(logits: torch.Tensor, gumbel: torch.Tensor, top_k: int, temperat
     need = topk_sample_workspace(rows, vocab, top_k) if rows else 0
     if workspace is None:
         workspace = torch.empty(max(need, 8), dtype=torch.uint8, device=logits.device)
-    for n, t in (("logits", logits), ("gumbel", gumbel), ("token_out", token_out),
-                 ("prob_out", prob_out), ("workspace", workspace)):
-        _cuda_contig(n, t)
+    _check_tensors((("logits", logits), ("gumbel", gumbel), ("token_out", token_out),
+                    ("prob_out", prob_out), ("workspace", workspace)))
     if gumbel.dtype != torch.float32 or tuple(gumbel.shape) != (rows, top_k):
         raise ValueError("gumbel must be float32 [rows, top_k]")
     if token_out.dtype != torch.int32 or prob_out.dtype != torch.float32:
@@ -349,7 +349,8 @@ def set_streaming(enable: bool) -> bool:
 
 
 def device_errors(clear: bool = True) -> int:
-    """Device-side error bits (1 = a bulk copy timed out); synchronises."""
+    """Device-side error bits (1: a bulk-copy wait timed out; 2: a KV-cache slot
+    out of range was skipped); synchronises the device."""
     v = ctypes.c_uint32(0)
     _check(lib().arops_device_errors(ctypes.byref(v), 1 if clear else 0))
     return int(v.value)

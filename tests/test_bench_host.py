@@ -106,3 +106,12 @@ def test_decode_calls_group_by_operator(norm):
     norm_op = "add_layernorm" if norm == "layer" else "add_rmsnorm"
     assert {k: len(v) for k, v in groups.items()} == {norm_op: 56, "mrope_qk": 28, "swiglu": 28}
     assert all(bench.KERNEL_OF[k] for k in groups)
+
+
+def test_e2e_pipeline_covers_every_operator_once():
+    """The end-to-end pipeline copies in, runs and copies out every operator of
+    the step exactly once, whatever order it takes them in."""
+    names = [name for _, name in bench.Step.E2E_GROUPS]
+    assert sorted(names) == sorted(bench.Step.OPS)
+    groups = [g for g, _ in bench.Step.E2E_GROUPS]
+    assert len(set(groups)) == len(groups)

@@ -76,10 +76,17 @@ def measured_hbm_peak() -> tuple[float, str]:
 
 
 def source_digest(*rel: str) -> str:
+    """Digest of the code of the given sources: `//` comments, trailing blanks
+    and blank lines are left out (the sources keep no `//` inside string
+    literals), so an edit to comments alone keeps the digest and any change to
+    the code itself changes it."""
     h = hashlib.sha256()
     for r in rel:
-        with open(os.path.join(ROOT, r), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, r), encoding="utf-8") as f:
+            for line in f.read().splitlines():
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -188,7 +188,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
 }
 
 // ---------------------------------------------------------------------------
-// Streaming kernel (default for 16-byte-aligned q/k).  Each warp owns tokens
+// Streaming kernel (opt-in: arops_set_streaming(1), for 16-byte-aligned q/k;
+// measured slower on B200 than the register kernel).  Each warp owns tokens
 // gw, gw + nw, ... (gw = global warp index, nw = warps in the grid) and a ring
 // of `slots` shared-memory slots, each holding one token's q and k heads.  Lane
 // 0 keeps `slots` tokens in flight as bulk copies (TMA); the warp evaluates the

@@ -1,21 +1,25 @@
-// RMSNorm and fused residual-add + RMSNorm (sm_100a).
+// RMSNorm, LayerNorm and their fused residual-add forms (sm_100a).
 //
 // RMSNorm: y = gamma * x / sqrt(mean(x^2) + eps) over each row
 // ("Optimising autoregressive speech models", §09, the RMSNorm equation and
-// module).  Norm+Residual (Triton kernel-fusion post for Qwen3-TTS, section 3):
-// residual_out = round(x + residual_in), y = RMSNorm(residual_out), in one pass.
+// module); LayerNorm: y = gamma * (x - mean) / sqrt(var + eps) + beta (same
+// section).  Norm+Residual (Triton kernel-fusion post for Qwen3-TTS, section 3):
+// residual_out = round(x + residual_in), y = norm(residual_out), in one pass.
 //
-// Two designs.  The streaming kernel (below) stages rows through shared memory
-// with bulk copies and is the default for 16-byte-aligned rows.  The register
-// kernels keep the row in registers:  a row of `hidden` elements is split into
-// 16-byte vectors; a group of 32*GW threads owns the row and every thread holds
-// VPL vectors, so global memory is read once and written once (x, residual ->
-// residual_out, y) with fully coalesced 128-bit accesses.  The sum of squares is
-// accumulated in fp32, reduced with warp shuffles and, for GW > 1 warps per row,
-// one shared-memory step.  rsqrtf of (sum / hidden + eps) scales the row; the
-// product x * r * gamma is rounded once to the storage type.  gamma is read
-// through the read-only path together with each row (it stays L1/L2 resident),
-// so a row costs one memory round trip, which matters most for decode batches.
+// Two designs.  The register kernels (the default) keep the row in registers:
+// a row of `hidden` elements is split into 16-byte vectors; a group of 32*GW
+// threads owns the row and every thread holds VPL vectors, so global memory is
+// read once and written once (x, residual -> residual_out, y) with fully
+// coalesced 128-bit accesses.  The sum of squares is accumulated in fp32,
+// reduced with warp shuffles and, for GW > 1 warps per row, one shared-memory
+// step; rsqrtf of (sum * 1/hidden + eps) scales the row and x * r * gamma is
+// rounded once to the storage type.  gamma is read through the read-only path
+// together with each row, so a row costs one memory round trip.  A problem of
+// at most one vector per resident thread (a decode step's few rows) takes one
+// vector per lane with the row spread over GW = hidden/256 warps; larger ones
+// take 8 vectors per lane, one warp per row up to 2048 bf16 elements.  The
+// streaming kernel (opt-in, arops_set_streaming) stages rows through shared
+// memory with bulk copies instead; it measured slower on B200.
 //
 // Rows longer than 4096 vectors, and unaligned or ragged rows, take a looped
 // kernel that makes a second pass over the row (served from L2).
@@ -26,16 +30,16 @@ namespace arops {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Streaming kernel (the default for 16-byte-aligned rows).  A persistent CTA
+// Streaming kernel (opt-in: arops_set_streaming(1)).  A persistent CTA
 // owns rows blockIdx.x, blockIdx.x + gridDim.x, ...  One thread keeps `stages`
 // rows in flight as bulk copies (TMA) into a ring of shared-memory slots, each
 // slot holding the row of x (and of the residual); gamma is copied once per
 // CTA.  As a row lands, the CTA adds the residual, writes residual_out, reduces
 // the sum of squares (warp shuffles, then one shared-memory step), and writes
 // y.  With several CTAs per SM and 4 stages, an SM has its whole share of a
-// 4096 x 2048 problem requested within the first microsecond, so the kernel
-// runs at the rate DRAM returns data rather than at the rate warps can issue
-// dependent loads.
+// 4096 x 2048 problem requested within the first microsecond.  On B200 it ran
+// slower than the register kernels (21.0 vs 17.0 us for 4096 x 2048): the ring
+// left too few warps for the arithmetic.
 // ---------------------------------------------------------------------------
 template <typename T, bool ADD, int THREADS>
 __global__ void __launch_bounds__(THREADS)

@@ -4,8 +4,13 @@
 // Pure streaming work (two reads, one write per element, ~1 flop per byte), so
 // the kernel is shaped for HBM: 16-byte coalesced accesses, U independent
 // vectors of each input in flight per thread before any math, evict-first
-// cache hints, and a grid-stride loop over a grid sized to the SM count.  The
-// ragged tail (n % 8 elements) is handled by block 0 in the same launch.
+// cache hints, one chunk of U vectors per thread per CTA on a grid the
+// hardware schedules as SMs free up.  Decode-size problems (at most one vector
+// per resident thread) take one vector per thread in CTAs of 128 or 512
+// threads, with plain stores.  The ragged tail (n % 8 elements) is handled by
+// block 0 in the same launch.  A streaming kernel that stages chunks through
+// shared memory with bulk copies is opt-in (arops_set_streaming) and measured
+// slower on B200.
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -114,7 +119,8 @@ swiglu_vec_kernel(const T* gate, const T* up, T* out, int64_t n)
 }
 
 // ---------------------------------------------------------------------------
-// Streaming kernel (default for 16-byte-aligned buffers with n % 8 == 0).  The
+// Streaming kernel (opt-in: arops_set_streaming(1), for 16-byte-aligned
+// buffers with n % 8 == 0).  The
 // flat array is cut into chunks of kChunk elements; warp gw of the grid owns
 // chunks gw, gw + nw, ... and a ring of `slots` shared-memory slots, each
 // holding one chunk of gate and of up.  Lane 0 keeps `slots` chunks in flight

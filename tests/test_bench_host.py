@@ -115,3 +115,15 @@ def test_e2e_pipeline_covers_every_operator_once():
     assert sorted(names) == sorted(bench.Step.OPS)
     groups = [g for g, _ in bench.Step.E2E_GROUPS]
     assert len(set(groups)) == len(groups)
+
+
+def test_source_digest_ignores_comments_but_not_code(tmp_path):
+    """The traffic records stay valid across comment edits and lapse on any
+    change to the code they were measured with."""
+    f = tmp_path / "k.cu"
+    f.write_text("// kernel\n__global__ void k(int* p) { p[0] = 1; }  // store one\n")
+    d0 = bench.source_digest(str(f))
+    f.write_text("// the kernel, reworded\n\n__global__ void k(int* p) { p[0] = 1; }\n")
+    assert bench.source_digest(str(f)) == d0
+    f.write_text("// kernel\n__global__ void k(int* p) { p[0] = 2; }  // store one\n")
+    assert bench.source_digest(str(f)) != d0

@@ -50,7 +50,10 @@ def build(mutant: int = 0, force: bool = False) -> str:
     os.makedirs(_BUILD, exist_ok=True)
     fd, tmp = tempfile.mkstemp(suffix=".so", dir=_BUILD)
     os.close(fd)
-    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+    # the oracle itself builds free of warnings; a planted mistake may leave a
+    # term unused, so mutants only report theirs
+    warn = ["-Wall", "-Wextra", "-Wpedantic"] + (["-Werror"] if int(mutant) == 0 else [])
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", *warn,
            "-shared", f"-DORACLE_MUTANT={int(mutant)}", _SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)

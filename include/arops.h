@@ -249,7 +249,14 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
                                                  void* stream);
 
 /*
- * Programmatic dependent launch.  When enabled (process-wide, default off),
+ * Library controls and diagnostics follow.  They are this library's own
+ * mechanisms; the pages define no such calls.
+ *
+ * Programmatic dependent launch.  The Triton kernel-fusion post for Qwen3-TTS
+ * (section 3) reaches its end-to-end result by pairing its fused kernels with a
+ * CUDA-graph decoder; this is the launch-level counterpart for chains of small
+ * kernels.  When enabled
+ * (process-wide, default off),
  * every kernel is launched with the programmatic-stream-serialisation attribute
  * so that it can be scheduled while the previous kernel on the stream drains;
  * each kernel waits for its predecessor's memory before touching global memory,
@@ -273,9 +280,11 @@ AROPS_API int arops_set_streaming(int enable);
 
 /*
  * Device-side error bits of the current device, OR-ed by kernels that abandon
- * their work: AROPS_DEVICE_ERR_TIMEOUT means a bulk copy into shared memory did
- * not complete within a second (the kernel's outputs are then undefined).  The
- * call synchronises the device (it is a plain copy from device memory) and, if
+ * part of their work: AROPS_DEVICE_ERR_TIMEOUT means a bulk copy into shared
+ * memory did not complete within a second (the kernel's outputs are then
+ * undefined); AROPS_DEVICE_ERR_BAD_INDEX (see arops_mrope_kv_append) means a
+ * token's cache slot was out of range and was not written.  The call
+ * synchronises the device (it is a plain copy from device memory) and, if
  * `clear` is non-zero, resets the bits.  Healthy runs always read 0.
  */
 #define AROPS_DEVICE_ERR_TIMEOUT 1u

@@ -227,15 +227,24 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
  * such as code running inside a host application's real-time audio or
  * streaming callback, where cudaMalloc is not allowed because it can block
  * and synchronise the device, or a plugin that only receives buffers from a
- * host that owns all device memory.  This entry point itself allocates
- * nothing and calls no allocating routine.
+ * host that owns all device memory.  This entry point calls no cudaMalloc,
+ * cudaFree or other allocating routine (the one-time module load of the
+ * set-up call below aside).
  *   - Limit: rows * ceil(vocab / 4096) * top_k * 8 bytes must not exceed 1 MiB
  *     (e.g. vocab 151936, top_k 50: up to 68 rows); larger shapes return
  *     AROPS_ERR_UNSUPPORTED with the numbers in arops_last_error(), before
  *     anything is launched.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on the device.
+ *   - The array has one instance per CUDA context.  Every call looks up its
+ *     address in the caller's current context (cudaGetSymbolAddress), so a
+ *     context the caller created itself, or a primary context that was reset
+ *     and created anew, gets its own instance.
+ *   - Set-up: a call with rows == 0 launches nothing but performs that lookup;
+ *     the first lookup in a context loads the library's device code there
+ *     (CUDA loads modules lazily by default), which reserves the array and may
+ *     synchronise the device.  Callers whose later calls run where that is not
+ *     allowed (a real-time callback) make one such call per context at set-up,
+ *     outside that path and before any stream capture.  After it, calls
+ *     allocate nothing and call no allocating routine.
  *   - All calls share the one array and it keeps the previous call's contents;
  *     no part of it needs to start at zero, since every slot a call reads is
  *     written earlier in that same call.  Calls whose kernels overlap on the

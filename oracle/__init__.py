@@ -291,19 +291,26 @@ class Oracle:
                                           layer_inputs["beta_" + key][layer], eps, dtype)
             return self.add_rmsnorm(x, r, layer_inputs["gamma_" + key][layer], eps, dtype)
 
+        m = self.mutant  # planted plumbing mistakes 19-22 (0: none)
+        if m == 22:
+            pos = pos + 1  # planted: positions one step ahead
         for layer in range(len(layer_inputs["x_attn"])):
             y, res = add_norm(layer_inputs["x_attn"][layer], res, "attn", layer)
+            mlp_key = "attn" if m == 21 else "mlp"  # 21 planted: the MLP norm takes the attention weights
             if not outputs:
-                _, res = add_norm(layer_inputs["x_mlp"][layer], res, "mlp", layer)
+                _, res = add_norm(layer_inputs["x_mlp"][layer], res, mlp_key, layer)
                 continue
             outs["y_attn"].append(self.round_to(y, dtype))
             qo, ko = self.mrope_qk(layer_inputs["q"][layer], layer_inputs["k"][layer], pos,
                                    sections, theta)
             outs["q"].append(self.round_to(qo, dtype))
-            outs["k"].append(self.round_to(ko, dtype))
-            y, res = add_norm(layer_inputs["x_mlp"][layer], res, "mlp", layer)
+            outs["k"].append(self.round_to(qo if m == 20 else ko, dtype))  # 20 planted: q for k
+            y, res = add_norm(layer_inputs["x_mlp"][layer], res, mlp_key, layer)
             outs["y_mlp"].append(self.round_to(y, dtype))
-            act = self.swiglu(layer_inputs["gate"][layer], layer_inputs["up"][layer])
+            g, u = layer_inputs["gate"][layer], layer_inputs["up"][layer]
+            if m == 19:
+                g, u = u, g  # planted: gate and up swapped
+            act = self.swiglu(g, u)
             outs["act"].append(self.round_to(act, dtype))
         if not outputs:
             outs = {}

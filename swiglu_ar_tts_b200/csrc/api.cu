@@ -54,26 +54,13 @@ bool valid_dtype(arops_dtype d)
 // out) OR a bit into it; arops_device_errors reads and clears it.
 __device__ unsigned int g_device_errors = 0;
 
-namespace {
-std::atomic<unsigned*> g_error_word[kMaxDevices];
-}
-
+// Looked up on every call rather than cached per device ordinal: a __device__
+// variable has one instance per CUDA context, and the caller's current context
+// need not be the one a cached address came from (a context of its own, or a
+// primary context reset and created anew).
 cudaError_t device_error_word(unsigned** word)
 {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess)
-        return err;
-    unsigned* p = (dev >= 0 && dev < kMaxDevices) ? g_error_word[dev].load() : nullptr;
-    if (p == nullptr) {
-        err = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_errors);
-        if (err != cudaSuccess)
-            return err;
-        if (dev >= 0 && dev < kMaxDevices)
-            g_error_word[dev].store(p);
-    }
-    *word = p;
-    return cudaSuccess;
+    return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_device_errors);
 }
 
 cudaError_t current_device_info(DeviceInfo* info)
@@ -112,10 +99,6 @@ void count_launch()
 }  // namespace arops
 
 using namespace arops;
-
-extern "C" {
-
-}  // extern "C"
 
 namespace {
 
@@ -377,10 +360,6 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
         topk_check("arops_topk_sample_noalloc", rows, vocab, top_k, temperature);
     if (st != AROPS_OK)
         return st;
-    if (rows == 0)
-        return ok();
-    if (!logits || !gumbel || !token_out || !prob_out)
-        return fail(AROPS_ERR_INVALID, "arops_topk_sample_noalloc: null pointer");
     const size_t need = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * 8u;
     if (need > topk_noalloc_scratch_bytes())
         return fail(AROPS_ERR_UNSUPPORTED,
@@ -388,10 +367,16 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
                     "(rows x ceil(vocab/4096) x top_k x 8) but the built-in array holds %zu; "
                     "use arops_topk_sample with a caller workspace",
                     need, topk_noalloc_scratch_bytes());
+    // resolved before the rows == 0 return, so that a call with no rows is the
+    // set-up call: it makes the current context load this code and its array
     uint64_t* scratch = nullptr;
     cudaError_t err = topk_noalloc_scratch(&scratch);
     if (err != cudaSuccess)
         return from_cuda(err, "arops_topk_sample_noalloc (scratch address)");
+    if (rows == 0)
+        return ok();
+    if (!logits || !gumbel || !token_out || !prob_out)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample_noalloc: null pointer");
     return from_cuda(launch_topk_sample(logits, gumbel, token_out, prob_out, rows, vocab, top_k,
                                         temperature, dtype, scratch,
                                         static_cast<cudaStream_t>(stream)),

@@ -91,8 +91,9 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     constexpr int G = 32 / P;                // heads per warp pass
     constexpr int HALF = P * E;              // head_dim / 2
     constexpr int D = 2 * HALF;
-    constexpr int F = (E >= G) ? E / G : 1;
-    constexpr bool kStream = U > 1;  // one pass per warp: decode-size launches  // angles evaluated per lane
+    constexpr int F = (E >= G) ? E / G : 1;  // angles evaluated per lane
+    // evict-first stores, except with one pass per warp (U == 1: decode-size launches)
+    constexpr bool kStream = U > 1;
     const int lane = threadIdx.x & 31;
     const int pv = lane % P;
     const int hg = lane / P;

@@ -26,7 +26,6 @@
 // is read, so it needs no clearing.
 #include <math.h>
 
-#include <atomic>
 #include <type_traits>
 
 #include "common.cuh"
@@ -546,36 +545,22 @@ constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
 
 static __device__ __align__(256) uint64_t g_topk_scratch[kNoAllocScratchBytes / sizeof(uint64_t)];
 
-namespace {
-constexpr int kScratchDevices = 64;
-std::atomic<uint64_t*> g_topk_scratch_addr[kScratchDevices];
-}  // namespace
-
 size_t topk_noalloc_scratch_bytes()
 {
     return kNoAllocScratchBytes;
 }
 
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// Device address of the scratch array in the current context.  In host code
+// the array's name is only a stand-in, so the address is looked up with
+// cudaGetSymbolAddress, on every call: the array has one instance per CUDA
+// context, and a cached address could belong to another context than the
+// caller's current one (a context the caller created itself, or a primary
+// context that was reset and created anew).  Once this code is loaded in the
+// context the lookup allocates nothing; the first lookup in a context loads it
+// (with lazy module loading, the CUDA default), which reserves the array.
 cudaError_t topk_noalloc_scratch(uint64_t** ptr)
 {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess)
-        return err;
-    if (dev < 0 || dev >= kScratchDevices)
-        return cudaErrorInvalidDevice;
-    uint64_t* p = g_topk_scratch_addr[dev].load();
-    if (p == nullptr) {
-        err = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_topk_scratch);
-        if (err != cudaSuccess)
-            return err;
-        g_topk_scratch_addr[dev].store(p);
-    }
-    *ptr = p;
-    return cudaSuccess;
+    return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_topk_scratch);
 }
 
 }  // namespace arops

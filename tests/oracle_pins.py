@@ -554,14 +554,70 @@ def pin_swiglu_tanh_form_and_limits(orc):
 # ---------------------------------------------------------------------------
 
 
+def _rmsnorm_torch_fp64(x, weight, eps):
+    """RMSNorm as the module of "Optimising autoregressive speech models", §09
+    ("How to swap") computes it, restated here and run by torch in fp64 on the
+    CPU: the reciprocal square root (torch.rsqrt) of the row's mean square plus
+    eps scales the row, then the weight multiplies each channel."""
+    xt = torch.as_tensor(np.asarray(x, dtype=np.float64))
+    w = torch.as_tensor(np.asarray(weight, dtype=np.float64))
+    scale = torch.rsqrt(xt.square().mean(dim=-1, keepdim=True) + eps)
+    return (xt * scale * w).numpy()
+
+
+def pin_rmsnorm_matches_section09_module_in_torch(orc):
+    """The oracle agrees with the §09 RMSNorm module run in torch fp64 (its
+    rsqrt-then-multiply order against the oracle's divide by sqrt) to ~1e-15,
+    and with torch's own fp64 rms_norm routine, on rows of mixed scale."""
+    rng = np.random.default_rng(60)
+    for rows, hidden, eps in ((7, 2048, 1e-6), (5, 1024, 1e-6), (3, 96, 0.25), (4, 33, 0.0)):
+        x = rng.standard_normal((rows, hidden)) * rng.uniform(1e-3, 30, size=(rows, 1))
+        w = 1.0 + 0.1 * rng.standard_normal(hidden)
+        y = orc.rmsnorm(x, w, eps)
+        np.testing.assert_allclose(y, _rmsnorm_torch_fp64(x, w, eps), rtol=4e-15, atol=1e-300)
+        lib = torch.nn.functional.rms_norm(torch.from_numpy(x), (hidden,), torch.from_numpy(w),
+                                           eps).numpy()
+        np.testing.assert_allclose(y, lib, rtol=4e-15, atol=1e-300)
+
+
+def pin_layernorm_matches_torch_layer_norm(orc):
+    """The oracle's LayerNorm agrees with torch's fp64 layer_norm (population
+    variance, eps inside the root, gamma and beta per channel)."""
+    rng = np.random.default_rng(61)
+    for rows, hidden, eps in ((6, 2048, 1e-6), (3, 40, 1e-2)):
+        x = rng.standard_normal((rows, hidden)) * 3 + rng.uniform(-5, 5, size=(rows, 1))
+        g = 1.0 + 0.1 * rng.standard_normal(hidden)
+        b = 0.1 * rng.standard_normal(hidden)
+        lib = torch.nn.functional.layer_norm(torch.from_numpy(x), (hidden,), torch.from_numpy(g),
+                                             torch.from_numpy(b), eps).numpy()
+        np.testing.assert_allclose(orc.layernorm(x, g, b, eps), lib, rtol=1e-13, atol=1e-14)
+
+
+def _half_ulp_close(got, exact, what):
+    """got is exact rounded to bf16: within half a bf16 ulp, i.e. 2^-8 |exact|
+    (plus a floor far below any value used here)."""
+    exact = np.asarray(exact, dtype=np.float64)
+    assert got.shape == exact.shape, (what, got.shape, exact.shape)
+    bad = np.abs(got - exact) > 2.0 ** -8 * np.abs(exact) + 1e-30
+    assert not bad.any(), f"{what}: {np.count_nonzero(bad)} elements off"
+
+
 def pin_decode_chain(orc):
-    """Over several steps the residual is the bf16 rounding, after every add, of
-    the running sum (torch fp32 add + bf16 cast); the attention-side norm of
-    each layer equals RMSNorm of that residual; at step s every q/k head is
-    1-D RoPE at position s (all three rows equal)."""
+    """Every output of the oracle's decode step against statements that do not
+    use the oracle's operators, over several steps of a small chain:
+      residual  the bf16 rounding, after every add, of the running sum (torch
+                fp32 add + bf16 cast);
+      y_attn    the §09 RMSNorm module in torch fp64 of the residual after the
+                attention-side add, with that layer's attention weights;
+      y_mlp     the same of the residual after the MLP-side add, with the MLP
+                weights;
+      q, k      1-D RoPE at position s written as a complex multiplication (all
+                three position rows equal the step s);
+      act       silu(gate) * up with the logistic written through tanh."""
     rng = np.random.default_rng(50)
     B, H, I, hq, hk, d, L = 2, 64, 96, 2, 1, 16, 3
     sections = (3, 3, 2)
+    eps = 1e-6
 
     def bf(shape, std=1.0, mean=0.0):
         return torch.from_numpy(rng.standard_normal(shape) * std + mean).float().bfloat16()
@@ -579,17 +635,32 @@ def pin_decode_chain(orc):
     res0 = bf((B, H), 2.0)
     res = res0.double().numpy()
     run = res0.clone()
+    f64 = lambda t: t.double().numpy()  # noqa: E731
     for step in range(4):
-        res, outs = orc.decode_step(res, inp, step, 1e-6, 1e6, sections, "bf16")
+        prev = res
+        res, outs = orc.decode_step(res, inp, step, eps, 1e6, sections, "bf16")
+        p = np.full(B, float(step))
         for layer in range(L):
             run_attn = (inp["x_attn"][layer].float() + run.float()).bfloat16()
-            y_ref = orc.round_to(orc.rmsnorm(run_attn, inp["gamma_attn"][layer], 1e-6), "bf16")
-            assert np.array_equal(outs["y_attn"][layer], y_ref)
+            _half_ulp_close(outs["y_attn"][layer],
+                            _rmsnorm_torch_fp64(f64(run_attn), f64(inp["gamma_attn"][layer]), eps),
+                            f"y_attn step {step} layer {layer}")
             run = (inp["x_mlp"][layer].float() + run_attn.float()).bfloat16()
-            p = np.full(B, float(step))
-            qref = _rope_1d_complex(inp["q"][layer].double().numpy(), p, 1e6)
-            assert np.max(np.abs(outs["q"][layer] - qref)) <= 2.0 ** -8 * max(1.0, np.max(np.abs(qref)))
+            _half_ulp_close(outs["y_mlp"][layer],
+                            _rmsnorm_torch_fp64(f64(run), f64(inp["gamma_mlp"][layer]), eps),
+                            f"y_mlp step {step} layer {layer}")
+            _half_ulp_close(outs["q"][layer], _rope_1d_complex(f64(inp["q"][layer]), p, 1e6),
+                            f"q step {step} layer {layer}")
+            _half_ulp_close(outs["k"][layer], _rope_1d_complex(f64(inp["k"][layer]), p, 1e6),
+                            f"k step {step} layer {layer}")
+            _half_ulp_close(outs["act"][layer],
+                            _silu_tanh(f64(inp["gate"][layer])) * f64(inp["up"][layer]),
+                            f"act step {step} layer {layer}")
         assert np.array_equal(res, run.double().numpy())
+        # the residual-only form of the step (outputs=False) carries the same residual
+        res_only, none = orc.decode_step(prev, inp, step, eps, 1e6, sections, "bf16",
+                                         outputs=False)
+        assert none == {} and np.array_equal(res_only, res)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

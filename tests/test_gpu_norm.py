@@ -7,7 +7,7 @@ import oracle
 import swiglu_ar_tts_b200 as ops
 from swiglu_ar_tts_b200 import inputs
 from gpu_util import Guarded, dev, misaligned, resident_threads
-from tolerance import check, to_f64
+from tolerance import LN_BAND, check, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -225,7 +225,7 @@ def test_layernorm_shapes(dtype, hidden):
     torch.cuda.synchronize()
     exact = oracle.get().layernorm(x, inp["gamma"], inp["beta"], EPS)
     scale = _ln_scale(to_f64(x), to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
-    check(y, exact, dtype, scale, what=f"layernorm {dtype} {rows}x{hidden}")
+    check(y, exact, dtype, scale, what=f"layernorm {dtype} {rows}x{hidden}", band=LN_BAND)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -241,7 +241,7 @@ def test_add_layernorm_shapes_past_one_wave(dtype, hidden):
                                                   inp["beta"], EPS, dtype)
     assert np.array_equal(to_f64(r_out), r_exact)
     scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
-    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}")
+    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}", band=LN_BAND)
 
 
 @pytest.mark.parametrize("in_place", [False, True])
@@ -255,7 +255,7 @@ def test_add_layernorm_bf16_4096x2048(in_place):
                                                   inp["beta"], EPS, "bf16")
     assert np.array_equal(to_f64(r_out), r_exact), "residual_out must be bit-exact"
     scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
-    check(y, y_exact, "bf16", scale, what="add_layernorm 4096x2048")
+    check(y, y_exact, "bf16", scale, what="add_layernorm 4096x2048", band=LN_BAND)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -270,7 +270,7 @@ def test_add_layernorm_shapes(dtype, hidden):
                                                   inp["beta"], EPS, dtype)
     assert np.array_equal(to_f64(r_out), r_exact)
     scale = _ln_scale(r_exact, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS)
-    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}")
+    check(y, y_exact, dtype, scale, what=f"add_layernorm {dtype} {rows}x{hidden}", band=LN_BAND)
 
 
 def test_layernorm_constant_rows_give_beta_and_guarded():
@@ -290,4 +290,5 @@ def test_layernorm_misaligned():
     y = ops.layernorm(misaligned(dev(inp["x"])), dev(inp["gamma"]), misaligned(dev(inp["beta"])), EPS)
     torch.cuda.synchronize()
     exact = oracle.get().layernorm(inp["x"], inp["gamma"], inp["beta"], EPS)
-    check(y, exact, "bf16", _ln_scale(to_f64(inp["x"]), to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS))
+    check(y, exact, "bf16", _ln_scale(to_f64(inp["x"]), to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS),
+          band=LN_BAND)

@@ -29,6 +29,11 @@ MUTANTS = {
     16: "sampling probability without the temperature",
     17: "KV cache row and position swapped",
     18: "k written into the V cache",
+    # decode-step plumbing (oracle/__init__.py, Oracle.decode_step)
+    19: "decode step: SwiGLU with gate and up swapped",
+    20: "decode step: rotated q reported where k belongs",
+    21: "decode step: MLP-side norm with the attention-side weights",
+    22: "decode step: positions one step ahead",
 }
 
 

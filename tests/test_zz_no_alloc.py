@@ -2,7 +2,8 @@
 
 arops_topk_sample_noalloc serves callers that cannot allocate device memory
 (for example code inside a host application's real-time audio callback, where
-cudaMalloc may block and synchronise the device): it takes its scratch from a
+cudaMalloc may block and synchronise the device, or a plugin that only receives
+buffers from a host that owns all device memory): it takes its scratch from a
 1 MiB array the library keeps in device memory.  This file is collected last
 (after every other test) and also passes when run alone in a fresh process.
 """
@@ -12,12 +13,15 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import swiglu_ar_tts_b200 as ops
 from swiglu_ar_tts_b200 import inputs
+from tolerance import to_f64
 
 pytestmark = pytest.mark.gpu
 
 _vp = ctypes.c_void_p
+_DT = {"f32": 0, "bf16": 1}
 
 
 def _lib():
@@ -29,36 +33,62 @@ def _lib():
     return L
 
 
-def _with_workspace(L, logits, gumbel, rows, vocab, k, temp, stream):
+def _noalloc(L, logits, gumbel, rows, vocab, k, temp, dtype, stream):
+    tok = torch.full((rows,), -1, dtype=torch.int32, device="cuda")
+    prob = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    st = L.arops_topk_sample_noalloc(logits.data_ptr(), gumbel.data_ptr(), tok.data_ptr(),
+                                     prob.data_ptr(), rows, vocab, k, temp, _DT[dtype], stream)
+    assert st == 0, L.arops_last_error()
+    return tok, prob
+
+
+def _with_workspace(L, logits, gumbel, rows, vocab, k, temp, dtype, stream):
     n = ctypes.c_size_t(0)
     assert L.arops_topk_sample_workspace(rows, vocab, k, ctypes.byref(n)) == 0
     ws = torch.empty(n.value, dtype=torch.uint8, device="cuda")
     tok = torch.empty(rows, dtype=torch.int32, device="cuda")
     prob = torch.empty(rows, dtype=torch.float32, device="cuda")
     st = L.arops_topk_sample(logits.data_ptr(), gumbel.data_ptr(), tok.data_ptr(), prob.data_ptr(),
-                             rows, vocab, k, temp, 1, ws.data_ptr(), n.value, stream)
+                             rows, vocab, k, temp, _DT[dtype], ws.data_ptr(), n.value, stream)
     assert st == 0, L.arops_last_error()
     return tok, prob
 
 
-def test_noalloc_matches_workspace_entry_point_two_calls():
+def test_noalloc_setup_call_launches_nothing():
+    """rows == 0 is the set-up call: it resolves the array in the current
+    context and launches nothing."""
+    L = _lib()
+    before = L.arops_launch_count()
+    st = L.arops_topk_sample_noalloc(None, None, None, None, 0, 151936, 50, 1.0, 1, None)
+    assert st == 0, L.arops_last_error()
+    assert L.arops_launch_count() == before
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_noalloc_two_calls_match_workspace_entry_point_and_oracle(dtype):
+    """Two calls in a row, each compared with the workspace entry point and with
+    the oracle.  The first call's logits sit 100 above the second's, so a key
+    the second call read from the first call's leftover scratch (instead of
+    writing it first) would outrank every real candidate and change the token."""
     L = _lib()
     stream = torch.cuda.current_stream().cuda_stream
-    # two calls in a row, different shapes: the second runs on the first's
-    # leftover scratch contents
-    for rows, vocab, k, temp, seed in ((5, 151936, 50, 0.8, 1), (17, 30000, 64, 1.3, 2)):
-        inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=seed)
-        logits = inp["logits"].cuda()
+    orc = oracle.get()
+    cases = ((5, 151936, 50, 0.8, 1, 100.0), (17, 30000, 64, 1.3, 2, 0.0))
+    for rows, vocab, k, temp, seed, shift in cases:
+        inp = inputs.topk_inputs(rows, vocab, k, dtype, seed=seed)
+        logits_host = (inp["logits"].float() + shift).to(inp["logits"].dtype)
+        logits = logits_host.cuda()
         gumbel = inp["gumbel"].cuda()
-        tok = torch.full((rows,), -1, dtype=torch.int32, device="cuda")
-        prob = torch.zeros(rows, dtype=torch.float32, device="cuda")
-        st = L.arops_topk_sample_noalloc(logits.data_ptr(), gumbel.data_ptr(), tok.data_ptr(),
-                                         prob.data_ptr(), rows, vocab, k, temp, 1, stream)
-        assert st == 0, L.arops_last_error()
-        t_ref, p_ref = _with_workspace(L, logits, gumbel, rows, vocab, k, temp, stream)
+        tok, prob = _noalloc(L, logits, gumbel, rows, vocab, k, temp, dtype, stream)
         torch.cuda.synchronize()
-        assert torch.equal(tok, t_ref)
-        np.testing.assert_allclose(prob.cpu().numpy(), p_ref.cpu().numpy(), rtol=1e-5, atol=0)
+        assert ops.device_errors(clear=True) == 0
+        t_ws, p_ws = _with_workspace(L, logits, gumbel, rows, vocab, k, temp, dtype, stream)
+        torch.cuda.synchronize()
+        t_orc, p_orc = orc.topk_sample(logits_host, inp["gumbel"], k, temp)
+        assert np.array_equal(tok.cpu().numpy(), t_orc)
+        np.testing.assert_allclose(to_f64(prob), p_orc, rtol=1e-5, atol=0)
+        assert torch.equal(tok, t_ws)
+        assert torch.equal(prob, p_ws)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():

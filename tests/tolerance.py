@@ -25,8 +25,13 @@ than 1e-5 of their size.
 On top of the element-wise check, every comparison also requires
 cosine(gpu, exact) >= 0.99999 in fp64 and max relative error <= 8e-3 (bf16) or
 1e-5 (fp32) over the elements with |exact| >= 1e-3 * rms(exact) and, where a
-cancellation scale is given (M-RoPE, LayerNorm), |exact| >= 0.5 * scale, i.e.
-away from cancellation (an output that keeps half of its operands' size).
+cancellation scale is given, |exact| >= band * scale, i.e. away from
+cancellation.  For M-RoPE band = 0.05 (an output that keeps a twentieth of its
+operands' size).  LayerNorm passes band = LN_BAND = 0.5: its fp32 outputs are
+held to 1e-5 relative, and at |exact| = 0.05 * scale its cancellation
+allowance 2^-19 * scale alone is 3.8e-5 of the output, so the relative bar
+there would contradict the allowance derived from the arithmetic; at 0.5 *
+scale the allowance is 3.8e-6 of the output, inside the 1e-5 bar.
 """
 from __future__ import annotations
 
@@ -58,8 +63,12 @@ def cosine(a: np.ndarray, b: np.ndarray) -> float:
     return float(np.dot(a, b) / (na * nb))
 
 
+# relative-error band of the LayerNorm comparisons (see the module docstring)
+LN_BAND = 0.5
+
+
 def check(gpu: torch.Tensor, exact: np.ndarray, dtype: str, cancel_scale: np.ndarray | None = None,
-          what: str = "") -> dict:
+          what: str = "", band: float = 0.05) -> dict:
     """Assert that ``gpu`` matches the unrounded fp64 oracle result ``exact``."""
     g = to_f64(gpu)
     exact = np.asarray(exact, dtype=np.float64)
@@ -104,8 +113,8 @@ def check(gpu: torch.Tensor, exact: np.ndarray, dtype: str, cancel_scale: np.nda
     rms = np.sqrt(np.mean(exact_f ** 2))
     big = np.abs(exact_f) >= 1e-3 * rms
     if cancel_scale is not None:
-        # away from cancellation: the result keeps at least half of its operands' size
-        big &= np.abs(exact_f) >= 0.5 * np.asarray(cancel_scale, dtype=np.float64)[fin]
+        # away from cancellation: the result keeps `band` of its operands' size
+        big &= np.abs(exact_f) >= band * np.asarray(cancel_scale, dtype=np.float64)[fin]
     if big.any():
         rel = np.max(np.abs(g[big] - exact_f[big]) / np.abs(exact_f[big]))
         assert rel <= (8e-3 if dtype == "bf16" else 1e-5), f"{what}: max rel err {rel}"

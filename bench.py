@@ -29,8 +29,8 @@ Multi-GPU (torchrun, one process per GPU): every rank runs the same step on its
 own GPU (replicas; the operators have no exchange step).  Times are the max
 over ranks; value is the total bytes of all ranks over that time.
 
-``--impl reference`` times the fp64 CPU oracle instead, on a 1/16 sample of the
-same step (rank 0 only).
+``--impl reference`` times the plain single-threaded fp64 CPU oracle instead, on
+the same whole step (rank 0 only; other ranks exit at once).
 """
 from __future__ import annotations
 
@@ -212,14 +212,9 @@ class Step:
         self.chain5.capture()
         self.chain256.capture()
         self.decode_step_index = 0
-        self.bytes = {
-            "rmsnorm": (2 * 64 * 1024 + 1024) * 4,
-            "add_rmsnorm": (4 * 4096 * 2048 + 2048) * 2,
-            "swiglu": 3 * 8192 * 6144 * 2,
-            "mrope_qk": 2 * 4096 * (16 + 8) * 128 * 2 + 3 * 4096 * 4,
-            "decode_b5": self.chain5.bytes_per_step(),
-            "decode_b256": self.chain256.bytes_per_step(),
-        }
+        self.bytes = step_bytes()
+        assert self.bytes["decode_b5"] == self.chain5.bytes_per_step()
+        assert self.bytes["decode_b256"] == self.chain256.bytes_per_step()
         # rows (tokens) one launch of each operator processes
         self.rows = {"rmsnorm": 64, "add_rmsnorm": 4096, "swiglu": 8192, "mrope_qk": 4096,
                      "decode_b5": 5, "decode_b256": 256}
@@ -253,9 +248,12 @@ class Step:
             self.chain256._graph.replay()
 
     def run(self, events=None) -> None:
-        """One step; ``events`` (2 per operator) bracket each operator."""
-        for i, name in enumerate(self.OPS):
+        """One step; ``events`` (2 per operator) bracket each operator.  The
+        step's set-up (the decode position ids) is enqueued before the first
+        event, so it falls outside every timed window and the step's time."""
+        for name in self.OPS:
             self.prepare_op(name)
+        for i, name in enumerate(self.OPS):
             if events is not None:
                 events[2 * i].record()
             self.run_op(name)
@@ -437,80 +435,199 @@ def decode_split(chain, reps: int = 10) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# each operator alone, inputs rotated through >= 4x L2
+# ---------------------------------------------------------------------------
+ISOLATED = (("rmsnorm", "rmsnorm"), ("add_rmsnorm", "add_rmsnorm"), ("swiglu", "swiglu"),
+            ("mrope_qk", "mrope_qk"), ("decode5", "decode_b5"), ("decode256", "decode_b256"))
+
+
+def isolated_ops(device, peak: float, peak_kind: str, launches: int = 100) -> dict:
+    """Each operator on its own, outside the timed steps: enough copies of its
+    buffers to cover 512 MB (4x L2; a decode step at batch 256 is 588 MB in one
+    copy), launches cycling through them so every launch reads from DRAM and
+    pays for earlier launches' write-backs.  ``us_median``: the median over
+    ``launches`` launches, each bracketed by its own CUDA events (launched
+    without programmatic dependent launch, so each starts on an idle GPU).
+    ``us_back_to_back``: the same launches enqueued back to back with
+    programmatic dependent launch between one pair of events, per launch (each
+    launch overlaps its predecessor's drain, as inside a step)."""
+    import swiglu_ar_tts_b200 as ops
+    from swiglu_ar_tts_b200 import opbench
+
+    out = {}
+    old = ops.set_pdl(False)
+    try:
+        for op, key in ISOLATED:
+            fns, nbytes, desc = opbench.make_rotation(op, None, device, None)
+            ops.set_pdl(False)
+            us = opbench.time_op(fns, launches)
+            ops.set_pdl(True)
+            for f in fns:
+                f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            torch.cuda._sleep(int(1e7))
+            e0.record()
+            for i in range(launches):
+                fns[i % len(fns)]()
+            e1.record()
+            torch.cuda.synchronize()
+            b2b = 1e3 * e0.elapsed_time(e1) / launches
+            med = statistics.median(us)
+            gbs = nbytes / (med * 1e-6) / 1e9
+            gbs_b2b = nbytes / (b2b * 1e-6) / 1e9
+            out[key] = {"shape": desc, "bytes": nbytes, "launches": launches,
+                        "us_median": round(med, 3), "us_min": round(min(us), 3),
+                        "gbs_median": round(gbs, 1),
+                        "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
+                        "us_back_to_back": round(b2b, 3), "gbs_back_to_back": round(gbs_b2b, 1),
+                        "frac_back_to_back": round(gbs_b2b / peak, 4)}
+            del fns
+            torch.cuda.empty_cache()
+    finally:
+        ops.set_pdl(old)
+    return out
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timings
 # ---------------------------------------------------------------------------
-def oracle_step(fraction: int = 1, decode_b256_rows: int | None = None) -> tuple[float, int, str]:
-    """Time the fp64 oracle on one step of the workload, every operator on 1/
-    ``fraction`` of its rows.  Returns (seconds, algorithmic bytes, description)."""
-    import oracle
-    from swiglu_ar_tts_b200 import inputs
+STEP_CONFIGS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode_b5", "decode_b256")
 
-    orc = oracle.get()
-    f64 = lambda t: t.detach().to(torch.float64).numpy()  # noqa: E731
-    r_add = 4096 // fraction
-    r_sw = 8192 // fraction
-    t_mr = 4096 // fraction
-    b256 = decode_b256_rows if decode_b256_rows is not None else max(1, 256 // fraction)
-    rn = inputs.rmsnorm_inputs(64, 1024, "f32", 0)
-    an = inputs.add_rmsnorm_inputs(r_add, 2048, "bf16", 0)
-    sw = inputs.swiglu_inputs(r_sw, 6144, "bf16", 0)
-    mr = inputs.mrope_inputs(t_mr)
-    c5 = inputs.decode_chain_inputs(inputs.ChainShape(batch=5))
-    c256 = inputs.decode_chain_inputs(inputs.ChainShape(batch=b256), seed=1000)
-    # operands widened to fp64 up front: the oracle's input format
-    rn = {k: f64(v) for k, v in rn.items()}
-    an = {k: f64(v) for k, v in an.items()}
-    sw = {k: f64(v) for k, v in sw.items()}
-    pos = mr["pos"].numpy()
-    mr = {k: f64(v) for k, v in mr.items() if k != "pos"}
-    chains = []
-    for c in (c5, c256):
-        chains.append((f64(c["residual"]),
-                       {k: [f64(t) for t in v] for k, v in c.items() if k != "residual"}))
-    t0 = time.perf_counter()
-    orc.round_to(orc.rmsnorm(rn["x"], rn["gamma"], 1e-6), "f32")
-    y, _ = orc.add_rmsnorm(an["x"], an["residual"], an["gamma"], 1e-6, "bf16")
-    orc.round_bf16(y)
-    orc.round_bf16(orc.swiglu(sw["gate"], sw["up"]))
-    qo, ko = orc.mrope_qk(mr["q"], mr["k"], pos, (24, 20, 20), 1e6)
-    orc.round_bf16(qo)
-    orc.round_bf16(ko)
-    for res, layer_inputs in chains:
-        orc.decode_step(res, layer_inputs, 0)
-    dt = time.perf_counter() - t0
-    per_row_layer = 81932
-    nbytes = ((2 * 64 * 1024 + 1024) * 4 + (4 * r_add * 2048 + 2048) * 2 + 3 * r_sw * 6144 * 2
-              + 2 * t_mr * 24 * 128 * 2 + 3 * t_mr * 4
-              + 28 * (5 * per_row_layer + 4 * 2048 * 2) + 28 * (b256 * per_row_layer + 4 * 2048 * 2))
-    desc = (f"one step with every operator on 1/{fraction} of its rows: rmsnorm 64x1024, "
-            f"add_rmsnorm {r_add}x2048, swiglu {r_sw}x6144, mrope {t_mr} tokens, decode 28 layers "
-            f"at batch 5 and at batch {b256}; single-threaded C oracle, fp64")
-    return dt, nbytes, desc
+
+def step_bytes() -> dict:
+    """Algorithmic HBM bytes of each operator of the step (every operand read
+    once, every output written once)."""
+    per_row_layer = 2 * 4 * 2048 * 2 + 2 * (16 + 8) * 128 * 2 + 3 * 4 + 3 * 6144 * 2  # 81,932
+    gammas = 2 * 2048 * 2  # two norm weights per layer
+    return {
+        "rmsnorm": (2 * 64 * 1024 + 1024) * 4,
+        "add_rmsnorm": (4 * 4096 * 2048 + 2048) * 2,
+        "swiglu": 3 * 8192 * 6144 * 2,
+        "mrope_qk": 2 * 4096 * (16 + 8) * 128 * 2 + 3 * 4096 * 4,
+        "decode_b5": 28 * (5 * per_row_layer + gammas),
+        "decode_b256": 28 * (256 * per_row_layer + gammas),
+    }
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+class OracleStep:
+    """The whole step (every configuration at full size) on the fp64 CPU
+    oracle, from the same seeded inputs as the GPU step, widened to fp64 once
+    up front (the oracle's input format).  ``run`` returns seconds per
+    configuration; each output is rounded to its dtype as the GPU writes it."""
+
+    def __init__(self):
+        from swiglu_ar_tts_b200 import inputs
+
+        f64 = lambda t: t.detach().to(torch.float64).numpy()  # noqa: E731
+        self.rn = {k: f64(v) for k, v in inputs.rmsnorm_inputs(64, 1024, "f32", 0).items()}
+        self.an = {k: f64(v) for k, v in inputs.add_rmsnorm_inputs(4096, 2048, "bf16", 0).items()}
+        self.sw = {k: f64(v) for k, v in inputs.swiglu_inputs(8192, 6144, "bf16", 0).items()}
+        mr = inputs.mrope_inputs(4096)
+        self.pos = mr["pos"].numpy()
+        self.mr = {k: f64(v) for k, v in mr.items() if k != "pos"}
+        self.chains = {}
+        for name, batch, seed in (("decode_b5", 5, 0), ("decode_b256", 256, 1000)):
+            c = inputs.decode_chain_inputs(inputs.ChainShape(batch=batch), seed=seed)
+            self.chains[name] = (f64(c["residual"]),
+                                 {k: [f64(t) for t in v] for k, v in c.items() if k != "residual"})
+        self.bytes = step_bytes()
+        self.sample = ("the whole step at full size: rmsnorm f32 64x1024, add_rmsnorm bf16 "
+                       "4096x2048, swiglu bf16 8192x6144, mrope bf16 4096 tokens, one 28-layer "
+                       "decode step at batch 5 and at batch 256 (every output of every layer)")
+
+    def run(self, orc) -> dict:
+        t = {}
+        c0 = time.perf_counter()
+        orc.round_to(orc.rmsnorm(self.rn["x"], self.rn["gamma"], 1e-6), "f32")
+        c1 = time.perf_counter()
+        t["rmsnorm"] = c1 - c0
+        y, _ = orc.add_rmsnorm(self.an["x"], self.an["residual"], self.an["gamma"], 1e-6, "bf16")
+        orc.round_bf16(y)
+        c2 = time.perf_counter()
+        t["add_rmsnorm"] = c2 - c1
+        orc.round_bf16(orc.swiglu(self.sw["gate"], self.sw["up"]))
+        c3 = time.perf_counter()
+        t["swiglu"] = c3 - c2
+        qo, ko = orc.mrope_qk(self.mr["q"], self.mr["k"], self.pos, (24, 20, 20), 1e6)
+        orc.round_bf16(qo)
+        orc.round_bf16(ko)
+        c4 = time.perf_counter()
+        t["mrope_qk"] = c4 - c3
+        for name in ("decode_b5", "decode_b256"):
+            res, layer_inputs = self.chains[name]
+            c5 = time.perf_counter()
+            orc.decode_step(res, layer_inputs, 0)
+            t[name] = time.perf_counter() - c5
+        return t
+
+
+def cpu_baseline_report(ostep: "OracleStep") -> dict:
+    """The oracle as it stands, timed on this host's cores on the whole step:
+    the plain single-threaded build (the reported value) and the row-parallel
+    OpenMP build of the same source on every core, with ms per configuration."""
+    import oracle
+
+    runs = {}
+    for kind, orc in (("single", oracle.get()), ("omp", oracle.get_omp())):
+        t = ostep.run(orc)
+        total = sum(t.values())
+        runs[kind] = {"value": sum(ostep.bytes.values()) / total / 1e9, "unit": UNIT,
+                      "threads": orc.threads(), "ms_per_step": round(1e3 * total, 1),
+                      "per_config_ms": {k: round(1e3 * v, 2) for k, v in t.items()}}
+    single = runs["single"]
+    return {"value": single["value"], "unit": UNIT, "cores": single["threads"], "kind": "oracle",
+            "sample": ostep.sample + f"; plain single-threaded C oracle, fp64 "
+                                     f"({single['ms_per_step'] / 1e3:.1f} s)",
+            "single": single, "omp": runs["omp"],
+            "per_config_ms": single["per_config_ms"],
+            "nproc": os.cpu_count(), "affinity_cores": len(os.sched_getaffinity(0)),
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    fraction = 16
+    import oracle
+
+    ostep = OracleStep()
+    orc = oracle.get()
     times = []
-    nbytes = 0
-    desc = ""
+    per_config = {k: 0.0 for k in STEP_CONFIGS}
     for i in range(args.warmup + args.steps):
-        dt, nbytes, desc = oracle_step(fraction)
+        t = ostep.run(orc)
         if i >= args.warmup:
-            times.append(dt)
+            times.append(sum(t.values()))
+            for k, v in t.items():
+                per_config[k] += v
     total = sum(times)
-    value = nbytes * len(times) / total / 1e9
+    value = sum(ostep.bytes.values()) * len(times) / total / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": desc, "global_batch": None,
-                   "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "config": {"workload": WORKLOAD, "global_batch": None, "parallelism": "replicas x1",
+                   "sample": ostep.sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+                         "sample": ostep.sample + "; plain single-threaded C oracle, fp64",
+                         "per_config_ms": {k: round(1e3 * v / len(times), 2)
+                                           for k, v in per_config.items()},
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -713,6 +830,8 @@ def main() -> None:
         run300[f"batch{batch}"] = {"graph_us_per_step": round(t["graph"], 2),
                                    "eager_us_per_step": round(t["eager"], 2)}
 
+    iso = isolated_ops(device, peak, peak_kind)
+
     # end to end: pinned host buffers in and out, through the same public calls
     step.setup_e2e()
     torch.cuda.synchronize()
@@ -740,9 +859,7 @@ def main() -> None:
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, nbytes, desc = oracle_step(1)
-        cpu = {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": desc + f" ({dt:.1f} s)"}
+        cpu = cpu_baseline_report(OracleStep())
 
     if pg is not None:
         pg.destroy_process_group()
@@ -768,6 +885,7 @@ def main() -> None:
         "us_per_decode_step": {"batch5": ops_report["decode_b5"]["us"],
                                "batch256": ops_report["decode_b256"]["us"]},
         "ops": ops_report,
+        "ops_isolated": iso,
         "roofline": roofline,
         "roofline_swiglu": roofline_swiglu,
         "kernels": kernels,

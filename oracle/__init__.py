@@ -37,14 +37,20 @@ _c_u16_p = ctypes.POINTER(ctypes.c_uint16)
 _c_i32_p = ctypes.POINTER(ctypes.c_int32)
 
 
-def lib_path(mutant: int = 0) -> str:
+def lib_path(mutant: int = 0, omp: bool = False) -> str:
+    if omp:
+        assert mutant == 0
+        return os.path.join(_BUILD, "liboracle_omp.so")
     name = "liboracle.so" if mutant == 0 else f"liboracle_mutant{mutant}.so"
     return os.path.join(_BUILD, name)
 
 
-def build(mutant: int = 0, force: bool = False) -> str:
-    """Compile the oracle (optionally with planted mistake ``mutant``)."""
-    out = lib_path(mutant)
+def build(mutant: int = 0, force: bool = False, omp: bool = False) -> str:
+    """Compile the oracle (optionally with planted mistake ``mutant``).  With
+    ``omp`` the same source is compiled with -fopenmp into liboracle_omp.so,
+    whose marked row loops run across the host cores (the multi-core CPU
+    baseline); the plain build is the oracle the tests use."""
+    out = lib_path(mutant, omp)
     if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
         return out
     os.makedirs(_BUILD, exist_ok=True)
@@ -54,6 +60,7 @@ def build(mutant: int = 0, force: bool = False) -> str:
     # term unused, so mutants only report theirs
     warn = ["-Wall", "-Wextra", "-Wpedantic"] + (["-Werror"] if int(mutant) == 0 else [])
     cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", *warn,
+           *(["-fopenmp"] if omp else []),
            "-shared", f"-DORACLE_MUTANT={int(mutant)}", _SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
@@ -76,9 +83,10 @@ def _ptr(a: np.ndarray, ctype):
 class Oracle:
     """ctypes view of one build of the oracle library."""
 
-    def __init__(self, mutant: int = 0):
+    def __init__(self, mutant: int = 0, omp: bool = False):
         self.mutant = mutant
-        self._lib = ctypes.CDLL(build(mutant))
+        self.omp = omp
+        self._lib = ctypes.CDLL(build(mutant, omp=omp))
         L = self._lib
         L.oracle_round_bf16_array.argtypes = [_c_double_p, _c_u16_p, ctypes.c_int64]
         L.oracle_bf16_value_array.argtypes = [_c_u16_p, _c_double_p, ctypes.c_int64]
@@ -104,7 +112,12 @@ class Oracle:
             _c_i32_p, _c_i32_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int64, ctypes.c_int64, _c_i32_p, ctypes.c_double, _c_double_p]
         L.oracle_mutant.restype = ctypes.c_int
+        L.oracle_threads.restype = ctypes.c_int
         assert L.oracle_mutant() == mutant
+
+    def threads(self) -> int:
+        """Host threads this build's row loops use (1 for the plain build)."""
+        return int(self._lib.oracle_threads())
 
     # -- dtype rounding ------------------------------------------------------
     def round_bf16(self, v) -> np.ndarray:
@@ -318,6 +331,7 @@ class Oracle:
 
 
 _default: Oracle | None = None
+_omp: Oracle | None = None
 
 
 def get() -> Oracle:
@@ -326,3 +340,12 @@ def get() -> Oracle:
     if _default is None:
         _default = Oracle(0)
     return _default
+
+
+def get_omp() -> Oracle:
+    """The row-parallel (OpenMP) build of the same oracle, for timing on all
+    host cores; its results equal the plain build's bit for bit."""
+    global _omp
+    if _omp is None:
+        _omp = Oracle(0, omp=True)
+    return _omp

@@ -39,6 +39,20 @@
 #define ORACLE_MUTANT 0
 #endif
 
+/*
+ * Row-parallel build.  Compiled with -fopenmp (liboracle_omp.so, the timed
+ * multi-core baseline) the loops marked OMP_ROWS split their independent rows,
+ * tokens or elements across the host's cores; in the plain build the mark
+ * expands to nothing and every loop runs sequentially, exactly as written.
+ * Nothing else differs between the two builds.
+ */
+#ifdef _OPENMP
+#include <omp.h>
+#define OMP_ROWS _Pragma("omp parallel for schedule(static)")
+#else
+#define OMP_ROWS
+#endif
+
 /* ------------------------------------------------------------------------- */
 /* bf16 <-> fp64.                                                             */
 /* bf16 is IEEE-754 binary32 with the low 16 mantissa bits removed: 1 sign    */
@@ -113,12 +127,14 @@ double oracle_bf16_value(uint16_t b)
 
 void oracle_round_bf16_array(const double* v, uint16_t* out, int64_t n)
 {
+    OMP_ROWS
     for (int64_t i = 0; i < n; ++i)
         out[i] = oracle_round_bf16(v[i]);
 }
 
 void oracle_bf16_value_array(const uint16_t* b, double* out, int64_t n)
 {
+    OMP_ROWS
     for (int64_t i = 0; i < n; ++i)
         out[i] = oracle_bf16_value(b[i]);
 }
@@ -139,6 +155,7 @@ static double round_to_dtype(double v, int dtype)
 void oracle_rmsnorm(const double* x, const double* gamma, double* y,
                     int64_t rows, int64_t hidden, double eps)
 {
+    OMP_ROWS
     for (int64_t r = 0; r < rows; ++r) {
         const double* xr = x + r * hidden;
         double* yr = y + r * hidden;
@@ -173,6 +190,7 @@ void oracle_add_rmsnorm(const double* x, const double* residual, const double* g
                         double* y, double* residual_out,
                         int64_t rows, int64_t hidden, double eps, int dtype)
 {
+    OMP_ROWS
     for (int64_t i = 0; i < rows * hidden; ++i) {
 #if ORACLE_MUTANT == 5
         residual_out[i] = round_to_dtype(x[i] - residual[i], dtype); /* planted: sign */
@@ -195,6 +213,7 @@ void oracle_add_rmsnorm(const double* x, const double* residual, const double* g
 void oracle_layernorm(const double* x, const double* gamma, const double* beta, double* y,
                       int64_t rows, int64_t hidden, double eps)
 {
+    OMP_ROWS
     for (int64_t r = 0; r < rows; ++r) {
         const double* xr = x + r * hidden;
         double* yr = y + r * hidden;
@@ -229,6 +248,7 @@ void oracle_add_layernorm(const double* x, const double* residual, const double*
                           const double* beta, double* y, double* residual_out,
                           int64_t rows, int64_t hidden, double eps, int dtype)
 {
+    OMP_ROWS
     for (int64_t i = 0; i < rows * hidden; ++i)
         residual_out[i] = round_to_dtype(x[i] + residual[i], dtype);
     oracle_layernorm(residual_out, gamma, beta, y, rows, hidden, eps);
@@ -298,6 +318,7 @@ void oracle_mrope_qk(const double* q, const double* k, double* q_out, double* k_
                      const int32_t* pos, int64_t tokens, int n_q_heads, int n_k_heads,
                      int head_dim, const int32_t sections[3], double theta)
 {
+    OMP_ROWS
     for (int64_t t = 0; t < tokens; ++t) {
         rotate_heads(q, q_out, pos, tokens, t, n_q_heads, head_dim, sections, theta);
         rotate_heads(k, k_out, pos, tokens, t, n_k_heads, head_dim, sections, theta);
@@ -353,6 +374,7 @@ void oracle_mrope_kv_append(const double* q, const double* k, const double* v, d
 /* ------------------------------------------------------------------------- */
 void oracle_swiglu(const double* gate, const double* up, double* out, int64_t n)
 {
+    OMP_ROWS
     for (int64_t i = 0; i < n; ++i) {
         double g = gate[i];
 #if ORACLE_MUTANT == 11
@@ -438,6 +460,16 @@ void oracle_topk_sample(const double* logits, const float* gumbel, int32_t* toke
         token_out[r] = (int32_t)scratch[best].idx;
         prob_out[r] = p;
     }
+}
+
+/* Host threads the row-parallel loops use (1 in the plain build). */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /* Number of the planted mistake this build carries (0 = none). */

@@ -51,3 +51,4 @@ def _built_libraries():
 
     build.build()
     oracle.build()
+    oracle.build(omp=True)

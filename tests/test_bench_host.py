@@ -31,10 +31,43 @@ def test_decode_step_algorithmic_bytes():
 
 
 def test_prefill_algorithmic_bytes():
-    assert (2 * 64 * 1024 + 1024) * 4 == 528_384
-    assert (4 * 4096 * 2048 + 2048) * 2 == 67_112_960
-    assert 3 * 8192 * 6144 * 2 == 301_989_888
-    assert 2 * 4096 * 24 * 128 * 2 + 3 * 4096 * 4 == 50_380_800
+    b = bench.step_bytes()
+    assert b["rmsnorm"] == (2 * 64 * 1024 + 1024) * 4 == 528_384
+    assert b["add_rmsnorm"] == (4 * 4096 * 2048 + 2048) * 2 == 67_112_960
+    assert b["swiglu"] == 3 * 8192 * 6144 * 2 == 301_989_888
+    assert b["mrope_qk"] == 2 * 4096 * 24 * 128 * 2 + 3 * 4096 * 4 == 50_380_800
+    assert (b["decode_b5"], b["decode_b256"]) == (11_699_856, 587_517_952)
+    assert sum(b.values()) == 1_019_229_840
+    assert tuple(b) == bench.STEP_CONFIGS == bench.Step.OPS
+
+
+def test_cpu_baseline_report_on_a_small_step(monkeypatch):
+    """The CPU-baseline record: plain and row-parallel builds of the oracle,
+    per-configuration times, host core count and CPU model (run here on a
+    reduced step whose configurations are cut to a few rows)."""
+    class Tiny(bench.OracleStep):
+        def __init__(self):
+            from swiglu_ar_tts_b200 import inputs
+            f64 = lambda t: t.double().numpy()  # noqa: E731
+            self.rn = {k: f64(v) for k, v in inputs.rmsnorm_inputs(4, 64, "f32", 0).items()}
+            self.an = {k: f64(v) for k, v in inputs.add_rmsnorm_inputs(4, 64, "bf16", 0).items()}
+            self.sw = {k: f64(v) for k, v in inputs.swiglu_inputs(4, 64, "bf16", 0).items()}
+            mr = inputs.mrope_inputs(8)
+            self.pos = mr["pos"].numpy()
+            self.mr = {k: f64(v) for k, v in mr.items() if k != "pos"}
+            shape = ChainShape(batch=2, layers=2)
+            c = inputs.decode_chain_inputs(shape)
+            chain = (f64(c["residual"]), {k: [f64(t) for t in v] for k, v in c.items() if k != "residual"})
+            self.chains = {"decode_b5": chain, "decode_b256": chain}
+            self.bytes = {k: 1000 for k in bench.STEP_CONFIGS}
+            self.sample = "tiny"
+
+    rep = bench.cpu_baseline_report(Tiny())
+    assert rep["kind"] == "oracle" and rep["cores"] == 1 and rep["single"]["threads"] == 1
+    assert rep["omp"]["threads"] >= 1 and rep["nproc"] >= 1 and rep["cpu_model"]
+    assert set(rep["per_config_ms"]) == set(bench.STEP_CONFIGS)
+    assert set(rep["omp"]["per_config_ms"]) == set(bench.STEP_CONFIGS)
+    assert rep["value"] == rep["single"]["value"] > 0
 
 
 def _rank(rank, world, port, q):

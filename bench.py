@@ -10,14 +10,20 @@ synthetic input:
   * M-RoPE bf16, q [4096 x 16 x 128], k [4096 x 8 x 128], sections [24, 20, 20]
   * one 28-layer decode step (add+norm, M-RoPE, add+norm, SwiGLU per layer) at
     batch 5 and at batch 256, each replayed from a CUDA graph.
-``value`` is the step's algorithmic HBM bytes (every operand read once, every
-output written once) divided by its device time, in GB/s, summed over ranks.
-The JSON line also gives per-operator times and GB/s, microseconds per decode
-step, the time, share and GB/s of each kernel type (the decode graphs are split
-across their kernels by timing each operator's launches as a graph of its
-own), the roofline of the dominant kernel and of the largest single launch
-(SwiGLU), an end-to-end figure with host buffers, and the oracle timed on the
-host cores.
+The step is captured once as a CUDA graph of its 228 launches, each launched
+with programmatic dependent launch, and every timed step is one replay of it
+between two CUDA events.  ``value`` is the step's algorithmic HBM bytes (every
+operand read once, every output written once) divided by its device time, in
+GB/s, summed over ranks.  The JSON line also gives each operator alone
+(``ops_isolated``: median of 100 event-bracketed launches over inputs rotated
+through >= 512 MB, and the per-launch time back to back), the step time split
+among the operators in proportion to what each adds to the step graph's time
+(``ops``),
+microseconds per decode step, the time, share and GB/s of each kernel type
+(each decode step split across its kernels by timing each operator's launches
+as a graph of its own), the roofline of the dominant kernel and of the largest
+single launch (SwiGLU), an end-to-end figure with host buffers, and the oracle
+timed on the host cores.
 
 L2: the step touches ~1 GB of distinct data, 8x the 126 MB L2, and no operator
 reuses data of another, so every operator's inputs were last touched hundreds
@@ -49,11 +55,13 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from swiglu_ar_tts_b200.step import STEP_CONFIGS, Step, step_bytes  # noqa: E402
+
 METRIC = "fused-op HBM GB/s & % of B200 peak; µs per decode step (5 candidates)"
 UNIT = "GB/s"
 WORKLOAD = ("hot-path pass: RMSNorm f32 64x1024; add+RMSNorm bf16 4096x2048; SwiGLU bf16 "
             "8192x6144; M-RoPE bf16 4096 tok x (16q+8k) heads x 128, sections [24,20,20]; "
-            "28-layer decode step at batch 5 and at batch 256 (CUDA graph)")
+            "28-layer decode step at batch 5 and at batch 256; the whole pass one CUDA graph")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -174,183 +182,32 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml, 5 ms"}
 
 
-# ---------------------------------------------------------------------------
-# the step
-# ---------------------------------------------------------------------------
-class Step:
-    """Device buffers and launches of one hot-path step."""
+def step_marginals(step, reps: int = 20, rounds: int = 5) -> tuple[dict, float]:
+    """What each operator adds to the step, in µs: the step graph's time minus
+    the time of the same graph with that operator left out (each graph
+    replayed ``reps`` times back to back between two events, the median of
+    ``rounds`` interleaved rounds).  Returns ({op: µs}, µs of the whole step
+    measured the same way)."""
+    graphs = {None: step.graph}
+    for name in step.OPS:
+        graphs[name] = step.capture(without=name)
+    times = {k: [] for k in graphs}
+    for _ in range(rounds):
+        for k, g in graphs.items():
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times[k].append(1e3 * e0.elapsed_time(e1) / reps)
+    full = statistics.median(times[None])
+    marg = {name: full - statistics.median(times[name]) for name in step.OPS}
+    del graphs
+    return marg, full
 
-    OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode_b5", "decode_b256")
-
-    def __init__(self, device: torch.device, pdl: bool = True):
-        import swiglu_ar_tts_b200 as ops
-        from swiglu_ar_tts_b200 import inputs
-        from swiglu_ar_tts_b200.chain import DecodeChain
-
-        self.ops = ops
-        self.device = device
-        self.host = {
-            "rmsnorm": inputs.rmsnorm_inputs(64, 1024, "f32", 0),
-            "add_rmsnorm": inputs.add_rmsnorm_inputs(4096, 2048, "bf16", 0),
-            "swiglu": inputs.swiglu_inputs(8192, 6144, "bf16", 0),
-            "mrope_qk": inputs.mrope_inputs(4096),
-        }
-        d = device
-        h = self.host
-        self.rn = {k: v.to(d) for k, v in h["rmsnorm"].items()}
-        self.rn["y"] = torch.empty_like(self.rn["x"])
-        self.an = {k: v.to(d) for k, v in h["add_rmsnorm"].items()}
-        self.an["y"] = torch.empty_like(self.an["x"])
-        self.an["residual_out"] = torch.empty_like(self.an["residual"])
-        self.sw = {k: v.to(d) for k, v in h["swiglu"].items()}
-        self.sw["out"] = torch.empty_like(self.sw["gate"])
-        self.mr = {k: v.to(d) for k, v in h["mrope_qk"].items()}
-        self.mr["q_out"] = torch.empty_like(self.mr["q"])
-        self.mr["k_out"] = torch.empty_like(self.mr["k"])
-        self.chain5 = DecodeChain(inputs.ChainShape(batch=5), device=d, pdl=pdl)
-        self.chain256 = DecodeChain(inputs.ChainShape(batch=256), device=d, seed=1000, pdl=pdl)
-        self.chain5.capture()
-        self.chain256.capture()
-        self.decode_step_index = 0
-        self.bytes = step_bytes()
-        assert self.bytes["decode_b5"] == self.chain5.bytes_per_step()
-        assert self.bytes["decode_b256"] == self.chain256.bytes_per_step()
-        # rows (tokens) one launch of each operator processes
-        self.rows = {"rmsnorm": 64, "add_rmsnorm": 4096, "swiglu": 8192, "mrope_qk": 4096,
-                     "decode_b5": 5, "decode_b256": 256}
-        # kernels of this library launched per step (graph replays bypass the
-        # launch counter, so their kernels are counted from the capture)
-        self.kernels_per_step = 4 + self.chain5.launches_per_step + self.chain256.launches_per_step
-
-    def prepare_op(self, name: str) -> None:
-        """Host-side set-up that precedes an operator: the decode step's position
-        ids (a 24-byte fill, outside the operator's timed window)."""
-        if name == "decode_b5":
-            self.chain5.set_position(self.decode_step_index % 300)
-        elif name == "decode_b256":
-            self.chain256.set_position(self.decode_step_index % 300)
-
-    def run_op(self, name: str) -> None:
-        ops = self.ops
-        if name == "rmsnorm":
-            ops.rmsnorm(self.rn["x"], self.rn["gamma"], 1e-6, out=self.rn["y"])
-        elif name == "add_rmsnorm":
-            ops.add_rmsnorm(self.an["x"], self.an["residual"], self.an["gamma"], 1e-6,
-                            y=self.an["y"], residual_out=self.an["residual_out"])
-        elif name == "swiglu":
-            ops.swiglu(self.sw["gate"], self.sw["up"], out=self.sw["out"])
-        elif name == "mrope_qk":
-            ops.mrope_qk(self.mr["q"], self.mr["k"], self.mr["pos"], (24, 20, 20), 1e6,
-                         q_out=self.mr["q_out"], k_out=self.mr["k_out"])
-        elif name == "decode_b5":
-            self.chain5._graph.replay()
-        elif name == "decode_b256":
-            self.chain256._graph.replay()
-
-    def run(self, events=None) -> None:
-        """One step; ``events`` (2 per operator) bracket each operator.  The
-        step's set-up (the decode position ids) is enqueued before the first
-        event, so it falls outside every timed window and the step's time."""
-        for name in self.OPS:
-            self.prepare_op(name)
-        for i, name in enumerate(self.OPS):
-            if events is not None:
-                events[2 * i].record()
-            self.run_op(name)
-            if events is not None:
-                events[2 * i + 1].record()
-        self.decode_step_index += 1
-
-    # -- end to end: host buffers in, results back to the host ------------------
-    def setup_e2e(self) -> None:
-        pin = lambda t: t.detach().cpu().pin_memory()  # noqa: E731
-        self.h_in = {
-            "rn": {k: pin(v) for k, v in self.host["rmsnorm"].items()},
-            "an": {k: pin(v) for k, v in self.host["add_rmsnorm"].items()},
-            "sw": {k: pin(v) for k, v in self.host["swiglu"].items()},
-            "mr": {k: pin(v) for k, v in self.host["mrope_qk"].items()},
-            "c5": [pin(t) for t in self._chain_inputs(self.chain5)],
-            "c256": [pin(t) for t in self._chain_inputs(self.chain256)],
-        }
-        self.h_out = {
-            "rn": [pin(torch.empty_like(self.rn["y"], device="cpu"))],
-            "an": [pin(torch.empty_like(self.an["y"], device="cpu")),
-                   pin(torch.empty_like(self.an["residual_out"], device="cpu"))],
-            "sw": [pin(torch.empty_like(self.sw["out"], device="cpu"))],
-            "mr": [pin(torch.empty_like(self.mr["q_out"], device="cpu")),
-                   pin(torch.empty_like(self.mr["k_out"], device="cpu"))],
-            "c5": [pin(torch.empty_like(t, device="cpu")) for t in self._chain_outputs(self.chain5)],
-            "c256": [pin(torch.empty_like(t, device="cpu")) for t in self._chain_outputs(self.chain256)],
-        }
-        nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)  # noqa: E731
-        self.h2d_bytes = (sum(nbytes(v.values()) for k, v in self.h_in.items() if isinstance(v, dict))
-                          + nbytes(self.h_in["c5"]) + nbytes(self.h_in["c256"]))
-        self.d2h_bytes = sum(nbytes(v) for v in self.h_out.values())
-        self.s_h2d = torch.cuda.Stream(self.device)
-        self.s_d2h = torch.cuda.Stream(self.device)
-
-    @staticmethod
-    def _chain_inputs(c):
-        ts = [c.residual]
-        for k in ("x_attn", "gamma_attn", "q", "k", "x_mlp", "gamma_mlp", "gate", "up"):
-            ts += c.inp[k]
-        return ts
-
-    @staticmethod
-    def _chain_outputs(c):
-        return [c.residual] + c.y_attn + c.q_out + c.k_out + c.y_mlp + c.act
-
-    # operators with the most output first: their copies back overlap the
-    # later operators' copies in, and the pipeline ends on small copies
-    E2E_GROUPS = (("c256", "decode_b256"), ("sw", "swiglu"), ("an", "add_rmsnorm"),
-                  ("mr", "mrope_qk"), ("c5", "decode_b5"), ("rn", "rmsnorm"))
-
-    def _e2e_in(self, g: str) -> list:
-        """(device input, pinned host source) pairs of operator group ``g``."""
-        if g in ("c5", "c256"):
-            c = self.chain5 if g == "c5" else self.chain256
-            return list(zip(self._chain_inputs(c), self.h_in[g]))
-        dev = {"rn": self.rn, "an": self.an, "sw": self.sw, "mr": self.mr}[g]
-        return [(dev[k], v) for k, v in self.h_in[g].items()]
-
-    def _e2e_out(self, g: str) -> list:
-        """(pinned host destination, device output) pairs of operator group ``g``."""
-        dev = {"rn": [self.rn["y"]], "an": [self.an["y"], self.an["residual_out"]],
-               "sw": [self.sw["out"]], "mr": [self.mr["q_out"], self.mr["k_out"]]}
-        if g in ("c5", "c256"):
-            srcs = self._chain_outputs(self.chain5 if g == "c5" else self.chain256)
-        else:
-            srcs = dev[g]
-        return list(zip(self.h_out[g], srcs))
-
-    def run_e2e(self) -> None:
-        """Host->device copies of every input, the step, device->host copies of
-        every output.  Three streams form a pipeline over the operators: the
-        inputs of operator i+1 cross PCIe while operator i computes and the
-        results of operator i-1 cross back (the two copy directions run at the
-        same time).  Events order each operator's copy-in, compute and
-        copy-out; the step starts after the previous step's copy-outs."""
-        nb = dict(non_blocking=True)
-        cur = torch.cuda.current_stream()
-        h2d, d2h = self.s_h2d, self.s_d2h
-        h2d.wait_stream(cur)
-        for g, name in self.E2E_GROUPS:
-            with torch.cuda.stream(h2d):
-                for dst, src in self._e2e_in(g):
-                    dst.copy_(src, **nb)
-            arrived = torch.cuda.Event()
-            arrived.record(h2d)
-            cur.wait_event(arrived)
-            self.prepare_op(name)
-            self.run_op(name)
-            done = torch.cuda.Event()
-            done.record(cur)
-            d2h.wait_event(done)
-            with torch.cuda.stream(d2h):
-                for dst, src in self._e2e_out(g):
-                    dst.copy_(src, **nb)
-        cur.wait_stream(d2h)
-        self.decode_step_index += 1
 
 def reduce_max(x: float, pg=None, device=None) -> float:
     """Max of ``x`` over the ranks of process group ``pg`` (identity without one).
@@ -492,24 +349,6 @@ def isolated_ops(device, peak: float, peak_kind: str, launches: int = 100) -> di
 # ---------------------------------------------------------------------------
 # CPU oracle timings
 # ---------------------------------------------------------------------------
-STEP_CONFIGS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode_b5", "decode_b256")
-
-
-def step_bytes() -> dict:
-    """Algorithmic HBM bytes of each operator of the step (every operand read
-    once, every output written once)."""
-    per_row_layer = 2 * 4 * 2048 * 2 + 2 * (16 + 8) * 128 * 2 + 3 * 4 + 3 * 6144 * 2  # 81,932
-    gammas = 2 * 2048 * 2  # two norm weights per layer
-    return {
-        "rmsnorm": (2 * 64 * 1024 + 1024) * 4,
-        "add_rmsnorm": (4 * 4096 * 2048 + 2048) * 2,
-        "swiglu": 3 * 8192 * 6144 * 2,
-        "mrope_qk": 2 * 4096 * (16 + 8) * 128 * 2 + 3 * 4096 * 4,
-        "decode_b5": 28 * (5 * per_row_layer + gammas),
-        "decode_b256": 28 * (256 * per_row_layer + gammas),
-    }
-
-
 def cpu_model() -> str:
     try:
         with open("/proc/cpuinfo") as f:
@@ -681,14 +520,13 @@ def main() -> None:
 
     ops.lib()
     step = Step(device, pdl=not args.no_pdl)
+    step.capture()
 
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
 
-    n_ops = len(Step.OPS)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_ops)]
-              for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(device)
     sampler.start()
     launches0 = ops.launch_count()
@@ -706,29 +544,33 @@ def main() -> None:
     eager_launches = ops.launch_count() - launches0
     clocks = sampler.stop()
 
-    per_op_ms = np.zeros(n_ops)
-    step_ms = []
-    for ev in events:
-        durs = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n_ops)]
-        per_op_ms += np.array(durs)
-        step_ms.append(ev[0].elapsed_time(ev[2 * n_ops - 1]))
-    per_op_ms /= args.steps
+    step_ms = [ev[0].elapsed_time(ev[1]) for ev in events]
     total_ms = max_over_ranks(float(sum(step_ms)))
     ms_per_step = total_ms / args.steps
     step_bytes = sum(step.bytes[o] for o in Step.OPS)
     value = aggregate_value(world, step_bytes, args.steps, total_ms)
+    step_us = 1e3 * ms_per_step
 
+    # The step runs its operators back to back in one graph, so no event can sit
+    # between two of them without breaking programmatic dependent launch.  Its
+    # device time is split among them in proportion to what each adds to it
+    # (step_marginals, outside the timed steps); each operator is also timed
+    # alone (isolated_ops).
     peak, peak_kind = measured_hbm_peak()
+    marg, marg_full = step_marginals(step)
+    scale = step_us / sum(marg.values())
     ops_report = {}
-    for i, name in enumerate(Step.OPS):
-        us = 1e3 * per_op_ms[i]
+    for name in Step.OPS:
+        us = marg[name] * scale
         gbs = step.bytes[name] / (us * 1e-6) / 1e9
         ops_report[name] = {"us": round(us, 3), "bytes": step.bytes[name], "gbs": round(gbs, 1),
                             "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
                             "frac_of_spec_hbm": round(gbs / SPEC_HBM_GBS, 4),
-                            "rows_per_s": round(step.rows[name] / (us * 1e-6))}
-    # time per kernel type in the step: prefill operators are timed directly;
-    # each decode graph is split across its operators' kernels (decode_split)
+                            "rows_per_s": round(step.rows[name] / (us * 1e-6)),
+                            "us_marginal": round(marg[name], 3)}
+    iso = isolated_ops(device, peak, peak_kind)
+    # time per kernel type in the step: prefill operators are one launch each;
+    # each decode step is split across its operators' kernels (decode_split)
     kernels: dict[str, dict] = {}
 
     def add_time(kernel, us, launches, nbytes):
@@ -746,10 +588,11 @@ def main() -> None:
             decode_launch_us.setdefault(KERNEL_OF[op], {})[name] = round(
                 frac * ops_report[name]["us"] / launches, 3)
     step_us = 1e3 * ms_per_step
-    for k in kernels.values():
+    for kname, k in kernels.items():
         k["share"] = round(k["us"] / step_us, 4)
         k["gbs"] = round(k["bytes"] / (k["us"] * 1e-6) / 1e9, 1)
         k["us"] = round(k["us"], 2)
+        k["us_per_decode_launch"] = decode_launch_us.get(kname, {})
     dominant = max(kernels, key=lambda k: kernels[k]["us"])
     dk = kernels[dominant]
     # traffic: DRAM bytes per launch averaged over the step's launches of the
@@ -830,8 +673,6 @@ def main() -> None:
         run300[f"batch{batch}"] = {"graph_us_per_step": round(t["graph"], 2),
                                    "eager_us_per_step": round(t["eager"], 2)}
 
-    iso = isolated_ops(device, peak, peak_kind)
-
     # end to end: pinned host buffers in and out, through the same public calls
     step.setup_e2e()
     torch.cuda.synchronize()
@@ -880,6 +721,13 @@ def main() -> None:
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": None, "parallelism": f"replicas x{world}",
                    "pdl": not args.no_pdl,
+                   "timing": "each step is one replay of a CUDA graph of all 228 launches "
+                             "(4 prefill, 112 + 112 decode), CUDA events around the replay; "
+                             "ops[*].us = the step time split in proportion to what each "
+                             "operator adds to the step graph's time (us_marginal: the "
+                             "graph's time minus that of the graph without the operator)",
+                   "step_split_scale": round(scale, 4),
+                   "step_us_in_marginal_runs": round(marg_full, 2),
                    "l2": "inputs larger than L2: the step streams ~1 GB of distinct data "
                          "(8x L2) and no operator reuses another's data; no flush buffer"},
         "us_per_decode_step": {"batch5": ops_report["decode_b5"]["us"],
@@ -893,7 +741,7 @@ def main() -> None:
         "decode_300_steps": run300,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "gpu_launches": eager_launches + args.steps * (step.kernels_per_step - 4),
+        "gpu_launches": eager_launches + args.steps * step.kernels_per_step,
         "clocks": clocks,
         "wall_s_timed": wall,
     }

@@ -204,14 +204,27 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  *   1 <= top_k <= min(64, vocab), vocab <= 262144, rows <= 65535,
  *   temperature > 0 and finite.
  *   workspace  device scratch of at least arops_topk_sample_workspace() bytes
- *              (8-byte aligned, caller-owned; contents need no initialisation
- *              and are overwritten).  Two calls in flight at once must not
- *              share one workspace.
- * Two kernels are enqueued on `stream` (per-slice candidates, then the merge
- * and the decision).
+ *              (16-byte aligned, caller-owned).  It starts with 256 KiB of
+ *              per-row arrival counters that must be zero when a call begins:
+ *              clear them once after allocating the workspace, with
+ *              arops_topk_sample_prepare (or any zero fill of the first 256
+ *              KiB); every call leaves them zero again, for any later shape.
+ *              The rest holds candidates and needs no initialisation.  Two
+ *              calls in flight at once must not share one workspace.
+ * One kernel is enqueued on `stream`: each 4096-logit slice's CTA writes its
+ * top_k candidates, and the last CTA of a row to finish (counted on the row's
+ * arrival counter) merges them and takes the decision; no CTA waits for
+ * another.  A counter found non-zero at the start of a call (a workspace that
+ * was not cleared) sets AROPS_DEVICE_ERR_WORKSPACE in the device error word,
+ * and that row's outputs are then undefined.
  */
+#define AROPS_DEVICE_ERR_WORKSPACE 4u
 AROPS_API arops_status arops_topk_sample_workspace(int64_t rows, int64_t vocab, int32_t top_k,
                                                    size_t* bytes);
+/* Clears the arrival counters of a new workspace (a zero fill of its first
+ * 256 KiB enqueued on `stream`); workspace_bytes must cover them. */
+AROPS_API arops_status arops_topk_sample_prepare(void* workspace, size_t workspace_bytes,
+                                                 void* stream);
 AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel,
                                          int32_t* token_out, float* prob_out, int64_t rows,
                                          int64_t vocab, int32_t top_k, float temperature,
@@ -220,9 +233,11 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
 
 /*
  * arops_topk_sample without a workspace argument: the same computation and
- * results, with the scratch taken from a 1 MiB array that the library itself
- * holds in device memory (a file-scope __device__ array; every GPU that loads
- * the library keeps it until the process exits).  The paper has no
+ * results, with the scratch taken from an array that the library itself holds
+ * in device memory (a file-scope __device__ array of 1.25 MiB: 256 KiB of
+ * arrival counters, zero when the library's device code is loaded, then 1 MiB
+ * of candidates; every GPU that loads the library keeps it until the process
+ * exits).  The paper has no
  * counterpart: it is here for callers that cannot allocate device memory,
  * such as code running inside a host application's real-time audio or
  * streaming callback, where cudaMalloc is not allowed because it can block
@@ -245,11 +260,12 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
  *     allowed (a real-time callback) make one such call per context at set-up,
  *     outside that path and before any stream capture.  After it, calls
  *     allocate nothing and call no allocating routine.
- *   - All calls share the one array and it keeps the previous call's contents;
- *     no part of it needs to start at zero, since every slot a call reads is
- *     written earlier in that same call.  Calls whose kernels overlap on the
- *     GPU (different streams, different host threads) race on the array:
- *     serialise them, e.g. by issuing them on one stream.
+ *   - All calls share the one array and it keeps the previous call's contents:
+ *     the counters start at zero and every call leaves them zero, and every
+ *     candidate slot a call reads is written earlier in that same call.  Calls
+ *     whose kernels overlap on the GPU (different streams, different host
+ *     threads) race on the array: serialise them, e.g. by issuing them on one
+ *     stream.
  */
 AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float* gumbel,
                                                  int32_t* token_out, float* prob_out,
@@ -264,13 +280,16 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
  * Programmatic dependent launch.  The Triton kernel-fusion post for Qwen3-TTS
  * (section 3) reaches its end-to-end result by pairing its fused kernels with a
  * CUDA-graph decoder; this is the launch-level counterpart for chains of small
- * kernels.  When enabled
- * (process-wide, default off),
- * every kernel is launched with the programmatic-stream-serialisation attribute
- * so that it can be scheduled while the previous kernel on the stream drains;
- * each kernel waits for its predecessor's memory before touching global memory,
+ * kernels.  When enabled (process-wide, default off), every kernel is launched
+ * with the programmatic-stream-serialisation attribute so that it can be
+ * scheduled while the previous kernel on the stream drains; each kernel waits
+ * for its predecessor's memory before it reads activations or writes anything,
  * so results and stream-order semantics are unchanged.  It only shortens the
- * gaps between back-to-back launches (decode steps).  Returns the old setting.
+ * gaps between back-to-back launches (decode steps).
+ * Contract while enabled: the norms read their weights before that wait, so
+ * gamma and beta must not be written by the kernel launched immediately before
+ * on the same stream (kernels launched earlier have completed by then); model
+ * weights meet it.  Returns the old setting.
  */
 AROPS_API int arops_set_pdl(int enable);
 
@@ -292,7 +311,9 @@ AROPS_API int arops_set_streaming(int enable);
  * part of their work: AROPS_DEVICE_ERR_TIMEOUT means a bulk copy into shared
  * memory did not complete within a second (the kernel's outputs are then
  * undefined); AROPS_DEVICE_ERR_BAD_INDEX (see arops_mrope_kv_append) means a
- * token's cache slot was out of range and was not written.  The call
+ * token's cache slot was out of range and was not written;
+ * AROPS_DEVICE_ERR_WORKSPACE (see arops_topk_sample) means a sampling
+ * workspace's counters were not cleared.  The call
  * synchronises the device (it is a plain copy from device memory) and, if
  * `clear` is non-zero, resets the bits.  Healthy runs always read 0.
  */
@@ -321,7 +342,7 @@ AROPS_API const char* arops_last_error(void);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 AROPS_API int arops_version(void);
 
-#define AROPS_VERSION 10000
+#define AROPS_VERSION 20000
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "mrope_kv_append",
     "swiglu", "set_pdl",
-    "set_streaming", "topk_sample", "topk_sample_workspace",
+    "set_streaming", "topk_sample", "topk_sample_workspace", "topk_sample_prepare",
     "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
 ]
@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, fn).restype = ctypes.c_int
         L.arops_topk_sample_workspace.argtypes = [_i64, _i64, _i32, ctypes.POINTER(ctypes.c_size_t)]
         L.arops_topk_sample_workspace.restype = ctypes.c_int
+        L.arops_topk_sample_prepare.argtypes = [_vp, ctypes.c_size_t, _vp]
+        L.arops_topk_sample_prepare.restype = ctypes.c_int
         L.arops_topk_sample.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i32, ctypes.c_float,
                                         ctypes.c_int, _vp, ctypes.c_size_t, _vp]
         L.arops_topk_sample.restype = ctypes.c_int
@@ -302,6 +304,17 @@ def topk_sample_workspace(rows: int, vocab: int, top_k: int) -> int:
     return int(n.value)
 
 
+def topk_sample_prepare(workspace: torch.Tensor) -> torch.Tensor:
+    """Clears the arrival counters of a new sampling workspace (a uint8 device
+    tensor) on the current stream; needed once, before its first use."""
+    _check_tensors((("workspace", workspace),))
+    with torch.cuda.device(workspace.device):
+        _check(lib().arops_topk_sample_prepare(workspace.data_ptr(),
+                                               workspace.numel() * workspace.element_size(),
+                                               _stream(workspace)))
+    return workspace
+
+
 def topk_sample(logits: torch.Tensor, gumbel: torch.Tensor, top_k: int, temperature: float = 1.0,
                 workspace: torch.Tensor | None = None, token_out: torch.Tensor | None = None,
                 prob_out: torch.Tensor | None = None):
@@ -309,8 +322,9 @@ def topk_sample(logits: torch.Tensor, gumbel: torch.Tensor, top_k: int, temperat
     top_k logits of each row.  logits [rows, vocab] (bf16/f32); gumbel
     [rows, top_k] float32 Gumbel(0,1) draws, draw j for the j-th largest logit.
     Returns (token int32 [rows], probability float32 [rows]).  ``workspace`` is
-    a uint8 device tensor of at least topk_sample_workspace() bytes (allocated
-    here if omitted)."""
+    a uint8 device tensor of at least topk_sample_workspace() bytes whose
+    counters were cleared once (topk_sample_prepare); allocated and cleared
+    here if omitted."""
     if logits.dim() != 2:
         raise ValueError("logits must be [rows, vocab]")
     rows, vocab = logits.shape
@@ -320,7 +334,9 @@ def topk_sample(logits: torch.Tensor, gumbel: torch.Tensor, top_k: int, temperat
         prob_out = torch.empty(rows, dtype=torch.float32, device=logits.device)
     need = topk_sample_workspace(rows, vocab, top_k) if rows else 0
     if workspace is None:
-        workspace = torch.empty(max(need, 8), dtype=torch.uint8, device=logits.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=logits.device)
+        if rows:
+            topk_sample_prepare(workspace)
     _check_tensors((("logits", logits), ("gumbel", gumbel), ("token_out", token_out),
                     ("prob_out", prob_out), ("workspace", workspace)))
     if gumbel.dtype != torch.float32 or tuple(gumbel.shape) != (rows, top_k):
@@ -350,7 +366,8 @@ def set_streaming(enable: bool) -> bool:
 
 def device_errors(clear: bool = True) -> int:
     """Device-side error bits (1: a bulk-copy wait timed out; 2: a KV-cache slot
-    out of range was skipped); synchronises the device."""
+    out of range was skipped; 4: a sampling workspace's counters were not
+    cleared); synchronises the device."""
     v = ctypes.c_uint32(0)
     _check(lib().arops_device_errors(ctypes.byref(v), 1 if clear else 0))
     return int(v.value)

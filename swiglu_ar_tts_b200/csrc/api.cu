@@ -317,8 +317,23 @@ AROPS_API arops_status arops_topk_sample_workspace(int64_t rows, int64_t vocab, 
     const arops_status st = topk_check("arops_topk_sample_workspace", rows, vocab, top_k, 1.0f);
     if (st != AROPS_OK)
         return st;
-    *bytes = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * sizeof(uint64_t);
+    *bytes = topk_counter_bytes() +
+             (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * sizeof(uint64_t);
     return ok();
+}
+
+AROPS_API arops_status arops_topk_sample_prepare(void* workspace, size_t workspace_bytes,
+                                                 void* stream)
+{
+    if (!workspace)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample_prepare: workspace is null");
+    if (workspace_bytes < topk_counter_bytes())
+        return fail(AROPS_ERR_INVALID,
+                    "arops_topk_sample_prepare: workspace of %zu bytes < the %zu bytes of counters",
+                    workspace_bytes, topk_counter_bytes());
+    return from_cuda(cudaMemsetAsync(workspace, 0, topk_counter_bytes(),
+                                     static_cast<cudaStream_t>(stream)),
+                     "arops_topk_sample_prepare");
 }
 
 AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel,
@@ -336,14 +351,15 @@ AROPS_API arops_status arops_topk_sample(const void* logits, const float* gumbel
         return ok();
     if (!logits || !gumbel || !token_out || !prob_out || !workspace)
         return fail(AROPS_ERR_INVALID, "arops_topk_sample: null pointer");
-    const size_t need = (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * 8u;
+    const size_t need =
+        topk_counter_bytes() + (size_t)rows * (size_t)topk_slices(vocab) * (size_t)top_k * 8u;
     if (workspace_bytes < need)
         return fail(AROPS_ERR_INVALID, "arops_topk_sample: workspace of %zu bytes < %zu needed",
                     workspace_bytes, need);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 7u) != 0)
-        return fail(AROPS_ERR_INVALID, "arops_topk_sample: workspace not 8-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+        return fail(AROPS_ERR_INVALID, "arops_topk_sample: workspace not 16-byte aligned");
     return from_cuda(launch_topk_sample(logits, gumbel, token_out, prob_out, rows, vocab, top_k,
-                                        temperature, dtype, static_cast<uint64_t*>(workspace),
+                                        temperature, dtype, workspace,
                                         static_cast<cudaStream_t>(stream)),
                      "arops_topk_sample");
 }
@@ -369,7 +385,7 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
                     need, topk_noalloc_scratch_bytes());
     // resolved before the rows == 0 return, so that a call with no rows is the
     // set-up call: it makes the current context load this code and its array
-    uint64_t* scratch = nullptr;
+    void* scratch = nullptr;
     cudaError_t err = topk_noalloc_scratch(&scratch);
     if (err != cudaSuccess)
         return from_cuda(err, "arops_topk_sample_noalloc (scratch address)");

@@ -44,6 +44,13 @@ __device__ __forceinline__ void prefetch_l2_line(const void* p)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// ORs `bits` into the library's device error word (a file-scope __device__
+// variable whose address kernels receive as a parameter; device_error_word()).
+__device__ __forceinline__ void record_device_error(unsigned* word, unsigned bits)
+{
+    atomicOr(word, bits);
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte vectors of the storage type, unpacked to / packed from fp32.
 // ---------------------------------------------------------------------------
@@ -143,8 +150,8 @@ struct DeviceInfo {
 // SM count of the current device (queried once per device).
 cudaError_t current_device_info(DeviceInfo* info);
 
-// Device address of the library's error word on the current device (resolved
-// once per device with cudaGetSymbolAddress).
+// Device address of the library's error word in the current context (looked
+// up with cudaGetSymbolAddress on every call).
 cudaError_t device_error_word(unsigned** word);
 
 // Whether kernels are launched with the PDL attribute.
@@ -256,21 +263,24 @@ struct AppendArgs {
 cudaError_t launch_mrope_append(const MropeArgs& a, const AppendArgs& x, arops_dtype dtype,
                                 cudaStream_t stream);
 
-// Fused softmax + top-k sampling (topk.cu).
+// Fused softmax + top-k sampling (topk.cu).  The workspace starts with
+// topk_counter_bytes() of per-row arrival counters (zero between calls), then
+// rows x slices x k candidate keys of 8 bytes.
 int topk_slices(int64_t vocab);
 int topk_max_k();
 int topk_max_slices();
+size_t topk_counter_bytes();
 cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
                                float* prob_out, int64_t rows, int64_t vocab, int k,
-                               float temperature, arops_dtype dtype, uint64_t* work,
+                               float temperature, arops_dtype dtype, void* workspace,
                                cudaStream_t stream);
 // Self-test of the bounded mbarrier wait (selftest.cu).
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, int* waited_out,
                                          cudaStream_t stream);
 
-// The allocation-free variant's built-in scratch array: its size, and its
-// device address on the current device.
+// The allocation-free variant's built-in scratch array: the candidate bytes it
+// holds (after its counters), and its device address in the current context.
 size_t topk_noalloc_scratch_bytes();
-cudaError_t topk_noalloc_scratch(uint64_t** ptr);
+cudaError_t topk_noalloc_scratch(void** ptr);
 
 }  // namespace arops

@@ -66,11 +66,41 @@ __device__ __forceinline__ int32_t position_of(int j, const MropeParams& prm, in
     return (j < prm.sec0) ? pt : ((j < prm.sec01) ? ph : pw);
 }
 
+// cos/sin of the angles a lane applies, for token t: the lanes of pair block
+// pv split the block's E angles between them (F each) and share them with
+// shuffles, so every lane of the warp must take part.
+template <int E, int P>
+__device__ __forceinline__ void token_angles(const int32_t* __restrict__ pos, int64_t tokens,
+                                             int64_t t, const double* inv_freq,
+                                             const MropeParams& prm, int lane, float* c, float* s)
+{
+    constexpr int G = 32 / P;                // heads per warp pass
+    constexpr int F = (E >= G) ? E / G : 1;  // angles evaluated per lane
+    const int pv = lane % P;
+    const int hg = lane / P;
+    const int j0 = pv * E;
+    const int32_t pt = __ldg(pos + t);
+    const int32_t ph = __ldg(pos + tokens + t);
+    const int32_t pw = __ldg(pos + 2 * tokens + t);
+    float cs[F], sn[F];
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        const int j = j0 + ((hg * F + f) % E);
+        rope_cos_sin(inv_freq[j], position_of(j, prm, pt, ph, pw), &cs[f], &sn[f]);
+    }
+#pragma unroll
+    for (int m = 0; m < E; ++m) {
+        const int src = pv + P * ((m / F) % G);
+        c[m] = __shfl_sync(0xFFFFFFFFu, cs[m % F], src);
+        s[m] = __shfl_sync(0xFFFFFFFFu, sn[m % F], src);
+    }
+}
+
 constexpr int kWarpsPerCta = 4;
 
 // Token of warp unit `unit` and which of the token's `splits` warps it is.
-// splits > 1 only for launches of at most one head pass per resident warp, so
-// the unit index fits 32 bits there and the division stays a 32-bit one.
+// The launchers take splits > 1 only when tokens * splits < 2^32, so the unit
+// index fits 32 bits there and the division stays a 32-bit one.
 __device__ __forceinline__ int64_t unit_token(int64_t unit, int splits, int& part)
 {
     if (splits == 1) {
@@ -91,7 +121,6 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
     constexpr int G = 32 / P;                // heads per warp pass
     constexpr int HALF = P * E;              // head_dim / 2
     constexpr int D = 2 * HALF;
-    constexpr int F = (E >= G) ? E / G : 1;  // angles evaluated per lane
     // evict-first stores, except with one pass per warp (U == 1: decode-size launches)
     constexpr bool kStream = U > 1;
     const int lane = threadIdx.x & 31;
@@ -126,9 +155,6 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
         int part = 0;
         const int64_t t = unit_token(unit, splits, part);
         const int h_first = hg + part * G * U;
-        const int32_t pt = __ldg(pos + t);
-        const int32_t ph = __ldg(pos + tokens + t);
-        const int32_t pw = __ldg(pos + 2 * tokens + t);
 
         // the first batch of heads is loaded before the angles are evaluated, so
         // the q/k loads and the position loads share one memory latency
@@ -146,22 +172,8 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
             }
         };
         load_batch(h_first);
-
-        // this lane's share of the E angles of block pv ...
-        float cs[F], sn[F];
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-            const int j = j0 + ((hg * F + f) % E);
-            rope_cos_sin(inv_freq[j], position_of(j, prm, pt, ph, pw), &cs[f], &sn[f]);
-        }
-        // ... gathered from the lanes that evaluated them
         float c[E], s[E];
-#pragma unroll
-        for (int m = 0; m < E; ++m) {
-            const int src = pv + P * ((m / F) % G);
-            c[m] = __shfl_sync(0xFFFFFFFFu, cs[m % F], src);
-            s[m] = __shfl_sync(0xFFFFFFFFu, sn[m % F], src);
-        }
+        token_angles<E, P>(pos, tokens, t, inv_freq, prm, lane, c, s);
 
         for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
             if (h0 != h_first)
@@ -377,8 +389,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     constexpr int G = 32 / P;
     constexpr int HALF = P * E;
     constexpr int D = 2 * HALF;
-    constexpr int F = (E >= G) ? E / G : 1;
-    constexpr bool kStream = U > 1;  // one pass per warp: decode-size launches
+    // evict-first stores, except with one pass per warp (U == 1: decode-size launches)
+    constexpr bool kStream = U > 1;
     const int lane = threadIdx.x & 31;
     const int pv = lane % P;
     const int hg = lane / P;
@@ -413,9 +425,6 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
         int part = 0;
         const int64_t t = unit_token(unit, splits, part);
         const int h_first = hg + part * G * U;
-        const int32_t pt = __ldg(pos + t);
-        const int32_t ph = __ldg(pos + tokens + t);
-        const int32_t pw = __ldg(pos + 2 * tokens + t);
         int64_t cb = -1, cs = -1;
         if (hk > 0) {
             cb = __ldg(ca.loc + t);
@@ -445,20 +454,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
             }
         };
         load_batch(h_first);
-
-        float cs_[F], sn_[F];
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-            const int j = j0 + ((hg * F + f) % E);
-            rope_cos_sin(inv_freq[j], position_of(j, prm, pt, ph, pw), &cs_[f], &sn_[f]);
-        }
         float c[E], s[E];
-#pragma unroll
-        for (int m = 0; m < E; ++m) {
-            const int src = pv + P * ((m / F) % G);
-            c[m] = __shfl_sync(0xFFFFFFFFu, cs_[m % F], src);
-            s[m] = __shfl_sync(0xFFFFFFFFu, sn_[m % F], src);
-        }
+        token_angles<E, P>(pos, tokens, t, inv_freq, prm, lane, c, s);
 
         for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
             if (h0 != h_first)
@@ -572,8 +569,18 @@ inline bool one_pass_per_warp(int64_t tokens, int passes, int64_t cap)
     return tokens * passes <= cap;
 }
 
-// Otherwise heads per lane per pass: just enough passes to cover every head at
-// once (6 for 16 + 8 heads of 128), so no registers are held for absent heads.
+// Whether a token's passes may be shared by two warps (the unit index must
+// fit 32 bits, see unit_token).
+inline bool two_warps_per_token(int64_t tokens)
+{
+    return tokens * 2 <= (int64_t)UINT32_MAX;
+}
+
+// Otherwise a token with more than two passes is shared by two warps, each
+// loading its half of the passes at once (U = heads per lane in flight), so no
+// registers are held for absent heads and the grid has more, lighter warps:
+// 4096 tokens of 16 + 8 heads of 128 measured 9.15 us a launch back to back
+// on B200 with two warps of 3 passes, against 9.7 us with one warp of 6.
 template <typename T, int P>
 cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
 {
@@ -583,10 +590,13 @@ cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t 
         return launch_vec_u<T, P, 1>(a, prm, st, cap, passes);
     if (passes <= 2)
         return launch_vec_u<T, P, 2>(a, prm, st, cap);
-    if (passes <= 4)
-        return launch_vec_u<T, P, 4>(a, prm, st, cap);
-    if (passes <= 6)
-        return launch_vec_u<T, P, 6>(a, prm, st, cap);
+    if (two_warps_per_token(a.tokens) && passes <= 8) {
+        if (passes <= 4)
+            return launch_vec_u<T, P, 2>(a, prm, st, cap, 2);
+        if (passes <= 6)
+            return launch_vec_u<T, P, 3>(a, prm, st, cap, 2);
+        return launch_vec_u<T, P, 4>(a, prm, st, cap, 2);
+    }
     return launch_vec_u<T, P, kHeadUnroll>(a, prm, st, cap);
 }
 
@@ -696,10 +706,13 @@ cudaError_t launch_append_p(const MropeArgs& a, const AppendArgs& x, const Mrope
         return launch_append_u<T, P, 1>(a, x, prm, ca, word, st, cap, passes);
     if (passes <= 2)
         return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap);
-    if (passes <= 4)
-        return launch_append_u<T, P, 4>(a, x, prm, ca, word, st, cap);
-    if (passes <= 6)
-        return launch_append_u<T, P, 6>(a, x, prm, ca, word, st, cap);
+    if (two_warps_per_token(a.tokens) && passes <= 8) {  // as in launch_vec
+        if (passes <= 4)
+            return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap, 2);
+        if (passes <= 6)
+            return launch_append_u<T, P, 3>(a, x, prm, ca, word, st, cap, 2);
+        return launch_append_u<T, P, 4>(a, x, prm, ca, word, st, cap, 2);
+    }
     return launch_append_u<T, P, kHeadUnroll>(a, x, prm, ca, word, st, cap);
 }
 

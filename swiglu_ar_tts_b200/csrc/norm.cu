@@ -13,13 +13,14 @@
 // coalesced 128-bit accesses.  The sum of squares is accumulated in fp32,
 // reduced with warp shuffles and, for GW > 1 warps per row, one shared-memory
 // step; rsqrtf of (sum * 1/hidden + eps) scales the row and x * r * gamma is
-// rounded once to the storage type.  gamma is read through the read-only path
-// together with each row, so a row costs one memory round trip.  A problem of
-// at most one vector per resident thread (a decode step's few rows) takes one
-// vector per lane with the row spread over GW = hidden/256 warps; larger ones
-// take 8 vectors per lane, one warp per row up to 2048 bf16 elements.  The
-// streaming kernel (opt-in, arops_set_streaming) stages rows through shared
-// memory with bulk copies instead; it measured slower on B200.
+// rounded once to the storage type.  gamma (and beta) is read through the
+// read-only path once per thread, before the dependency wait, so a row costs
+// one memory round trip.  A problem of at most one vector per resident thread
+// (a decode step's few rows) takes one vector per lane with the row spread
+// over GW = hidden/256 warps; larger ones take 4 or 8 vectors per lane, one or
+// two warps per row up to 2048 bf16 elements.  The streaming kernel (opt-in,
+// arops_set_streaming) stages rows through shared memory with bulk copies
+// instead; it measured slower on B200.
 //
 // Rows longer than 4096 vectors, and unaligned or ragged rows, take a looped
 // kernel that makes a second pass over the row (served from L2).
@@ -228,7 +229,22 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
     __shared__ float red[2][GW];
     __shared__ float shift;
 
-    // this group's first row and the weights into L2 while the previous kernel drains
+    // The weights a thread applies are the same for every row it handles, so
+    // they are loaded once, into registers, before the dependency wait: with
+    // programmatic dependent launch the caller guarantees that gamma and beta
+    // are not written by the kernel launched just before this one (every
+    // earlier kernel has completed by the time this one starts).  This
+    // group's first row goes into L2 while the previous kernel drains.
+    uint4 gv[VPL], bv[LN ? VPL : 1];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int vi = gt + i * G;
+        if (vi < nvec) {
+            gv[i] = __ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E));
+            if constexpr (LN)
+                bv[i] = __ldg(reinterpret_cast<const uint4*>(beta + (size_t)vi * E));
+        }
+    }
     {
         const int64_t row0 = (int64_t)blockIdx.x * ROWS_PER_CTA + group;
         const uint32_t row_bytes = (uint32_t)hidden * sizeof(T);
@@ -236,11 +252,6 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
             prefetch_l2(x + (size_t)row0 * hidden, row_bytes);
             if constexpr (ADD)
                 prefetch_l2(residual_in + (size_t)row0 * hidden, row_bytes);
-        }
-        if (tid == 0 && blockIdx.x < 64) {  // later CTAs find them in L2 already
-            prefetch_l2(gamma, row_bytes);
-            if constexpr (LN)
-                prefetch_l2(beta, row_bytes);
         }
     }
     pdl_wait();
@@ -250,18 +261,7 @@ norm_rows_kernel(const T* x, const T* residual_in, T* residual_out, const T* __r
     for (int64_t row = (int64_t)blockIdx.x * ROWS_PER_CTA + group; row < rows;
          row += (int64_t)gridDim.x * ROWS_PER_CTA) {
         const size_t base = (size_t)row * (size_t)hidden;
-        uint4 v[VPL], gv[VPL], bv[LN ? VPL : 1];
-        // the weights are loaded with the row, not after the reduction: a load
-        // issued after the shuffles would add a dependent round trip to every row
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int vi = gt + i * G;
-            if (vi < nvec) {
-                gv[i] = __ldg(reinterpret_cast<const uint4*>(gamma + (size_t)vi * E));
-                if constexpr (LN)
-                    bv[i] = __ldg(reinterpret_cast<const uint4*>(beta + (size_t)vi * E));
-            }
-        }
+        uint4 v[VPL];
         float s1 = 0.f;  // sum of x^2 (RMSNorm) or of x (LayerNorm)
         if constexpr (ADD) {
             uint4 r[VPL];
@@ -559,6 +559,16 @@ cudaError_t launch_rows_wide(const T* x, const T* ri, T* ro, const T* g, const T
                   st, x, ri, ro, g, b, y, rows, hidden, eps, 1.0f / (float)hidden);
 }
 
+// VPL vectors per lane, GW warps per row, one row per CTA.
+template <typename T, bool ADD, bool LN, int VPL, int GW>
+cudaError_t launch_rows_vpl(const T* x, const T* ri, T* ro, const T* g, const T* b, T* y,
+                            int64_t rows, int hidden, float eps, cudaStream_t st, int64_t cap)
+{
+    const int64_t grid = std::min<int64_t>(rows, cap);
+    return launch(norm_rows_kernel<T, ADD, LN, VPL, GW>, dim3((unsigned)grid), dim3(32 * GW), 0,
+                  st, x, ri, ro, g, b, y, rows, hidden, eps, 1.0f / (float)hidden);
+}
+
 template <typename T, bool ADD, bool LN, int GW>
 cudaError_t launch_rows_gwn(const T* x, const T* ri, T* ro, const T* g, const T* b, T* y,
                             int64_t rows, int hidden, float eps, cudaStream_t st, int64_t cap)
@@ -603,6 +613,20 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
         // few rows) is latency-bound: after the dependency wait each warp then
         // has one load, a few flops and one store per tensor, and the row's
         // reduction runs across warps, instead of one warp walking the whole row.
+        // Once every SM has a row of its own (256 decode rows), two vectors per
+        // lane over half as many warps measured faster in chains of dependent
+        // launches on B200 (1.78 against 1.85 us a launch for 256 x 2048), and
+        // slower below that (1.43 against 1.36 us for 5 x 2048).
+        if (rows * nvec <= (int64_t)di.sm_count * 2048 && rows >= di.sm_count && nvec > 64 &&
+            nvec <= 1024) {
+            if (nvec <= 128)
+                return launch_rows_vpl<T, ADD, LN, 2, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            if (nvec <= 256)
+                return launch_rows_vpl<T, ADD, LN, 2, 4>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            if (nvec <= 512)
+                return launch_rows_vpl<T, ADD, LN, 2, 8>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            return launch_rows_vpl<T, ADD, LN, 2, 16>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+        }
         if (rows * nvec <= (int64_t)di.sm_count * 2048 && nvec > 32) {
             if (nvec <= 64)
                 return launch_rows_wide<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
@@ -619,8 +643,11 @@ cudaError_t launch_norm_t(const void* xv, const void* riv, void* rov, const void
             return launch_rows_gw1<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 128)
             return launch_rows_gw1<T, ADD, LN, 4>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+        // two warps of 4 vectors per lane (80 registers) rather than one warp of
+        // 8 (160): 4096 x 2048 bf16 add+RMSNorm measured 11.25 against 11.5 us
+        // a launch back to back on B200, with bit-identical residuals
         if (nvec <= 256)
-            return launch_rows_gw1<T, ADD, LN, 8>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
+            return launch_rows_vpl<T, ADD, LN, 4, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 512)
             return launch_rows_gwn<T, ADD, LN, 2>(x, ri, ro, g, b, y, rows, h, eps, st, cap);
         if (nvec <= 1024)

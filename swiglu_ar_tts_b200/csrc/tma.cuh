@@ -86,9 +86,4 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     return true;
 }
 
-__device__ __forceinline__ void record_device_error(unsigned* word, unsigned bits)
-{
-    atomicOr(word, bits);
-}
-
 }  // namespace arops

@@ -8,22 +8,22 @@
 // rank): Gumbel-max sampling from softmax(logits / T) restricted to the top k.
 // prob_out is that token's probability under the same restricted softmax.
 //
-// Two kernels:
-//   topk_slice_kernel   grid (slices, rows): a CTA turns its 4096-logit slice
-//                       into keys (order-preserving bits of the value, then the
-//                       inverted position, so that larger keys are larger logits
-//                       and, among equal logits, lower indices: every key is
-//                       distinct; 32 bits for bf16, 48 for fp32), finds its k
-//                       largest with a block-wide select in registers and
-//                       shared memory (select_top_k below), and writes them to
-//                       the workspace as (value bits, inverted 24-bit
-//                       vocabulary index) keys.
-//   topk_sample_kernel  grid (rows): selects the row's k largest among the
-//                       slices' candidates the same way, ranks those k by
-//                       counting, then takes the sampling decision and the
-//                       probability for its row.
-// The workspace holds rows x slices x k keys; every slot is written before it
-// is read, so it needs no clearing.
+// One kernel, grid (slices, rows).  A CTA turns its 4096-logit slice into
+// keys (order-preserving bits of the value, then the inverted position, so
+// that larger keys are larger logits and, among equal logits, lower indices:
+// every key is distinct; 32 bits for bf16, 48 for fp32), finds its k largest
+// with a block-wide select in registers and shared memory (select_top_k
+// below), and writes them to the workspace as (value bits, inverted 24-bit
+// vocabulary index) keys.  It then arrives on its row's counter; the CTA that
+// arrives last (it sees slices - 1 earlier arrivals) resets the counter to 0,
+// selects the row's k largest among the slices' candidates the same way, ranks
+// those k by counting, and takes the sampling decision and the probability.
+// No CTA waits for another: the others simply exit.
+//
+// Workspace: a fixed region of per-row arrival counters (kCounterBytes; they
+// must be zero before a workspace's first call and every call leaves the ones
+// it used at zero), then rows x slices x k candidate keys, every one written
+// before it is read.
 #include <math.h>
 
 #include <type_traits>
@@ -37,7 +37,13 @@ constexpr int kSlice = 4096;        // logits per slice
 constexpr int kSliceThreads = 512;  // 8 logits per thread
 constexpr int kMaxTopK = 64;
 constexpr int kMaxSlices = 64;  // merged candidates: kMaxSlices * kMaxTopK = 4096 keys
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = kSliceThreads;  // the last slice CTA of a row merges
+constexpr int kMaxRows = 65535;                 // grid y
+// Arrival counters at the start of the workspace, one per row up to kMaxRows
+// (so every shape finds them at the same place), padded to 256 KiB.
+constexpr size_t kCounterBytes = size_t(1) << 18;
+static_assert(kCounterBytes >= sizeof(unsigned) * kMaxRows, "a counter per row");
+constexpr unsigned kDeviceErrWorkspace = 4u;  // a counter was not zero when a call began
 
 // IEEE float bits, reordered so that unsigned comparison follows the value.
 __device__ __forceinline__ uint32_t order_bits(float v)
@@ -308,6 +314,93 @@ struct LocalKey {
     static constexpr int BITS = KeyBits<T>::V + 16;
 };
 
+constexpr int kMergePerThread = kMaxSlices * kMaxTopK / kMergeThreads;  // 8
+
+// The row's merge and decision, run by the CTA that arrived last: the k
+// largest of the slices' n = slices * k candidate keys (read through L2: other
+// CTAs wrote them), ranked by counting, then the sampling decision.
+template <typename T>
+__device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float* __restrict__ g,
+                                 float temperature, int32_t* token_out, float* prob_out,
+                                 SelectState& st, uint64_t* sel, uint64_t* ranked)
+{
+    uint64_t key[kMergePerThread];
+    bool valid[kMergePerThread];
+#pragma unroll
+    for (int m = 0; m < kMergePerThread; ++m) {
+        const int i = threadIdx.x + m * kMergeThreads;
+        // padding keys (0) of short slices are not candidates
+        key[m] = (i < n) ? __ldcg(cand + i) : 0ull;
+        valid[m] = key[m] != 0ull;
+    }
+    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
+#pragma unroll
+    for (int m = 0; m < kMergePerThread; ++m)
+        if (valid[m] && selected(key[m], st)) {
+            const int slot = atomicAdd(&st.count, 1);
+            if (slot < k)
+                sel[slot] = key[m];
+        }
+    __syncthreads();
+    // order the k candidates by counting: rank = number of larger keys
+    if ((int)threadIdx.x < k) {
+        const uint64_t mine = sel[threadIdx.x];
+        int rank = 0;
+        for (int j = 0; j < k; ++j)
+            rank += sel[j] > mine;
+        ranked[rank] = mine;
+    }
+    __syncthreads();
+
+    // Warp 0 takes the decision, two ranks per lane (k <= 64).  Per rank j:
+    // e_j = exp((l_j - l_0) / T) and the score fl(fl(l_j / T) + g_j), two
+    // correctly rounded operations.  The token is the first rank with the
+    // largest score, as a scan in rank order that moves on only to a strictly
+    // larger score finds it: NaN scores after rank 0 never win, a NaN at rank 0
+    // always does.
+    if (threadIdx.x >= 32)
+        return;
+    const int lane = threadIdx.x;
+    const float l0 = cand_value<T>(ranked[0]);
+    float ej[2], bs = 0.f, z = 0.f;
+    int bj = k;  // none yet
+    float s0 = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = lane + 32 * r;
+        ej[r] = 0.f;
+        if (j < k) {
+            const float l = cand_value<T>(ranked[j]);
+            ej[r] = expf((l - l0) / temperature);
+            const float sc = __fadd_rn(__fdiv_rn(l, temperature), g[j]);
+            if (j == 0)
+                s0 = sc;
+            if (!isnan(sc) && (bj == k || sc > bs)) {
+                bs = sc;
+                bj = j;
+            }
+            z += ej[r];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
+        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, o);
+        if (oj < k && (bj == k || os > bs || (os == bs && oj < bj))) {
+            bs = os;
+            bj = oj;
+        }
+        z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    }
+    s0 = __shfl_sync(0xFFFFFFFFu, s0, 0);
+    const int best = isnan(s0) ? 0 : bj;
+    const float eb = __shfl_sync(0xFFFFFFFFu, best < 32 ? ej[0] : ej[1], best & 31);
+    if (lane == 0) {
+        *token_out = (int32_t)cand_index(ranked[best]);
+        *prob_out = eb / z;
+    }
+}
+
 // VEC: rows start on 16-byte boundaries, so a thread loads its 16 logits as
 // 16-byte vectors (positions (v * 256 + thread) * E + e); otherwise one
 // element at a time (positions thread + 256 m).  Either way every position of
@@ -317,12 +410,18 @@ struct LocalKey {
 // against 256 for 5 x 151936 on B200).
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kSliceThreads, 2)
-topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices,
-                  uint64_t* __restrict__ work)
+topk_sample_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices,
+                   unsigned* __restrict__ counters, uint64_t* __restrict__ work,
+                   const float* __restrict__ gumbel, float temperature,
+                   int32_t* __restrict__ token_out, float* __restrict__ prob_out,
+                   unsigned* err_word)
 {
     using K = typename LocalKey<T>::type;
     constexpr int E = Vec<T>::N;
     __shared__ SelectState st;
+    __shared__ uint64_t sel[kMaxTopK];
+    __shared__ uint64_t ranked[kMaxTopK];
+    __shared__ int last;
     const int64_t row = blockIdx.y;
     const int64_t first = (int64_t)blockIdx.x * kSlice;
     const T* lr = logits + row * vocab;
@@ -370,7 +469,8 @@ topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices
         key[m] = valid[m] ? (((K)KeyBits<T>::of(val[m]) << 16) | (K)(0xFFFFu - (uint32_t)pos[m]))
                           : K(0);
     }
-    uint64_t* out = work + (row * slices + blockIdx.x) * (int64_t)k;
+    uint64_t* row_cand = work + row * slices * (int64_t)k;
+    uint64_t* out = row_cand + blockIdx.x * (int64_t)k;
     if (n <= k) {
         // the whole slice is a candidate; the unused slots get keys below any logit
 #pragma unroll
@@ -378,108 +478,36 @@ topk_slice_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slices
             if (pos[m] < k)
                 out[pos[m]] = valid[m] ? cand_key<T>(val[m], first + pos[m]) : 0ull;
         }
-        return;
-    }
-    select_top_k<LocalKey<T>::BITS>(key, valid, k, st);
+    } else {
+        select_top_k<LocalKey<T>::BITS>(key, valid, k, st);
 #pragma unroll
-    for (int m = 0; m < kPerThread; ++m)
-        if (valid[m] && selected(key[m], st)) {
-            const int slot = atomicAdd(&st.count, 1);
-            if (slot < k)  // exactly k are selected; the test only guards the bound
-                out[slot] = cand_key<T>(val[m], first + pos[m]);
-        }
-}
-
-constexpr int kMergePerThread = kMaxSlices * kMaxTopK / kMergeThreads;  // 8
-
-template <typename T>
-__global__ void __launch_bounds__(kMergeThreads)
-topk_sample_kernel(const uint64_t* __restrict__ work, int slices, int k,
-                   const float* __restrict__ gumbel, float temperature,
-                   int32_t* __restrict__ token_out, float* __restrict__ prob_out)
-{
-    __shared__ SelectState st;
-    __shared__ uint64_t sel[kMaxTopK];
-    __shared__ uint64_t ranked[kMaxTopK];
-    const int64_t row = blockIdx.x;
-    const int n = slices * k;
-    pdl_wait();
-    pdl_allow_dependents();
-    uint64_t key[kMergePerThread];
-    bool valid[kMergePerThread];
-#pragma unroll
-    for (int m = 0; m < kMergePerThread; ++m) {
-        const int i = threadIdx.x + m * kMergeThreads;
-        // padding keys (0) of short slices are not candidates
-        key[m] = (i < n) ? work[row * n + i] : 0ull;
-        valid[m] = key[m] != 0ull;
-    }
-    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
-#pragma unroll
-    for (int m = 0; m < kMergePerThread; ++m)
-        if (valid[m] && selected(key[m], st)) {
-            const int slot = atomicAdd(&st.count, 1);
-            if (slot < k)
-                sel[slot] = key[m];
-        }
-    __syncthreads();
-    // order the k candidates by counting: rank = number of larger keys
-    if (threadIdx.x < k) {
-        const uint64_t mine = sel[threadIdx.x];
-        int rank = 0;
-        for (int j = 0; j < k; ++j)
-            rank += sel[j] > mine;
-        ranked[rank] = mine;
-    }
-    __syncthreads();
-
-    // Warp 0 takes the decision, two ranks per lane (k <= 64).  Per rank j:
-    // e_j = exp((l_j - l_0) / T) and the score fl(fl(l_j / T) + g_j), two
-    // correctly rounded operations.  The token is the first rank with the
-    // largest score, as a scan in rank order that moves on only to a strictly
-    // larger score finds it: NaN scores after rank 0 never win, a NaN at rank 0
-    // always does.
-    if (threadIdx.x >= 32)
-        return;
-    const int lane = threadIdx.x;
-    const float l0 = cand_value<T>(ranked[0]);
-    float ej[2], bs = 0.f, z = 0.f;
-    int bj = k;  // none yet
-    float s0 = 0.f;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int j = lane + 32 * r;
-        ej[r] = 0.f;
-        if (j < k) {
-            const float l = cand_value<T>(ranked[j]);
-            ej[r] = expf((l - l0) / temperature);
-            const float sc = __fadd_rn(__fdiv_rn(l, temperature), gumbel[row * k + j]);
-            if (j == 0)
-                s0 = sc;
-            if (!isnan(sc) && (bj == k || sc > bs)) {
-                bs = sc;
-                bj = j;
+        for (int m = 0; m < kPerThread; ++m)
+            if (valid[m] && selected(key[m], st)) {
+                const int slot = atomicAdd(&st.count, 1);
+                if (slot < k)  // exactly k are selected; the test only guards the bound
+                    out[slot] = cand_key<T>(val[m], first + pos[m]);
             }
-            z += ej[r];
-        }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
-        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, o);
-        if (oj < k && (bj == k || os > bs || (os == bs && oj < bj))) {
-            bs = os;
-            bj = oj;
-        }
-        z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    // Arrival: the barrier orders every thread's candidate stores before thread
+    // 0's fence, which makes them visible device-wide before the count (a
+    // cumulative release); the CTA that counts last fences again before its
+    // reads (acquire) and so sees every other CTA's stores, and merges.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();  // release: the CTA's stores, ordered by the barrier, before the count
+        const unsigned before = atomicAdd(counters + row, 1u);
+        __threadfence();  // acquire: the other CTAs' stores before this CTA's reads
+        if (before >= (unsigned)slices)  // the counter was not zero when the call began
+            record_device_error(err_word, kDeviceErrWorkspace);
+        last = before == (unsigned)slices - 1u;
+        if (last)
+            counters[row] = 0;  // every CTA of the row has arrived: ready for the next call
     }
-    s0 = __shfl_sync(0xFFFFFFFFu, s0, 0);
-    const int best = isnan(s0) ? 0 : bj;
-    const float eb = __shfl_sync(0xFFFFFFFFu, best < 32 ? ej[0] : ej[1], best & 31);
-    if (lane == 0) {
-        token_out[row] = (int32_t)cand_index(ranked[best]);
-        prob_out[row] = eb / z;
-    }
+    __syncthreads();
+    if (!last)
+        return;
+    merge_and_sample<T>(row_cand, slices * k, k, gumbel + row * k, temperature, token_out + row,
+                        prob_out + row, st, sel, ranked);
 }
 
 }  // namespace
@@ -499,37 +527,43 @@ int topk_max_slices()
     return kMaxSlices;
 }
 
+size_t topk_counter_bytes()
+{
+    return kCounterBytes;
+}
+
 cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
                                float* prob_out, int64_t rows, int64_t vocab, int k,
-                               float temperature, arops_dtype dtype, uint64_t* work,
+                               float temperature, arops_dtype dtype, void* workspace,
                                cudaStream_t stream)
 {
     const int slices = topk_slices(vocab);
-    const dim3 grid1((unsigned)slices, (unsigned)rows);
+    const dim3 grid((unsigned)slices, (unsigned)rows);
     const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
     const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
-    cudaError_t err;
-    if (dtype == AROPS_BF16) {
-        const auto* lg = static_cast<const __nv_bfloat16*>(logits);
-        err = vec ? launch(topk_slice_kernel<__nv_bfloat16, true>, grid1, dim3(kSliceThreads), 0,
-                           stream, lg, vocab, k, slices, work)
-                  : launch(topk_slice_kernel<__nv_bfloat16, false>, grid1, dim3(kSliceThreads), 0,
-                           stream, lg, vocab, k, slices, work);
-    } else {
-        const auto* lg = static_cast<const float*>(logits);
-        err = vec ? launch(topk_slice_kernel<float, true>, grid1, dim3(kSliceThreads), 0, stream,
-                           lg, vocab, k, slices, work)
-                  : launch(topk_slice_kernel<float, false>, grid1, dim3(kSliceThreads), 0, stream,
-                           lg, vocab, k, slices, work);
-    }
+    unsigned* counters = static_cast<unsigned*>(workspace);
+    uint64_t* work = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(workspace) +
+                                                 kCounterBytes);
+    unsigned* word = nullptr;
+    cudaError_t err = device_error_word(&word);
     if (err != cudaSuccess)
         return err;
-    if (dtype == AROPS_BF16)
-        return launch(topk_sample_kernel<__nv_bfloat16>, dim3((unsigned)rows), dim3(kMergeThreads),
-                      0, stream, (const uint64_t*)work, slices, k, gumbel, temperature, token_out,
-                      prob_out);
-    return launch(topk_sample_kernel<float>, dim3((unsigned)rows), dim3(kMergeThreads), 0, stream,
-                  (const uint64_t*)work, slices, k, gumbel, temperature, token_out, prob_out);
+    if (dtype == AROPS_BF16) {
+        const auto* lg = static_cast<const __nv_bfloat16*>(logits);
+        return vec ? launch(topk_sample_kernel<__nv_bfloat16, true>, grid, dim3(kSliceThreads), 0,
+                            stream, lg, vocab, k, slices, counters, work, gumbel, temperature,
+                            token_out, prob_out, word)
+                   : launch(topk_sample_kernel<__nv_bfloat16, false>, grid, dim3(kSliceThreads), 0,
+                            stream, lg, vocab, k, slices, counters, work, gumbel, temperature,
+                            token_out, prob_out, word);
+    }
+    const auto* lg = static_cast<const float*>(logits);
+    return vec ? launch(topk_sample_kernel<float, true>, grid, dim3(kSliceThreads), 0, stream, lg,
+                        vocab, k, slices, counters, work, gumbel, temperature, token_out,
+                        prob_out, word)
+               : launch(topk_sample_kernel<float, false>, grid, dim3(kSliceThreads), 0, stream, lg,
+                        vocab, k, slices, counters, work, gumbel, temperature, token_out,
+                        prob_out, word);
 }
 
 // ---------------------------------------------------------------------------
@@ -539,11 +573,15 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
 // real-time audio or streaming callback, where cudaMalloc is off limits
 // because it can block and synchronise the device, or a plugin that is handed
 // buffers by a host application that owns all device memory.  Every GPU that
-// loads the library holds this array until the process exits.
+// loads the library holds this array until the process exits.  It holds the
+// arrival counters (zero when the module is loaded, as every __device__
+// variable without an initialiser is, and left zero by every call) and then
+// 1 MiB of candidate keys.
 // ---------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB of candidates
 
-static __device__ __align__(256) uint64_t g_topk_scratch[kNoAllocScratchBytes / sizeof(uint64_t)];
+static __device__ __align__(256) uint64_t
+    g_topk_scratch[(kCounterBytes + kNoAllocScratchBytes) / sizeof(uint64_t)];
 
 size_t topk_noalloc_scratch_bytes()
 {
@@ -558,9 +596,9 @@ size_t topk_noalloc_scratch_bytes()
 // context that was reset and created anew).  Once this code is loaded in the
 // context the lookup allocates nothing; the first lookup in a context loads it
 // (with lazy module loading, the CUDA default), which reserves the array.
-cudaError_t topk_noalloc_scratch(uint64_t** ptr)
+cudaError_t topk_noalloc_scratch(void** ptr)
 {
-    return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_topk_scratch);
+    return cudaGetSymbolAddress(ptr, g_topk_scratch);
 }
 
 }  // namespace arops

@@ -6,8 +6,10 @@
 Shapes are the operators' workload sizes (add+RMSNorm bf16 4096x2048, SwiGLU
 bf16 8192x6144, M-RoPE bf16 4096 tokens x 16/8 heads x 128, RMSNorm fp32
 64x1024, decode steps at batch 5 and 256); ``--rows`` scales the row count.
-Prints one line per operator: median and mean microseconds per launch and the
-algorithmic HBM GB/s (every operand read once, every output written once).
+Prints one line per operator: median and minimum microseconds per launch (each
+launch between its own pair of events), the per-launch time of the same
+launches back to back, and the algorithmic HBM GB/s (every operand read once,
+every output written once) of both.
 
 Each operator gets enough copies of its buffers to cover 512 MB (4x the L2) and
 successive launches cycle through them, so every launch reads from DRAM and
@@ -23,13 +25,21 @@ import statistics
 import torch
 
 from . import (add_layernorm, add_rmsnorm, layernorm, mrope_qk, rmsnorm, set_pdl, set_streaming,
-               mrope_kv_append, swiglu, topk_sample, topk_sample_workspace)
+               mrope_kv_append, swiglu, topk_sample, topk_sample_prepare,
+               topk_sample_workspace)
 from . import inputs as I
 from .chain import DecodeChain
 
 OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode5", "decode256")
 EXTRA_OPS = ("layernorm", "add_layernorm", "decode5_ln", "decode256_ln", "topk_sample",
-             "mrope_kv_append")
+             "mrope_kv_append", "copy_add_rmsnorm", "copy_mrope_qk", "copy_swiglu")
+# Size-matched device copies: a plain device-to-device copy (torch's copy
+# kernel, not this library's) that reads half and writes half of an
+# operator's algorithmic bytes at the workload size, as the ceiling a kernel
+# of that size and launch pattern can reach.
+COPY_OF = {"copy_add_rmsnorm": (4 * 4096 * 2048 + 2048) * 2,
+           "copy_mrope_qk": 2 * 4096 * 24 * 128 * 2 + 3 * 4096 * 4,
+           "copy_swiglu": 3 * 8192 * 6144 * 2}
 
 
 CHAIN_PDL = True
@@ -96,12 +106,18 @@ def make(op: str, rows: int | None, dev: torch.device, seed: int = 0):
     if op == "topk_sample":
         r = rows or 5
         t = {k: v.to(dev) for k, v in I.topk_inputs(r, 151936, 50, "bf16", seed).items()}
-        ws = torch.empty(topk_sample_workspace(r, 151936, 50), dtype=torch.uint8, device=dev)
+        ws = topk_sample_prepare(torch.empty(topk_sample_workspace(r, 151936, 50),
+                                             dtype=torch.uint8, device=dev))
         tok = torch.empty(r, dtype=torch.int32, device=dev)
         prob = torch.empty(r, dtype=torch.float32, device=dev)
         return ((lambda: topk_sample(t["logits"], t["gumbel"], 50, 0.8, workspace=ws,
                                      token_out=tok, prob_out=prob)),
                 r * 151936 * 2 + r * 50 * 4 + r * 8, f"bf16 {r}x151936, top-50")
+    if op in COPY_OF:
+        half = COPY_OF[op] // 2 // 16 * 16
+        src = torch.randint(0, 255, (half,), dtype=torch.uint8, device=dev)
+        dst = torch.empty_like(src)
+        return (lambda: dst.copy_(src)), 2 * half, f"device copy of {half} B"
     if op.startswith("decode"):
         b = rows or (5 if op.startswith("decode5") else 256)
         norm = "layer" if op.endswith("_ln") else "rms"
@@ -134,6 +150,23 @@ def time_op(fns, iters: int) -> list[float]:
     return [1e3 * a.elapsed_time(b) for a, b in ev]
 
 
+def time_back_to_back(fns, iters: int) -> float:
+    """Microseconds per launch of ``iters`` launches enqueued back to back
+    between one pair of events (with programmatic dependent launch when it is
+    enabled, each launch overlaps its predecessor's drain)."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(1e7))
+    e0.record()
+    for i in range(iters):
+        fns[i % len(fns)]()
+    e1.record()
+    torch.cuda.synchronize()
+    return 1e3 * e0.elapsed_time(e1) / iters
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", default="all", choices=("all",) + OPS + EXTRA_OPS)
@@ -156,13 +189,17 @@ def main() -> None:
     for op in (OPS if a.op == "all" else (a.op,)):
         fns, nbytes, desc = make_rotation(op, a.rows, dev, a.copies)
         us = time_op(fns, a.iters)
+        b2b = time_back_to_back(fns, a.iters)
         med = statistics.median(us)
         rec = {"op": op, "shape": desc, "bytes": nbytes, "us_median": round(med, 3),
                "us_mean": round(statistics.fmean(us), 3), "us_min": round(min(us), 3),
-               "gbs_median": round(nbytes / (med * 1e-6) / 1e9, 1)}
+               "gbs_median": round(nbytes / (med * 1e-6) / 1e9, 1),
+               "us_back_to_back": round(b2b, 3),
+               "gbs_back_to_back": round(nbytes / (b2b * 1e-6) / 1e9, 1)}
         print(json.dumps(rec) if a.json else
               f"{op:12s} {desc:40s} median {med:9.3f} us  min {min(us):9.3f} us  "
-              f"{rec['gbs_median']:8.1f} GB/s", flush=True)
+              f"{rec['gbs_median']:8.1f} GB/s  back to back {b2b:9.3f} us "
+              f"{rec['gbs_back_to_back']:8.1f} GB/s", flush=True)
 
 
 if __name__ == "__main__":

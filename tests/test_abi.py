@@ -38,7 +38,7 @@ def test_header_declares_the_operators():
 def test_every_declared_symbol_is_exported(L):
     for n in _declared_symbols():
         assert hasattr(L, n), n
-    assert L.arops_version() == 10000
+    assert L.arops_version() == 20000
 
 
 def test_status_strings(L):
@@ -99,7 +99,7 @@ def test_topk_sample_argument_errors(L):
 
     n = C.c_size_t(0)
     assert L.arops_topk_sample_workspace(5, 151936, 50, C.byref(n)) == 0
-    assert n.value == 5 * 38 * 50 * 8
+    assert n.value == (1 << 18) + 5 * 38 * 50 * 8  # arrival counters, then candidates
     assert L.arops_topk_sample_workspace(5, 100, 0, C.byref(n)) == 1
     assert L.arops_topk_sample_workspace(5, 100, 101, C.byref(n)) == 1
     assert L.arops_topk_sample_workspace(5, 1000, 65, C.byref(n)) == 2
@@ -111,4 +111,7 @@ def test_topk_sample_argument_errors(L):
     assert L.arops_topk_sample(1, 1, 1, 1, 5, 1000, 5, 0.0, 1, 8, 1 << 20, None) == 1
     assert L.arops_topk_sample(1, 1, 1, 1, 5, 1000, 5, 1.0, 1, 9, 1 << 20, None) == 1  # misaligned
     assert L.arops_topk_sample(None, None, None, None, 0, 1000, 5, 1.0, 1, None, 0, None) == 0
+    L.arops_topk_sample_prepare.argtypes = [C.c_void_p, C.c_size_t, C.c_void_p]
+    assert L.arops_topk_sample_prepare(None, 1 << 20, None) == 1
+    assert L.arops_topk_sample_prepare(16, (1 << 18) - 1, None) == 1  # smaller than the counters
     assert L.arops_launch_count() == before

@@ -65,6 +65,43 @@ def test_rmsnorm_shapes_past_one_wave(dtype, hidden):
     check(y, exact, dtype, what=f"rmsnorm {dtype} {rows}x{hidden}")
 
 
+def _sm_count() -> int:
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+# Decode-size problems with at least one row per SM (256 decode candidates)
+# take two vectors per lane over hidden/512 warps (bf16); fewer rows take one
+# vector per lane.  Widths on both sides of each warp count, rows at the SM
+# count and above, all four norms.
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hidden", [264, 1000, 1024, 2048, 4000, 8192])
+@pytest.mark.parametrize("extra_rows", [0, 57])
+def test_norms_with_a_row_per_sm(dtype, hidden, extra_rows):
+    nvec = hidden // (8 if dtype == "bf16" else 4)
+    rows = _sm_count() + extra_rows
+    if rows * nvec > _sm_count() * 2048:
+        rows = _sm_count() * 2048 // nvec  # still within one vector per resident thread
+    orc = oracle.get()
+    inp = _ln_inputs(rows, hidden, dtype, hidden + extra_rows)
+    x, r, g, b = dev(inp["x"]), dev(inp["residual"]), dev(inp["gamma"]), dev(inp["beta"])
+    y = ops.rmsnorm(x, g, EPS)
+    y2, r_out = ops.add_rmsnorm(x, r, g, EPS, residual_out=torch.empty_like(r))
+    y3 = ops.layernorm(x, g, b, EPS)
+    y4, r_out4 = ops.add_layernorm(x, r, g, b, EPS, residual_out=torch.empty_like(r))
+    torch.cuda.synchronize()
+    check(y, orc.rmsnorm(inp["x"], inp["gamma"], EPS), dtype, what=f"rmsnorm {rows}x{hidden}")
+    y2_e, r_e = orc.add_rmsnorm(inp["x"], inp["residual"], inp["gamma"], EPS, dtype)
+    assert np.array_equal(to_f64(r_out), r_e) and np.array_equal(to_f64(r_out4), r_e)
+    check(y2, y2_e, dtype, what=f"add_rmsnorm {rows}x{hidden}")
+    xr = to_f64(inp["x"])
+    check(y3, orc.layernorm(inp["x"], inp["gamma"], inp["beta"], EPS), dtype,
+          _ln_scale(xr, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS),
+          what=f"layernorm {rows}x{hidden}", band=LN_BAND)
+    y4_e, _ = orc.add_layernorm(inp["x"], inp["residual"], inp["gamma"], inp["beta"], EPS, dtype)
+    check(y4, y4_e, dtype, _ln_scale(r_e, to_f64(inp["gamma"]), to_f64(inp["beta"]), EPS),
+          what=f"add_layernorm {rows}x{hidden}", band=LN_BAND)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_rmsnorm_large_bf16_prefill(dtype, family):
     y, exact = _run_rmsnorm(4096, 2048, dtype, seed=3)

@@ -106,18 +106,50 @@ def test_topk_sample_distribution():
     assert chi2 < 25.0, (counts, n * p)
 
 
+COUNTER_BYTES = 1 << 18  # the workspace's arrival counters (one per row, up to 65535 rows)
+
+
 def test_topk_sample_workspace_is_exact_and_guarded():
     rows, vocab, k = 5, 50000, 32
     need = ops.topk_sample_workspace(rows, vocab, k)
-    assert need == rows * ((vocab + 4095) // 4096) * k * 8
+    assert need == COUNTER_BYTES + rows * ((vocab + 4095) // 4096) * k * 8
     ws = Guarded((need // 4,), torch.float32)  # canaries on both sides of the workspace
+    w8 = ws.t.view(torch.uint8)
+    ops.topk_sample_prepare(w8)
     inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=12)
-    tok, prob = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.1,
-                                workspace=ws.t.view(torch.uint8))
+    tok, prob = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.1, workspace=w8)
     torch.cuda.synchronize()
     ws.check()
+    assert not w8[:COUNTER_BYTES].any()  # the call left its counters at zero
     t_ref, p_ref = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 1.1)
     assert np.array_equal(tok.cpu().numpy(), t_ref)
+
+
+def test_topk_sample_one_workspace_for_many_shapes():
+    """The counters sit at a fixed place and every call leaves them at zero, so
+    one prepared workspace serves calls of any shape in turn."""
+    shapes = ((5, 151936, 50), (33, 70000, 64), (3, 4096, 7), (64, 151936, 50), (1, 100, 1))
+    need = max(ops.topk_sample_workspace(r, v, k) for r, v, k in shapes)
+    w8 = ops.topk_sample_prepare(torch.empty(need, dtype=torch.uint8, device="cuda"))
+    for i, (r, v, k) in enumerate(shapes):
+        inp = inputs.topk_inputs(r, v, k, "bf16", seed=40 + i)
+        tok, prob = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 0.9, workspace=w8)
+        t_ref, p_ref = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 0.9)
+        assert np.array_equal(tok.cpu().numpy(), t_ref), (r, v, k)
+        np.testing.assert_allclose(to_f64(prob), p_ref, rtol=1e-5, atol=0)
+    assert not w8[:COUNTER_BYTES].any()
+
+
+def test_topk_sample_flags_a_workspace_whose_counters_were_not_cleared():
+    """Counters left non-zero (a workspace never prepared) are reported in the
+    device error word; the kernel still completes."""
+    rows, vocab, k = 2, 10000, 8
+    w8 = torch.full((ops.topk_sample_workspace(rows, vocab, k),), 0xA5, dtype=torch.uint8,
+                    device="cuda")
+    inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=3)
+    ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.0, workspace=w8)
+    torch.cuda.synchronize()
+    assert ops.device_errors(clear=True) == 4  # AROPS_DEVICE_ERR_WORKSPACE
 
 
 def test_topk_sample_empty_rows():

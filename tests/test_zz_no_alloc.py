@@ -3,8 +3,9 @@
 arops_topk_sample_noalloc serves callers that cannot allocate device memory
 (for example code inside a host application's real-time audio callback, where
 cudaMalloc may block and synchronise the device, or a plugin that only receives
-buffers from a host that owns all device memory): it takes its scratch from a
-1 MiB array the library keeps in device memory.  This file is collected last
+buffers from a host that owns all device memory): it takes its scratch from an
+array the library keeps in device memory (arrival counters, then 1 MiB of
+candidates).  This file is collected last
 (after every other test) and also passes when run alone in a fresh process.
 """
 import ctypes
@@ -45,7 +46,7 @@ def _noalloc(L, logits, gumbel, rows, vocab, k, temp, dtype, stream):
 def _with_workspace(L, logits, gumbel, rows, vocab, k, temp, dtype, stream):
     n = ctypes.c_size_t(0)
     assert L.arops_topk_sample_workspace(rows, vocab, k, ctypes.byref(n)) == 0
-    ws = torch.empty(n.value, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(n.value, dtype=torch.uint8, device="cuda")  # counters start at zero
     tok = torch.empty(rows, dtype=torch.int32, device="cuda")
     prob = torch.empty(rows, dtype=torch.float32, device="cuda")
     st = L.arops_topk_sample(logits.data_ptr(), gumbel.data_ptr(), tok.data_ptr(), prob.data_ptr(),

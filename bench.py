@@ -99,7 +99,9 @@ def source_digest(*rel: str) -> str:
 
 
 def ncu_traffic(kernel: str, sources: tuple[str, ...]) -> float | None:
-    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json),
+    """Memory traffic per launch recorded from an ncu capture
+    (profiles/traffic.json): DRAM reads plus the bytes the kernel wrote into L2
+    (all of which reach DRAM once; most are still in L2 when the kernel ends),
     or None when absent or when the kernel's sources changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -109,7 +111,7 @@ def ncu_traffic(kernel: str, sources: tuple[str, ...]) -> float | None:
         return None
     if rec.get("source_digest") != source_digest(*sources):
         return None
-    return float(rec["dram_bytes_per_launch"])
+    return float(rec.get("traffic_bytes_per_launch", rec["dram_bytes_per_launch"]))
 
 
 class ClockSampler:
@@ -608,9 +610,9 @@ def main() -> None:
                 "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
                 "us_per_decode_launch": decode_launch_us.get(dominant, {}),
                 "note": "dominant by share of step time; achieved = its algorithmic bytes per "
-                        "step / its time per step; traffic = DRAM bytes per launch, averaged "
-                        "over the step's prefill and decode launches (reads = operands, "
-                        "outputs still in L2 at kernel end); all but 2 of its launches are "
+                        "step / its time per step; traffic = DRAM reads + bytes written into "
+                        "L2 per launch (ncu, profiles/traffic.json), averaged over the step's "
+                        "prefill and decode launches; all but 2 of its launches are "
                         "decode launches of 45 KB to 4.2 MB, bound by the latency of a "
                         "dependent launch (us_per_decode_launch) rather than by bandwidth"}
     sw_us = ops_report["swiglu"]["us"]

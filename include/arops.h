@@ -286,10 +286,12 @@ AROPS_API arops_status arops_topk_sample_noalloc(const void* logits, const float
  * for its predecessor's memory before it reads activations or writes anything,
  * so results and stream-order semantics are unchanged.  It only shortens the
  * gaps between back-to-back launches (decode steps).
- * Contract while enabled: the norms read their weights before that wait, so
- * gamma and beta must not be written by the kernel launched immediately before
- * on the same stream (kernels launched earlier have completed by then); model
- * weights meet it.  Returns the old setting.
+ * Contract while enabled: some read-only parameters are read before that
+ * wait, so they must not be written by the kernel launched immediately before
+ * on the same stream (kernels launched earlier have completed by then): gamma
+ * and beta of the norms, and pos of arops_mrope_qk.  Model weights, and
+ * position ids written ahead of a decode step, meet it.  Returns the old
+ * setting.
  */
 AROPS_API int arops_set_pdl(int enable);
 

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <string>
 
 #include "arops.h"
@@ -224,6 +225,24 @@ cudaError_t resident_ctas(K kernel, int threads, size_t smem, int* ctas)
             return e;
     }
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, kernel, threads, smem);
+}
+
+// CTAs of `Kernel` (at `threads` threads per CTA, no dynamic shared memory)
+// that `waves` full waves fill on a device of `sm_count` SMs.  The resident
+// CTAs per SM are looked up once per kernel (every device this library runs on
+// is the same part); a failed lookup counts one per SM.
+template <auto Kernel>
+int64_t wave_ctas(int threads, int sm_count, int waves)
+{
+    static std::atomic<int> per_sm{0};
+    int v = per_sm.load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, Kernel, threads, 0) != cudaSuccess ||
+            v < 1)
+            v = 1;
+        per_sm.store(v, std::memory_order_relaxed);
+    }
+    return (int64_t)v * sm_count * waves;
 }
 
 // Launchers (one per operator), called after argument validation.

@@ -70,18 +70,15 @@ __device__ __forceinline__ int32_t position_of(int j, const MropeParams& prm, in
 // pv split the block's E angles between them (F each) and share them with
 // shuffles, so every lane of the warp must take part.
 template <int E, int P>
-__device__ __forceinline__ void token_angles(const int32_t* __restrict__ pos, int64_t tokens,
-                                             int64_t t, const double* inv_freq,
-                                             const MropeParams& prm, int lane, float* c, float* s)
+__device__ __forceinline__ void token_angles(int32_t pt, int32_t ph, int32_t pw,
+                                             const double* inv_freq, const MropeParams& prm,
+                                             int lane, float* c, float* s)
 {
     constexpr int G = 32 / P;                // heads per warp pass
     constexpr int F = (E >= G) ? E / G : 1;  // angles evaluated per lane
     const int pv = lane % P;
     const int hg = lane / P;
     const int j0 = pv * E;
-    const int32_t pt = __ldg(pos + t);
-    const int32_t ph = __ldg(pos + tokens + t);
-    const int32_t pw = __ldg(pos + 2 * tokens + t);
     float cs[F], sn[F];
 #pragma unroll
     for (int f = 0; f < F; ++f) {
@@ -99,8 +96,8 @@ __device__ __forceinline__ void token_angles(const int32_t* __restrict__ pos, in
 constexpr int kWarpsPerCta = 4;
 
 // Token of warp unit `unit` and which of the token's `splits` warps it is.
-// The launchers take splits > 1 only when tokens * splits < 2^32, so the unit
-// index fits 32 bits there and the division stays a 32-bit one.
+// splits > 1 only for launches of at most one head pass per resident warp, so
+// the unit index fits 32 bits there and the division stays a 32-bit one.
 __device__ __forceinline__ int64_t unit_token(int64_t unit, int splits, int& part)
 {
     if (splits == 1) {
@@ -148,13 +145,42 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
         }
     }
     fill_inv_freq(inv_freq, HALF, prm);
+    // Decode-size launches (U == 1: one unit per warp) issue their token's
+    // position loads before the dependency wait, so that the loads complete
+    // while the previous kernel drains (with programmatic dependent launch the
+    // caller guarantees that the position ids are not written by the kernel
+    // launched just before this one).  Only the loads move: evaluating the
+    // angles there too measured slower, the window before the wait being
+    // shorter than that work.
+    int32_t pt0 = 0, ph0 = 0, pw0 = 0;
+    if constexpr (U == 1) {
+        if (unit0 < units) {
+            int part0 = 0;
+            const int64_t t0 = unit_token(unit0, splits, part0);
+            pt0 = __ldg(pos + t0);
+            ph0 = __ldg(pos + tokens + t0);
+            pw0 = __ldg(pos + 2 * tokens + t0);
+        }
+    }
     pdl_wait();
     pdl_allow_dependents();
 
-    for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
+    const int64_t unit_stride = (int64_t)gridDim.x * kWarpsPerCta;
+    for (int64_t unit = unit0; unit < units; unit += unit_stride) {
         int part = 0;
         const int64_t t = unit_token(unit, splits, part);
         const int h_first = hg + part * G * U;
+        // the warp's next token into L2 while this one is worked on (a grid of
+        // one wave walks several tokens per warp); decode-size launches (U ==
+        // 1, one unit per warp) leave even the branch out, as the norm does
+        if (U > 1 && lane == 0 && part == 0 && unit + unit_stride < units) {
+            int part_n = 0;
+            const int64_t tn = unit_token(unit + unit_stride, splits, part_n);
+            if (hq > 0)
+                prefetch_l2(q + (size_t)tn * hq * D, (uint32_t)(hq * D * sizeof(T)));
+            if (hk > 0)
+                prefetch_l2(k + (size_t)tn * hk * D, (uint32_t)(hk * D * sizeof(T)));
+        }
 
         // the first batch of heads is loaded before the angles are evaluated, so
         // the q/k loads and the position loads share one memory latency
@@ -173,7 +199,11 @@ mrope_vec_kernel(const T* q, const T* k, T* q_out, T* k_out, const int32_t* __re
         };
         load_batch(h_first);
         float c[E], s[E];
-        token_angles<E, P>(pos, tokens, t, inv_freq, prm, lane, c, s);
+        if (U == 1 && unit == unit0)
+            token_angles<E, P>(pt0, ph0, pw0, inv_freq, prm, lane, c, s);
+        else
+            token_angles<E, P>(__ldg(pos + t), __ldg(pos + tokens + t), __ldg(pos + 2 * tokens + t),
+                               inv_freq, prm, lane, c, s);
 
         for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
             if (h0 != h_first)
@@ -421,10 +451,22 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
     pdl_wait();
     pdl_allow_dependents();
 
-    for (int64_t unit = unit0; unit < units; unit += (int64_t)gridDim.x * kWarpsPerCta) {
+    const int64_t unit_stride = (int64_t)gridDim.x * kWarpsPerCta;
+    for (int64_t unit = unit0; unit < units; unit += unit_stride) {
         int part = 0;
         const int64_t t = unit_token(unit, splits, part);
         const int h_first = hg + part * G * U;
+        // the warp's next token into L2 while this one is worked on
+        if (U > 1 && lane == 0 && part == 0 && unit + unit_stride < units) {
+            int part_n = 0;
+            const int64_t tn = unit_token(unit + unit_stride, splits, part_n);
+            if (hq > 0)
+                prefetch_l2(q + (size_t)tn * hq * D, (uint32_t)(hq * D * sizeof(T)));
+            if (hk > 0) {
+                prefetch_l2(k + (size_t)tn * hk * D, (uint32_t)(hk * D * sizeof(T)));
+                prefetch_l2(v + (size_t)tn * hk * D, (uint32_t)(hk * D * sizeof(T)));
+            }
+        }
         int64_t cb = -1, cs = -1;
         if (hk > 0) {
             cb = __ldg(ca.loc + t);
@@ -455,7 +497,8 @@ mrope_append_kernel(const T* q, const T* k, const T* v, T* q_out, T* k_cache, T*
         };
         load_batch(h_first);
         float c[E], s[E];
-        token_angles<E, P>(pos, tokens, t, inv_freq, prm, lane, c, s);
+        token_angles<E, P>(__ldg(pos + t), __ldg(pos + tokens + t), __ldg(pos + 2 * tokens + t),
+                           inv_freq, prm, lane, c, s);
 
         for (int h0 = h_first; h0 < nh; h0 += G * U * splits) {
             if (h0 != h_first)
@@ -569,35 +612,38 @@ inline bool one_pass_per_warp(int64_t tokens, int passes, int64_t cap)
     return tokens * passes <= cap;
 }
 
-// Whether a token's passes may be shared by two warps (the unit index must
-// fit 32 bits, see unit_token).
-inline bool two_warps_per_token(int64_t tokens)
+// Otherwise one warp per token with every pass's heads in flight at once (U =
+// passes, so no registers are held for absent heads), on a grid of one wave of
+// resident CTAs: each warp walks several tokens and prefetches its next token
+// into L2 while it works on the current one.  4096 tokens of 16 + 8 heads of
+// 128 measured 8.1 us a launch back to back on B200, against 9.2 us with one
+// warp per token and 1,024 CTAs, and 8.5 us with two warps per token.
+constexpr int kPrefillWaves = 1;
+
+template <typename T, int P, int U>
+cudaError_t launch_vec_wave(const MropeArgs& a, const MropeParams& prm, cudaStream_t st,
+                            int64_t cap, int sm_count)
 {
-    return tokens * 2 <= (int64_t)UINT32_MAX;
+    cap = std::min<int64_t>(
+        cap, wave_ctas<mrope_vec_kernel<T, P, U>>(32 * kWarpsPerCta, sm_count, kPrefillWaves));
+    return launch_vec_u<T, P, U>(a, prm, st, cap);
 }
 
-// Otherwise a token with more than two passes is shared by two warps, each
-// loading its half of the passes at once (U = heads per lane in flight), so no
-// registers are held for absent heads and the grid has more, lighter warps:
-// 4096 tokens of 16 + 8 heads of 128 measured 9.15 us a launch back to back
-// on B200 with two warps of 3 passes, against 9.7 us with one warp of 6.
 template <typename T, int P>
-cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap)
+cudaError_t launch_vec(const MropeArgs& a, const MropeParams& prm, cudaStream_t st, int64_t cap,
+                       int sm_count)
 {
     constexpr int G = 32 / P;
     const int passes = (int)ceil_div(a.n_q_heads + a.n_k_heads, G);
     if (one_pass_per_warp(a.tokens, passes, cap))
         return launch_vec_u<T, P, 1>(a, prm, st, cap, passes);
     if (passes <= 2)
-        return launch_vec_u<T, P, 2>(a, prm, st, cap);
-    if (two_warps_per_token(a.tokens) && passes <= 8) {
-        if (passes <= 4)
-            return launch_vec_u<T, P, 2>(a, prm, st, cap, 2);
-        if (passes <= 6)
-            return launch_vec_u<T, P, 3>(a, prm, st, cap, 2);
-        return launch_vec_u<T, P, 4>(a, prm, st, cap, 2);
-    }
-    return launch_vec_u<T, P, kHeadUnroll>(a, prm, st, cap);
+        return launch_vec_wave<T, P, 2>(a, prm, st, cap, sm_count);
+    if (passes <= 4)
+        return launch_vec_wave<T, P, 4>(a, prm, st, cap, sm_count);
+    if (passes <= 6)
+        return launch_vec_wave<T, P, 6>(a, prm, st, cap, sm_count);
+    return launch_vec_wave<T, P, kHeadUnroll>(a, prm, st, cap, sm_count);
 }
 
 // Streaming launch; cudaErrorNotSupported when two slots per warp do not fit.
@@ -666,12 +712,12 @@ cudaError_t launch_mrope_t(const MropeArgs& a, const MropeParams& prm, cudaStrea
     }
     if (aligned && half % E == 0) {
         switch (half / E) {
-        case 1: return launch_vec<T, 1>(a, prm, st, cap);
-        case 2: return launch_vec<T, 2>(a, prm, st, cap);
-        case 4: return launch_vec<T, 4>(a, prm, st, cap);
-        case 8: return launch_vec<T, 8>(a, prm, st, cap);
-        case 16: return launch_vec<T, 16>(a, prm, st, cap);
-        case 32: return launch_vec<T, 32>(a, prm, st, cap);
+        case 1: return launch_vec<T, 1>(a, prm, st, cap, di.sm_count);
+        case 2: return launch_vec<T, 2>(a, prm, st, cap, di.sm_count);
+        case 4: return launch_vec<T, 4>(a, prm, st, cap, di.sm_count);
+        case 8: return launch_vec<T, 8>(a, prm, st, cap, di.sm_count);
+        case 16: return launch_vec<T, 16>(a, prm, st, cap, di.sm_count);
+        case 32: return launch_vec<T, 32>(a, prm, st, cap, di.sm_count);
         default: break;
         }
     }
@@ -696,24 +742,33 @@ cudaError_t launch_append_u(const MropeArgs& a, const AppendArgs& x, const Mrope
                   (int)a.n_q_heads, (int)a.n_k_heads, splits, prm, ca, word);
 }
 
+template <typename T, int P, int U>
+cudaError_t launch_append_wave(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
+                               const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap,
+                               int sm_count)
+{
+    cap = std::min<int64_t>(
+        cap, wave_ctas<mrope_append_kernel<T, P, U>>(32 * kWarpsPerCta, sm_count, kPrefillWaves));
+    return launch_append_u<T, P, U>(a, x, prm, ca, word, st, cap);
+}
+
 template <typename T, int P>
 cudaError_t launch_append_p(const MropeArgs& a, const AppendArgs& x, const MropeParams& prm,
-                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap)
+                            const CacheArgs& ca, unsigned* word, cudaStream_t st, int64_t cap,
+                            int sm_count)
 {
     constexpr int G = 32 / P;
     const int passes = (int)ceil_div(a.n_q_heads + 2 * a.n_k_heads, G);
     if (one_pass_per_warp(a.tokens, passes, cap))
         return launch_append_u<T, P, 1>(a, x, prm, ca, word, st, cap, passes);
+    // as in launch_vec: one warp per token, one wave of resident CTAs
     if (passes <= 2)
-        return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap);
-    if (two_warps_per_token(a.tokens) && passes <= 8) {  // as in launch_vec
-        if (passes <= 4)
-            return launch_append_u<T, P, 2>(a, x, prm, ca, word, st, cap, 2);
-        if (passes <= 6)
-            return launch_append_u<T, P, 3>(a, x, prm, ca, word, st, cap, 2);
-        return launch_append_u<T, P, 4>(a, x, prm, ca, word, st, cap, 2);
-    }
-    return launch_append_u<T, P, kHeadUnroll>(a, x, prm, ca, word, st, cap);
+        return launch_append_wave<T, P, 2>(a, x, prm, ca, word, st, cap, sm_count);
+    if (passes <= 4)
+        return launch_append_wave<T, P, 4>(a, x, prm, ca, word, st, cap, sm_count);
+    if (passes <= 6)
+        return launch_append_wave<T, P, 6>(a, x, prm, ca, word, st, cap, sm_count);
+    return launch_append_wave<T, P, kHeadUnroll>(a, x, prm, ca, word, st, cap, sm_count);
 }
 
 template <typename T>
@@ -740,12 +795,12 @@ cudaError_t launch_append_t(const MropeArgs& a, const AppendArgs& x, const Mrope
     const int64_t cap = (int64_t)di.sm_count * 64;
     if (aligned && half % E == 0) {
         switch (half / E) {
-        case 1: return launch_append_p<T, 1>(a, x, prm, ca, word, st, cap);
-        case 2: return launch_append_p<T, 2>(a, x, prm, ca, word, st, cap);
-        case 4: return launch_append_p<T, 4>(a, x, prm, ca, word, st, cap);
-        case 8: return launch_append_p<T, 8>(a, x, prm, ca, word, st, cap);
-        case 16: return launch_append_p<T, 16>(a, x, prm, ca, word, st, cap);
-        case 32: return launch_append_p<T, 32>(a, x, prm, ca, word, st, cap);
+        case 1: return launch_append_p<T, 1>(a, x, prm, ca, word, st, cap, di.sm_count);
+        case 2: return launch_append_p<T, 2>(a, x, prm, ca, word, st, cap, di.sm_count);
+        case 4: return launch_append_p<T, 4>(a, x, prm, ca, word, st, cap, di.sm_count);
+        case 8: return launch_append_p<T, 8>(a, x, prm, ca, word, st, cap, di.sm_count);
+        case 16: return launch_append_p<T, 16>(a, x, prm, ca, word, st, cap, di.sm_count);
+        case 32: return launch_append_p<T, 32>(a, x, prm, ca, word, st, cap, di.sm_count);
         default: break;
         }
     }

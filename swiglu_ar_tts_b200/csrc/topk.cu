@@ -45,6 +45,17 @@ constexpr size_t kCounterBytes = size_t(1) << 18;
 static_assert(kCounterBytes >= sizeof(unsigned) * kMaxRows, "a counter per row");
 constexpr unsigned kDeviceErrWorkspace = 4u;  // a counter was not zero when a call began
 
+// atomicAdd with release and acquire semantics at GPU scope.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // IEEE float bits, reordered so that unsigned comparison follows the value.
 __device__ __forceinline__ uint32_t order_bits(float v)
 {
@@ -324,6 +335,15 @@ __device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float
                                  float temperature, int32_t* token_out, float* prob_out,
                                  SelectState& st, uint64_t* sel, uint64_t* ranked)
 {
+    // warp 0's Gumbel draws (two ranks per lane), loaded with the keys so that
+    // their latency is not paid again at the decision
+    float gdraw[2] = {0.f, 0.f};
+    if (threadIdx.x < 32) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if ((int)threadIdx.x + 32 * r < k)
+                gdraw[r] = __ldg(g + threadIdx.x + 32 * r);
+    }
     uint64_t key[kMergePerThread];
     bool valid[kMergePerThread];
 #pragma unroll
@@ -372,7 +392,7 @@ __device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float
         if (j < k) {
             const float l = cand_value<T>(ranked[j]);
             ej[r] = expf((l - l0) / temperature);
-            const float sc = __fadd_rn(__fdiv_rn(l, temperature), g[j]);
+            const float sc = __fadd_rn(__fdiv_rn(l, temperature), gdraw[r]);
             if (j == 0)
                 s0 = sc;
             if (!isnan(sc) && (bj == k || sc > bs)) {
@@ -489,14 +509,15 @@ topk_sample_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slice
             }
     }
     // Arrival: the barrier orders every thread's candidate stores before thread
-    // 0's fence, which makes them visible device-wide before the count (a
-    // cumulative release); the CTA that counts last fences again before its
-    // reads (acquire) and so sees every other CTA's stores, and merges.
+    // 0's count, an atomic add with release and acquire semantics at GPU scope
+    // (release is cumulative: it covers the stores the barrier ordered before
+    // it), so the CTA that counts last sees every other CTA's stores, and
+    // merges.
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();  // release: the CTA's stores, ordered by the barrier, before the count
-        const unsigned before = atomicAdd(counters + row, 1u);
-        __threadfence();  // acquire: the other CTAs' stores before this CTA's reads
+        // release: the CTA's stores, ordered by the barrier, before the count;
+        // acquire: the other CTAs' stores before this CTA's reads
+        const unsigned before = atomic_add_acq_rel_gpu(counters + row, 1u);
         if (before >= (unsigned)slices)  // the counter was not zero when the call began
             record_device_error(err_word, kDeviceErrWorkspace);
         last = before == (unsigned)slices - 1u;

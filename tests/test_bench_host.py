@@ -112,11 +112,15 @@ def test_reduce_max_without_group_is_identity():
     assert bench.reduce_max(2.5) == 2.5
 
 
-def test_traffic_record_tracks_kernel_source(tmp_path):
-    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["swiglu_vec_kernel"]
-    got = bench.ncu_traffic("swiglu_vec_kernel", tuple(rec["sources"]))
+@pytest.mark.parametrize("kernel", ["swiglu_vec_kernel", "norm_rows_kernel"])
+def test_traffic_record_tracks_kernel_source(kernel):
+    """The recorded traffic is DRAM reads plus bytes written into L2, reported
+    only while the kernel's sources are the ones captured."""
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+    got = bench.ncu_traffic(kernel, tuple(rec["sources"]))
     if rec["source_digest"] == bench.source_digest(*rec["sources"]):
-        assert got == rec["dram_bytes_per_launch"]
+        assert got == rec["traffic_bytes_per_launch"]
+        assert got >= rec["dram_bytes_per_launch"]  # includes the writes still in L2
     else:  # the kernel changed since the capture: the bench must report null
         assert got is None
     assert bench.ncu_traffic("no_such_kernel", tuple(rec["sources"])) is None

@@ -35,6 +35,27 @@ from . import DTYPES, ArOpsError, lib
 from .inputs import EPS, SECTIONS, THETA, ChainShape, decode_chain_inputs, normal
 
 
+def _pack(tensors, device, fill: bool = True):
+    """One flat device buffer holding a view shaped like each tensor (copied
+    into it when ``fill``), every view starting on a 16-byte boundary."""
+    dtype = tensors[0].dtype
+    esize = tensors[0].element_size()
+    align = max(1, 16 // esize)
+    offs, total = [], 0
+    for t in tensors:
+        assert t.dtype == dtype
+        offs.append(total)
+        total += -(-t.numel() // align) * align
+    flat = torch.empty(max(total, 1), dtype=dtype, device=device)
+    views = []
+    for t, o in zip(tensors, offs):
+        v = flat[o:o + t.numel()].view(t.shape)
+        if fill:
+            v.copy_(t)
+        views.append(v)
+    return flat, views
+
+
 class DecodeChain:
     def __init__(self, shape: ChainShape, dtype: str = "bf16", seed: int = 0,
                  device: str | torch.device = "cuda", eps: float = EPS, theta: float = THETA,
@@ -61,13 +82,23 @@ class DecodeChain:
         d = self.device
         self.residual0 = host["residual"].to(d)
         self.residual = self.residual0.clone()
-        self.inp = {k: [t.to(d).contiguous() for t in v] for k, v in host.items() if k != "residual"}
+        # Every per-layer input lives in one flat device buffer (`flat_in`) and
+        # every per-layer output in another (`flat_out`), as views: a step's
+        # inputs or outputs then move to or from the host as one copy each.
+        # Each view starts on a 16-byte boundary (all sizes are multiples of 16
+        # bytes for these shapes; odd ones are padded).
+        in_keys = [k for k in host if k != "residual"]
+        self.flat_in, views = _pack([t for k in in_keys for t in host[k]], d)
+        self.inp = {}
+        for k in in_keys:
+            self.inp[k], views = views[:len(host[k])], views[len(host[k]):]
         L, B = shape.layers, shape.batch
-        self.y_attn = [torch.empty_like(t) for t in self.inp["x_attn"]]
-        self.y_mlp = [torch.empty_like(t) for t in self.inp["x_mlp"]]
-        self.q_out = [torch.empty_like(t) for t in self.inp["q"]]
-        self.k_out = [torch.empty_like(t) for t in self.inp["k"]]
-        self.act = [torch.empty_like(t) for t in self.inp["gate"]]
+        outs = ([t for t in self.inp["x_attn"]] + [t for t in self.inp["x_mlp"]] +
+                [t for t in self.inp["q"]] + [t for t in self.inp["k"]] +
+                [t for t in self.inp["gate"]])
+        self.flat_out, views = _pack(outs, d, fill=False)
+        self.y_attn, self.y_mlp = views[:L], views[L:2 * L]
+        self.q_out, self.k_out, self.act = views[2 * L:3 * L], views[3 * L:4 * L], views[4 * L:]
         self.pos = torch.zeros(3, B, dtype=torch.int32, device=d)  # the step's position ids
         self._graph: torch.cuda.CUDAGraph | None = None
         self._graph_stream: int | None = None

@@ -315,6 +315,30 @@ __device__ __forceinline__ bool selected(K key, const SelectState& st)
     return (key >> st.shift) >= ((K)st.tau >> st.shift);
 }
 
+// First output slot of this thread's `count` selected keys: the block's
+// selected keys are laid out warp by warp and, within a warp, lane by lane (a
+// warp scan and one barrier; `warp_tot` holds one count per warp).  Every
+// thread of the block must call it.
+__device__ __forceinline__ int selected_offset(int count, int* warp_tot)
+{
+    const int lane = (int)(threadIdx.x & 31);
+    const int warp = (int)(threadIdx.x >> 5);
+    int incl = count;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    if (lane == 31)
+        warp_tot[warp] = incl;
+    __syncthreads();
+    int base = incl - count;
+    for (int w = 0; w < warp; ++w)
+        base += warp_tot[w];
+    return base;
+}
+
 constexpr int kPerThread = kSlice / kSliceThreads;  // 8
 
 // In-slice keys: value bits above the inverted 16-bit position in the slice
@@ -354,13 +378,20 @@ __device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float
         valid[m] = key[m] != 0ull;
     }
     select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
+    {
+        int count = 0;
 #pragma unroll
-    for (int m = 0; m < kMergePerThread; ++m)
-        if (valid[m] && selected(key[m], st)) {
-            const int slot = atomicAdd(&st.count, 1);
-            if (slot < k)
-                sel[slot] = key[m];
-        }
+        for (int m = 0; m < kMergePerThread; ++m)
+            count += valid[m] && selected(key[m], st);
+        int slot = selected_offset(count, reinterpret_cast<int*>(st.warp_top));
+#pragma unroll
+        for (int m = 0; m < kMergePerThread; ++m)
+            if (valid[m] && selected(key[m], st)) {
+                if (slot < k)
+                    sel[slot] = key[m];
+                ++slot;
+            }
+    }
     __syncthreads();
     // order the k candidates by counting: rank = number of larger keys
     if ((int)threadIdx.x < k) {
@@ -500,12 +531,17 @@ topk_sample_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slice
         }
     } else {
         select_top_k<LocalKey<T>::BITS>(key, valid, k, st);
+        int count = 0;
+#pragma unroll
+        for (int m = 0; m < kPerThread; ++m)
+            count += valid[m] && selected(key[m], st);
+        int slot = selected_offset(count, reinterpret_cast<int*>(st.warp_top));
 #pragma unroll
         for (int m = 0; m < kPerThread; ++m)
             if (valid[m] && selected(key[m], st)) {
-                const int slot = atomicAdd(&st.count, 1);
                 if (slot < k)  // exactly k are selected; the test only guards the bound
                     out[slot] = cand_key<T>(val[m], first + pos[m]);
+                ++slot;
             }
     }
     // Arrival: the barrier orders every thread's candidate stores before thread

@@ -198,14 +198,15 @@ class Step:
 
     @staticmethod
     def _chain_inputs(c):
-        ts = [c.residual]
-        for k in ("x_attn", "gamma_attn", "q", "k", "x_mlp", "gamma_mlp", "gate", "up"):
-            ts += c.inp[k]
-        return ts
+        """A decode step's inputs: the residual and the flat buffer holding
+        every layer's inputs (one copy each)."""
+        return [c.residual, c.flat_in]
 
     @staticmethod
     def _chain_outputs(c):
-        return [c.residual] + c.y_attn + c.q_out + c.k_out + c.y_mlp + c.act
+        """A decode step's outputs: the residual and the flat buffer holding
+        every layer's outputs."""
+        return [c.residual, c.flat_out]
 
     # operators with the most output first: their copies back overlap the
     # later operators' copies in, and the pipeline ends on small copies

@@ -61,8 +61,10 @@ METRIC = "fused-op HBM GB/s & % of B200 peak; µs per decode step (5 candidates)
 UNIT = "GB/s"
 WORKLOAD = ("hot-path pass: RMSNorm f32 64x1024; add+RMSNorm bf16 4096x2048; SwiGLU bf16 "
             "8192x6144; M-RoPE bf16 4096 tok x (16q+8k) heads x 128, sections [24,20,20]; "
-            "28-layer decode step at batch 5 and at batch 256; the whole pass one CUDA graph")
+            "28-layer decode step at batch 5 and at batch 256")
 FALLBACK_HBM_GBS = 6650.0
+L2_NOTE = ("inputs larger than L2: the step streams ~1 GB of distinct data (8x L2) and no "
+           "operator reuses another's data; no flush buffer")
 
 
 # ---------------------------------------------------------------------------
@@ -463,7 +465,8 @@ def run_reference(args) -> None:
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": None, "parallelism": "replicas x1",
-                   "sample": ostep.sample},
+                   "l2": L2_NOTE},
+        "method": {"sample": ostep.sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
                          "sample": ostep.sample + "; plain single-threaded C oracle, fp64",
                          "per_config_ms": {k: round(1e3 * v / len(times), 2)
@@ -722,16 +725,15 @@ def main() -> None:
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": None, "parallelism": f"replicas x{world}",
-                   "pdl": not args.no_pdl,
+                   "l2": L2_NOTE},
+        "method": {"pdl": not args.no_pdl,
                    "timing": "each step is one replay of a CUDA graph of all 228 launches "
                              "(4 prefill, 112 + 112 decode), CUDA events around the replay; "
                              "ops[*].us = the step time split in proportion to what each "
                              "operator adds to the step graph's time (us_marginal: the "
                              "graph's time minus that of the graph without the operator)",
                    "step_split_scale": round(scale, 4),
-                   "step_us_in_marginal_runs": round(marg_full, 2),
-                   "l2": "inputs larger than L2: the step streams ~1 GB of distinct data "
-                         "(8x L2) and no operator reuses another's data; no flush buffer"},
+                   "step_us_in_marginal_runs": round(marg_full, 2)},
         "us_per_decode_step": {"batch5": ops_report["decode_b5"]["us"],
                                "batch256": ops_report["decode_b256"]["us"]},
         "ops": ops_report,

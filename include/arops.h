@@ -211,12 +211,20 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  *              KiB); every call leaves them zero again, for any later shape.
  *              The rest holds candidates and needs no initialisation.  Two
  *              calls in flight at once must not share one workspace.
- * One kernel is enqueued on `stream`: each 4096-logit slice's CTA writes its
- * top_k candidates, and the last CTA of a row to finish (counted on the row's
- * arrival counter) merges them and takes the decision; no CTA waits for
- * another.  A counter found non-zero at the start of a call (a workspace that
- * was not cleared) sets AROPS_DEVICE_ERR_WORKSPACE in the device error word,
- * and that row's outputs are then undefined.
+ * One kernel is enqueued on `stream`.  When every row's cluster fits on the
+ * device at once (a few rows: 7 of 151936 logits on a B200) and the cluster
+ * kernel is enabled (arops_set_topk_cluster, the default), it is the
+ * single-pass cluster kernel: a thread-block cluster of up to 16 CTAs per row
+ * holds the row's logits in registers, the CTAs select the row's top_k
+ * together through each other's shared memory, and the cluster's first CTA
+ * ranks them and takes the decision; it does not touch the workspace.
+ * Otherwise it is the slice kernel: each 4096-logit
+ * slice's CTA writes its top_k candidates to the workspace, and the last CTA
+ * of a row to finish (counted on the row's arrival counter) merges them and
+ * takes the decision; no CTA waits for another.  The two give identical
+ * results.  A counter found non-zero at the start of a slice-kernel call (a
+ * workspace that was not cleared) sets AROPS_DEVICE_ERR_WORKSPACE in the
+ * device error word, and that row's outputs are then undefined.
  */
 #define AROPS_DEVICE_ERR_WORKSPACE 4u
 AROPS_API arops_status arops_topk_sample_workspace(int64_t rows, int64_t vocab, int32_t top_k,
@@ -309,6 +317,15 @@ AROPS_API int arops_set_pdl(int enable);
 AROPS_API int arops_set_streaming(int enable);
 
 /*
+ * Top-k sampling kernel selection (process-wide).  Enabled (the default),
+ * arops_topk_sample and arops_topk_sample_noalloc take the single-pass cluster
+ * kernel for calls whose rows' clusters the device holds at once; disabled,
+ * always the slice kernel.  Both give identical results; the control exists
+ * for measurement and testing.  Returns the old setting.
+ */
+AROPS_API int arops_set_topk_cluster(int enable);
+
+/*
  * Device-side error bits of the current device, OR-ed by kernels that abandon
  * part of their work: AROPS_DEVICE_ERR_TIMEOUT means a bulk copy into shared
  * memory did not complete within a second (the kernel's outputs are then
@@ -344,7 +361,7 @@ AROPS_API const char* arops_last_error(void);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 AROPS_API int arops_version(void);
 
-#define AROPS_VERSION 20000
+#define AROPS_VERSION 20100
 
 #ifdef __cplusplus
 }

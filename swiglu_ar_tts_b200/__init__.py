@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "rmsnorm", "add_rmsnorm", "layernorm", "add_layernorm", "mrope_qk", "mrope_kv_append",
     "swiglu", "set_pdl",
-    "set_streaming", "topk_sample", "topk_sample_workspace", "topk_sample_prepare",
+    "set_streaming", "set_topk_cluster", "topk_sample", "topk_sample_workspace", "topk_sample_prepare",
     "device_errors", "launch_count",
     "lib", "lib_path", "ArOpsError", "DTYPES",
 ]
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.arops_set_pdl.restype = ctypes.c_int
         L.arops_set_streaming.argtypes = [ctypes.c_int]
         L.arops_set_streaming.restype = ctypes.c_int
+        L.arops_set_topk_cluster.argtypes = [ctypes.c_int]
+        L.arops_set_topk_cluster.restype = ctypes.c_int
         L.arops_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         L.arops_device_errors.restype = ctypes.c_int
         L.arops_launch_count.restype = ctypes.c_uint64
@@ -362,6 +364,13 @@ def set_streaming(enable: bool) -> bool:
     """Choose the shared-memory streaming kernels or the register kernels (the
     default); returns the old setting.  Both give results within tolerance."""
     return bool(lib().arops_set_streaming(1 if enable else 0))
+
+
+def set_topk_cluster(enable: bool) -> bool:
+    """Choose the single-pass cluster kernel for top-k sampling (the default,
+    where the device can hold its clusters) or the slice kernel; returns the
+    old setting.  Both give identical results."""
+    return bool(lib().arops_set_topk_cluster(1 if enable else 0))
 
 
 def device_errors(clear: bool = True) -> int:

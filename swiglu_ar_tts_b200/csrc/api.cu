@@ -15,6 +15,7 @@ namespace {
 thread_local char g_last_error[512] = "";
 std::atomic<int> g_pdl{0};
 std::atomic<int> g_streaming{0};
+std::atomic<int> g_topk_cluster{1};
 std::atomic<uint64_t> g_launches{0};
 
 constexpr int kMaxDevices = 64;
@@ -89,6 +90,11 @@ bool pdl_enabled()
 bool streaming_enabled()
 {
     return g_streaming.load(std::memory_order_relaxed) != 0;
+}
+
+bool topk_cluster_enabled()
+{
+    return g_topk_cluster.load(std::memory_order_relaxed) != 0;
 }
 
 void count_launch()
@@ -435,6 +441,11 @@ AROPS_API int arops_set_pdl(int enable)
 AROPS_API int arops_set_streaming(int enable)
 {
     return g_streaming.exchange(enable ? 1 : 0);
+}
+
+AROPS_API int arops_set_topk_cluster(int enable)
+{
+    return g_topk_cluster.exchange(enable ? 1 : 0);
 }
 
 AROPS_API uint64_t arops_launch_count(void)

@@ -8,7 +8,11 @@
 // rank): Gumbel-max sampling from softmax(logits / T) restricted to the top k.
 // prob_out is that token's probability under the same restricted softmax.
 //
-// One kernel, grid (slices, rows).  A CTA turns its 4096-logit slice into
+// Two kernels give the same results.  The cluster kernel (second half of this
+// file) runs a row per thread-block cluster with the selection exchanged
+// through distributed shared memory; it is taken while every row's cluster is
+// resident at once (a few rows).  The slice kernel serves every other call:
+// grid (slices, rows).  A CTA turns its 4096-logit slice into
 // keys (order-preserving bits of the value, then the inverted position, so
 // that larger keys are larger logits and, among equal logits, lower indices:
 // every key is distinct; 32 bits for bf16, 48 for fp32), finds its k largest
@@ -351,6 +355,64 @@ struct LocalKey {
 
 constexpr int kMergePerThread = kMaxSlices * kMaxTopK / kMergeThreads;  // 8
 
+// The sampling decision, taken by warp 0 of the calling CTA (every thread
+// may call it; the others return at once).  ranked[0..k) holds the row's k
+// candidate keys from the largest down; gdraw holds the Gumbel draws of ranks
+// lane and lane + 32 in warp 0.
+template <typename T>
+__device__ __forceinline__ void sample_decision(const uint64_t* ranked, int k,
+                                                const float (&gdraw)[2], float temperature,
+                                                int32_t* token_out, float* prob_out)
+{
+    // Two ranks per lane (k <= 64).  Per rank j:
+    // e_j = exp((l_j - l_0) / T) and the score fl(fl(l_j / T) + g_j), two
+    // correctly rounded operations.  The token is the first rank with the
+    // largest score, as a scan in rank order that moves on only to a strictly
+    // larger score finds it: NaN scores after rank 0 never win, a NaN at rank 0
+    // always does.
+    if (threadIdx.x >= 32)
+        return;
+    const int lane = threadIdx.x;
+    const float l0 = cand_value<T>(ranked[0]);
+    float ej[2], bs = 0.f, z = 0.f;
+    int bj = k;  // none yet
+    float s0 = 0.f;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = lane + 32 * r;
+        ej[r] = 0.f;
+        if (j < k) {
+            const float l = cand_value<T>(ranked[j]);
+            ej[r] = expf((l - l0) / temperature);
+            const float sc = __fadd_rn(__fdiv_rn(l, temperature), gdraw[r]);
+            if (j == 0)
+                s0 = sc;
+            if (!isnan(sc) && (bj == k || sc > bs)) {
+                bs = sc;
+                bj = j;
+            }
+            z += ej[r];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
+        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, o);
+        if (oj < k && (bj == k || os > bs || (os == bs && oj < bj))) {
+            bs = os;
+            bj = oj;
+        }
+        z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+    }
+    s0 = __shfl_sync(0xFFFFFFFFu, s0, 0);
+    const int best = isnan(s0) ? 0 : bj;
+    const float eb = __shfl_sync(0xFFFFFFFFu, best < 32 ? ej[0] : ej[1], best & 31);
+    if (lane == 0) {
+        *token_out = (int32_t)cand_index(ranked[best]);
+        *prob_out = eb / z;
+    }
+}
+
 // The row's merge and decision, run by the CTA that arrived last: the k
 // largest of the slices' n = slices * k candidate keys (read through L2: other
 // CTAs wrote them), ranked by counting, then the sampling decision.
@@ -403,53 +465,7 @@ __device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float
     }
     __syncthreads();
 
-    // Warp 0 takes the decision, two ranks per lane (k <= 64).  Per rank j:
-    // e_j = exp((l_j - l_0) / T) and the score fl(fl(l_j / T) + g_j), two
-    // correctly rounded operations.  The token is the first rank with the
-    // largest score, as a scan in rank order that moves on only to a strictly
-    // larger score finds it: NaN scores after rank 0 never win, a NaN at rank 0
-    // always does.
-    if (threadIdx.x >= 32)
-        return;
-    const int lane = threadIdx.x;
-    const float l0 = cand_value<T>(ranked[0]);
-    float ej[2], bs = 0.f, z = 0.f;
-    int bj = k;  // none yet
-    float s0 = 0.f;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int j = lane + 32 * r;
-        ej[r] = 0.f;
-        if (j < k) {
-            const float l = cand_value<T>(ranked[j]);
-            ej[r] = expf((l - l0) / temperature);
-            const float sc = __fadd_rn(__fdiv_rn(l, temperature), gdraw[r]);
-            if (j == 0)
-                s0 = sc;
-            if (!isnan(sc) && (bj == k || sc > bs)) {
-                bs = sc;
-                bj = j;
-            }
-            z += ej[r];
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
-        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, o);
-        if (oj < k && (bj == k || os > bs || (os == bs && oj < bj))) {
-            bs = os;
-            bj = oj;
-        }
-        z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
-    }
-    s0 = __shfl_sync(0xFFFFFFFFu, s0, 0);
-    const int best = isnan(s0) ? 0 : bj;
-    const float eb = __shfl_sync(0xFFFFFFFFu, best < 32 ? ej[0] : ej[1], best & 31);
-    if (lane == 0) {
-        *token_out = (int32_t)cand_index(ranked[best]);
-        *prob_out = eb / z;
-    }
+    sample_decision<T>(ranked, k, gdraw, temperature, token_out, prob_out);
 }
 
 // VEC: rows start on 16-byte boundaries, so a thread loads its 16 logits as
@@ -567,6 +583,480 @@ topk_sample_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slice
                         prob_out + row, st, sel, ranked);
 }
 
+// ---------------------------------------------------------------------------
+// Single-pass variant on a thread-block cluster: one cluster of `ncta` CTAs
+// (up to 16) per row, each CTA holding a contiguous chunk of the row's logits
+// in registers.  The select runs over the whole row at once: every CTA first
+// drops the keys below a floor that at least k of its keys reach (so none of
+// the dropped ones can be among the row's k largest), histograms the rest in
+// its shared memory, the cluster barrier publishes
+// the histograms, and every CTA sums the cluster's from its peers' shared
+// memory (distributed shared memory), so all CTAs reach the same decision
+// without any exchange through global memory.  Once the boundary bin holds at
+// most kSmallBin keys, every CTA pushes its keys from that bin up (at most
+// k - 1 + kSmallBin in all, the row's k largest among them) into the shared
+// memory of the cluster's first CTA, which ranks them by counting and takes
+// the sampling decision.  Two cluster barriers in the common case; a row whose
+// boundary bin is larger (ties, flat rows) takes further 8-bit digit rounds of
+// one barrier each.  Nothing is read or written outside the logits, the draws
+// and the outputs.
+// ---------------------------------------------------------------------------
+constexpr int kClThreads = 512;
+constexpr int kClWarps = kClThreads / 32;
+constexpr int kClMaxCtas = 16;                       // non-portable cluster size
+constexpr int kClPushSlots = 128;                   // >= kMaxTopK - 1 + kSmallBin
+static_assert(kMaxTopK - 1 + kSmallBin <= kClPushSlots, "room for every pushed key");
+static_assert(4 * kClPushSlots <= kClThreads, "four threads rank each pushed key");
+static_assert(kClWarps * 4 >= kMaxTopK, "at most four keys a warp make the floor");
+
+// Largest value over the warp.
+template <typename K>
+__device__ __forceinline__ K warp_max(K v)
+{
+    if constexpr (sizeof(K) == 4) {
+        return __reduce_max_sync(0xFFFFFFFFu, v);
+    } else {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const K u = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            v = u > v ? u : v;
+        }
+        return v;
+    }
+}
+
+// Distributed shared memory: the address of this CTA's shared variable `p` in
+// the shared memory of cluster CTA `rank`, and accesses through it.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank)
+{
+    const uint32_t local = (uint32_t)__cvta_generic_to_shared(p);
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    return remote;
+}
+
+// (No memory clobber: the cluster barriers order these loads; without it the
+// loads of one thread are issued together instead of one round trip each.)
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, uint64_t v)
+{
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_cluster_u32(uint32_t addr, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "r"(addr), "r"(v)
+                 : "memory");
+    return old;
+}
+
+// Barrier of all threads of the cluster: shared-memory writes before it (this
+// CTA's and remote ones) are visible to every thread of the cluster after it.
+__device__ __forceinline__ void cluster_barrier()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+struct ClusterSelect {
+    uint32_t hist[2][256];  // this CTA's histogram of a round (alternating buffers)
+    uint32_t ghist[256];    // the cluster's, summed from every CTA's
+    uint32_t warp_top[32];  // per-warp counts of the push
+    uint64_t warp_key[32];  // per-warp largest key
+    uint64_t warp_floor[32];  // per-warp r-th largest lane maximum
+    uint32_t cta_top;       // this CTA's largest leading 16 bits
+    uint64_t tau;           // bits of the boundary bin fixed so far (global-key layout)
+    int shift;              // the bin is the keys with (key >> shift) == (tau >> shift)
+    int need;               // keys still to take from the bin
+    int binsz;              // keys in the bin, over the whole row
+    int window;             // the first round found the bin
+    int64_t first;          // the chunk's first vocabulary index
+    uint32_t push_base;
+    // the first CTA's: keys pushed by the cluster, their count, their ranking
+    uint32_t push_count;
+    uint64_t cand[kClPushSlots];
+    uint64_t ranked[kMaxTopK];
+};
+
+// Row-wide key (cand_key's layout) of a CTA-local key of the chunk at `first`.
+template <typename T>
+__device__ __forceinline__ uint64_t row_key(typename LocalKey<T>::type lk, int64_t first)
+{
+    const uint64_t vbits = (uint64_t)(lk >> 16);
+    const uint32_t p = 0xFFFFu - (uint32_t)(lk & 0xFFFFu);
+    return (vbits << kIndexBits) |
+           (uint64_t)((1u << kIndexBits) - 1u - (uint32_t)(first + (int64_t)p));
+}
+
+// The smallest local key (as a 64-bit number) of the chunk at `first` whose
+// row key is at least `t`.  Within a chunk the map from local to row keys
+// keeps the order (the row key's index bits are the local ones plus
+// 2^24 - 2^16 - first), so `local >= threshold` tests `row key >= t` without
+// forming the row key.
+template <typename T>
+__device__ __forceinline__ uint64_t local_threshold(uint64_t t, int64_t first)
+{
+    const uint64_t vt = t >> kIndexBits;
+    const int64_t it = (int64_t)(t & ((1ull << kIndexBits) - 1ull));
+    const int64_t below = it - ((int64_t)(1 << kIndexBits) - 0x10000 - first);
+    if (below <= 0)
+        return vt << 16;
+    if (below > 0xFFFF)
+        return (vt + 1) << 16;
+    return (vt << 16) | (uint64_t)below;
+}
+
+// Warp 0, first round: the bin of the k-th largest key in the cluster's
+// histogram of distances below the row's largest leading 16 bits `ctop`.
+// Leaves window = 0 when the 256 bins hold fewer than k keys.
+__device__ __forceinline__ void cluster_window_scan(ClusterSelect& st, uint32_t ctop, int k, int gs)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t local = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+        local += st.ghist[8 * lane + b];
+    uint32_t upto = local;  // keys in this lane's bins and every nearer bin
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, upto, o);
+        if (lane >= o)
+            upto += v;
+    }
+    const uint32_t nearer = upto - local;
+    if (nearer < (uint32_t)k && upto >= (uint32_t)k) {
+        uint32_t run = nearer;
+        for (int b = 0; b < 8; ++b) {
+            const uint32_t h = st.ghist[8 * lane + b];
+            if (run + h >= (uint32_t)k) {
+                st.tau = (uint64_t)(ctop - (uint32_t)(8 * lane + b)) << gs;
+                st.shift = gs;
+                st.need = k - (int)run;
+                st.binsz = (int)h;
+                st.window = 1;
+                break;
+            }
+            run += h;
+        }
+    }
+}
+
+// Warp 0, a digit round: the bin of the need-th largest key among the keys of
+// the current bin, by the 8-bit digit at `shift`.
+__device__ __forceinline__ void cluster_digit_scan(ClusterSelect& st, int shift)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t local = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+        local += st.ghist[8 * lane + b];
+    uint32_t above = local;  // keys in this lane's bins and every higher bin
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, above, o);
+        if (lane + o < 32)
+            above += v;
+    }
+    const uint32_t higher = above - local;
+    const int need = st.need;
+    if (higher < (uint32_t)need && above >= (uint32_t)need) {
+        uint32_t run = higher;
+        for (int b = 7; b >= 0; --b) {
+            const uint32_t h = st.ghist[8 * lane + b];
+            if (run + h >= (uint32_t)need) {
+                st.tau |= (uint64_t)(8 * lane + b) << shift;
+                st.shift = shift;
+                st.need = need - (int)run;
+                st.binsz = (int)h;
+                break;
+            }
+            run += h;
+        }
+    }
+}
+
+// Sums this round's histogram buffer `h` over the cluster's CTAs into ghist
+// (threads 0..255; `delta` shifts each CTA's bins, zero after the first round).
+template <bool SHIFTED>
+__device__ __forceinline__ uint32_t cluster_hist_sum(const uint32_t* h, uint32_t ncta, uint32_t tc,
+                                                     uint32_t ctop)
+{
+    const uint32_t bin = threadIdx.x;
+    // all remote loads first, then the sum: one round trip in all
+    uint32_t v[kClMaxCtas];
+#pragma unroll
+    for (uint32_t c = 0; c < (uint32_t)kClMaxCtas; ++c) {
+        uint32_t delta = 0;
+        if constexpr (SHIFTED)
+            delta = ctop - __shfl_sync(0xFFFFFFFFu, tc, c & 31u);
+        v[c] = (c < ncta && bin >= delta) ? ld_cluster_u32(cluster_addr(h + (bin - delta), c)) : 0u;
+    }
+    uint32_t tot = 0;
+#pragma unroll
+    for (int c = 0; c < kClMaxCtas; ++c)
+        tot += v[c];
+    return tot;
+}
+
+// Grid (ncta, rows), clusters of ncta CTAs along x; CTA c of a row holds the
+// row's logits [c * chunk, (c + 1) * chunk), M per thread (chunk <= 512 M).
+// VEC: the chunk starts on a 16-byte boundary and thread t loads the 16-byte
+// vectors at chunk positions (v * 512 + t) * E; otherwise one element at a time.
+template <typename T, bool VEC, int M>
+__global__ void __launch_bounds__(kClThreads, (sizeof(T) == 2 && M <= 16) ? 2 : 1)
+topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int k,
+                    const float* __restrict__ gumbel, float temperature,
+                    int32_t* __restrict__ token_out, float* __restrict__ prob_out)
+{
+    using K = typename LocalKey<T>::type;
+    constexpr int E = Vec<T>::N;
+    constexpr int VS = LocalKey<T>::BITS - 16;  // leading 16 bits of a local key
+    constexpr int GB = KeyBits<T>::V + kIndexBits;
+    constexpr int GS = GB - 16;                 // leading 16 bits of a row key
+    static_assert(!VEC || M % E == 0, "whole vectors per thread");
+    __shared__ ClusterSelect st;
+    const int tid = (int)threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const uint32_t crank = cluster_ctarank();
+    const uint32_t ncta = cluster_nctarank();
+    const int64_t row = blockIdx.y;
+    const int64_t first = (int64_t)crank * chunk;
+    const int n = (int)(vocab - first < (int64_t)chunk ? (vocab - first > 0 ? vocab - first : 0)
+                                                       : (int64_t)chunk);
+    const T* src = logits + row * vocab + first;
+    // the chunk into L2 while the previous kernel drains, one line per thread
+    {
+        constexpr int kPerLine = 128 / sizeof(T);
+        for (int i = tid * kPerLine; i < n; i += kClThreads * kPerLine)
+            prefetch_l2_line(src + i);
+    }
+    for (int i = tid; i < 256; i += kClThreads)
+        st.hist[0][i] = 0;
+    if (tid == 0) {
+        st.push_count = 0;
+        st.window = 0;
+        st.first = first;
+    }
+    pdl_wait();
+    pdl_allow_dependents();
+
+    float gdraw[2] = {0.f, 0.f};  // the first CTA's warp 0: draws of ranks lane, lane + 32
+    if (crank == 0 && tid < 32) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if (tid + 32 * r < k)
+                gdraw[r] = __ldg(gumbel + row * k + tid + 32 * r);
+    }
+    K key[M];  // local keys; 0 marks a position past the chunk (no real key is 0)
+    if constexpr (VEC) {
+#pragma unroll
+        for (int v = 0; v < M / E; ++v) {
+            const int p0 = (v * kClThreads + tid) * E;
+            float f[E];
+            if (p0 + E <= n) {
+                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(src + p0)), f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < E; ++j)
+                    f[j] = (p0 + j < n) ? load_elem(src + p0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < E; ++j)
+                key[v * E + j] = (p0 + j < n) ? (((K)KeyBits<T>::of(f[j]) << 16) |
+                                                 (K)(0xFFFFu - (uint32_t)(p0 + j)))
+                                              : K(0);
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int p = tid + m * kClThreads;
+            key[m] = (p < n) ? (((K)KeyBits<T>::of(load_elem(src + p)) << 16) |
+                                (K)(0xFFFFu - (uint32_t)p))
+                             : K(0);
+        }
+    }
+
+    // First round.  Each warp finds the r = ceil(k / 16) largest of its lanes'
+    // largest keys; the smallest of the 16 warps' r-th values, `floor`, has at
+    // least 16 r >= k of the CTA's keys at or above it, so the CTA's k-th
+    // largest key, and with it the row's, is not below it: keys under `floor`
+    // take no further part (typically all but a few dozen of the chunk's).
+    // Then the CTA's largest leading 16 bits and its histogram of the
+    // distances below them (the 256 nearest values) over the remaining keys.
+    K floor;
+    uint32_t top;
+    {
+        K cur = 0;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            cur = max(cur, key[m]);
+        const int r = (k + kClWarps - 1) / kClWarps;
+        K wtop = 0, rth = 0;
+        for (int i = 0; i < r; ++i) {
+            const K w = warp_max(cur);
+            if (i == 0)
+                wtop = w;
+            rth = w;
+            if (cur == w)  // keys are distinct: the lane that holds it drops out
+                cur = 0;
+        }
+        if (lane == 0) {
+            st.warp_key[warp] = (uint64_t)wtop;
+            st.warp_floor[warp] = (uint64_t)rth;
+        }
+        __syncthreads();
+        uint64_t t = 0, f = ~0ull;
+#pragma unroll
+        for (int w = 0; w < kClWarps; ++w) {
+            t = max(t, st.warp_key[w]);
+            f = min(f, st.warp_floor[w]);
+        }
+        floor = (K)f;
+        top = (uint32_t)(t >> VS);
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        if (key[m] && key[m] >= floor) {
+            const uint32_t d = top - (uint32_t)(key[m] >> VS);
+            if (d < 256u)
+                atomicAdd(&st.hist[0][d], 1u);
+        }
+    }
+    if (tid == 0)
+        st.cta_top = top;
+    cluster_barrier();  // every CTA's histogram and largest bits are published
+
+    // The row's histogram of distances below its largest leading bits: a CTA
+    // whose own largest bits are delta below the row's contributes its bin
+    // d - delta to bin d (its window covers the row's, from below).
+    if (tid < 256) {
+        const uint32_t tc =
+            (uint32_t)lane < ncta ? ld_cluster_u32(cluster_addr(&st.cta_top, lane)) : 0u;
+        const uint32_t ctop = __reduce_max_sync(0xFFFFFFFFu, tc);
+        st.ghist[tid] = cluster_hist_sum<true>(st.hist[0], ncta, tc, ctop);
+        if (tid == 0)
+            st.tau = ctop;  // kept for warp 0's scan below
+    }
+    __syncthreads();
+    if (warp == 0)
+        cluster_window_scan(st, (uint32_t)st.tau, k, GS);
+    __syncthreads();
+
+    // Digit rounds, only while the boundary bin is large and not taken whole
+    // (or when the 256 nearest values held fewer than k keys).
+    bool more = !st.window || (st.need != st.binsz && st.binsz > kSmallBin);
+    int shift = st.window ? GS - 8 : GB - 8;
+    __syncthreads();  // every thread has read the first round's outcome
+    if (tid == 0 && !st.window) {
+        st.tau = 0;
+        st.need = k;
+    }
+    for (int round = 1; more; ++round, shift -= 8) {
+        uint32_t* h = st.hist[round & 1];
+        for (int i = tid; i < 256; i += kClThreads)
+            h[i] = 0;
+        __syncthreads();
+        const uint64_t high_mask = ~0ull << (shift + 8);
+        const uint64_t prefix = st.tau & high_mask;
+        // re-read each round, so that the row keys are formed here and not
+        // kept in registers across rounds
+        const int64_t f = *reinterpret_cast<volatile int64_t*>(&st.first);
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (key[m] && key[m] >= floor) {
+                const uint64_t g = row_key<T>(key[m], f);
+                if ((g & high_mask) == prefix)
+                    atomicAdd(&h[(uint32_t)(g >> shift) & 255u], 1u);
+            }
+        }
+        cluster_barrier();
+        if (tid < 256)
+            st.ghist[tid] = cluster_hist_sum<false>(h, ncta, 0u, 0u);
+        __syncthreads();
+        if (warp == 0)
+            cluster_digit_scan(st, shift);
+        __syncthreads();
+        more = st.need != st.binsz && st.binsz > kSmallBin;
+    }
+
+    // Push: every key from the boundary bin up (k - need above the bin, binsz
+    // in it: at most k - 1 + kSmallBin, or exactly k when the bin is taken
+    // whole) into the first CTA's shared memory, at a range reserved with one
+    // remote atomic per CTA.
+    uint64_t lthr = local_threshold<T>(st.tau, first);  // the bin's low bits are 0
+    lthr = max(lthr, (uint64_t)floor);
+    int cnt = 0;
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+        cnt += key[m] && (uint64_t)key[m] >= lthr;
+    const int off = selected_offset(cnt, reinterpret_cast<int*>(st.warp_top));
+    if (tid == kClThreads - 1) {
+        const uint32_t total = (uint32_t)(off + cnt);
+        st.push_base = total ? atom_add_cluster_u32(cluster_addr(&st.push_count, 0), total) : 0u;
+    }
+    __syncthreads();
+    {
+        uint32_t slot = st.push_base + (uint32_t)off;
+        const uint32_t cand0 = cluster_addr(&st.cand[0], 0);
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            if (key[m] && (uint64_t)key[m] >= lthr) {
+                if (slot < (uint32_t)kClPushSlots)  // never reached: the bound only guards
+                    st_cluster_u64(cand0 + 8u * slot, row_key<T>(key[m], first));
+                ++slot;
+            }
+        }
+    }
+    cluster_barrier();  // every push has landed; no CTA touches another's memory after this
+    if (crank != 0)
+        return;
+
+    // The first CTA: rank the pushed keys by counting, keep the k largest in
+    // order, and take the sampling decision.
+    // Four threads (adjacent lanes) per key, each counting the larger keys in a
+    // quarter of the list.
+    const int nc = min((int)st.push_count, kClPushSlots);
+    {
+        const int i = tid >> 2;
+        const int q = tid & 3;
+        const uint64_t mine = i < nc ? st.cand[i] : 0ull;
+        int larger = 0;
+        for (int j = q; j < nc; j += 4)
+            larger += st.cand[j] > mine;
+        larger += __shfl_xor_sync(0xFFFFFFFFu, larger, 1);
+        larger += __shfl_xor_sync(0xFFFFFFFFu, larger, 2);
+        if (i < nc && q == 0 && larger < k)
+            st.ranked[larger] = mine;
+    }
+    __syncthreads();
+    sample_decision<T>(st.ranked, k, gdraw, temperature, token_out + row, prob_out + row);
+}
+
 }  // namespace
 
 int topk_slices(int64_t vocab)
@@ -589,15 +1079,166 @@ size_t topk_counter_bytes()
     return kCounterBytes;
 }
 
+namespace {
+
+// Shape of the single-pass launch for a vocabulary: the fewest CTAs per
+// cluster (a power of two up to 16) that hold the row at 8 logits a thread,
+// else 16 CTAs; each CTA's chunk is a multiple of 8 logits (so every chunk of
+// a 16-byte-aligned row starts on a 16-byte boundary) and M = logits a thread.
+struct ClusterShape {
+    int ncta;
+    int chunk;
+    int m;
+};
+
+ClusterShape cluster_shape(int64_t vocab)
+{
+    int ncta = 1;
+    while (ncta < kClMaxCtas && (int64_t)ncta * kClThreads * 8 < vocab)
+        ncta *= 2;
+    const int64_t chunk = (int64_t)round_up((uint32_t)ceil_div(vocab, ncta), 8u);
+    const int m = (int)round_up((uint32_t)ceil_div(chunk, kClThreads), 8u);
+    return {ncta, (int)chunk, m};
+}
+
+// Clusters of `ncta` CTAs of `Kernel` that the current device holds at once
+// (0 if it cannot run them; above 8 CTAs it first allows the non-portable
+// cluster size on the kernel).  Looked up once per device and cluster size.
+template <auto Kernel>
+int cluster_capacity(int ncta)
+{
+    constexpr int kMaxDevices = 64;
+    constexpr int kSizes = 5;  // 1, 2, 4, 8, 16 CTAs
+    static std::atomic<int> cache[kMaxDevices][kSizes];  // capacity + 1; 0 = not looked up
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 0;
+    int slot = 0;
+    while ((1 << slot) < ncta && slot < kSizes - 1)
+        ++slot;
+    int v = cache[dev][slot].load(std::memory_order_relaxed);
+    if (v == 0) {
+        int clusters = 0;
+        if (ncta <= 8 ||
+            cudaFuncSetAttribute(Kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)ncta, 1);
+            cfg.blockDim = dim3(kClThreads);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)ncta;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&clusters, Kernel, &cfg) != cudaSuccess)
+                clusters = 0;
+        }
+        (void)cudaGetLastError();  // a refused query leaves no sticky error behind
+        v = clusters + 1;
+        cache[dev][slot].store(v, std::memory_order_relaxed);
+    }
+    return v - 1;
+}
+
+template <typename T, bool VEC, int M>
+cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* token_out,
+                             float* prob_out, int64_t rows, int64_t vocab, int k,
+                             float temperature, const ClusterShape& cs, cudaStream_t stream,
+                             bool* launched)
+{
+    constexpr auto kernel = topk_cluster_kernel<T, VEC, M>;
+    *launched = false;
+    // Only while every row's cluster is resident at once: beyond that the
+    // clusters run in waves and the slice kernel (many small CTAs) is faster
+    // (5 rows of 151936 logits: 11.2 against 12.3 us a launch back to back on
+    // B200; 8 rows: 18.4 against 14.7).
+    if (rows > cluster_capacity<kernel>(cs.ncta))
+        return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs.ncta, (unsigned)rows);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs.ncta;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (pdl_enabled()) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
+    }
+    *launched = true;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, cs.chunk, k, gumbel,
+                                               temperature, token_out, prob_out);
+    if (err == cudaSuccess)
+        count_launch();
+    return err;
+}
+
+template <typename T, bool VEC>
+cudaError_t launch_cluster_m(const T* logits, const float* gumbel, int32_t* token_out,
+                             float* prob_out, int64_t rows, int64_t vocab, int k,
+                             float temperature, const ClusterShape& cs, cudaStream_t stream,
+                             bool* launched)
+{
+    switch (cs.m) {
+    case 8:
+        return launch_cluster_t<T, VEC, 8>(logits, gumbel, token_out, prob_out, rows, vocab, k,
+                                           temperature, cs, stream, launched);
+    case 16:
+        return launch_cluster_t<T, VEC, 16>(logits, gumbel, token_out, prob_out, rows, vocab, k,
+                                            temperature, cs, stream, launched);
+    case 24:
+        return launch_cluster_t<T, VEC, 24>(logits, gumbel, token_out, prob_out, rows, vocab, k,
+                                            temperature, cs, stream, launched);
+    case 32:
+        return launch_cluster_t<T, VEC, 32>(logits, gumbel, token_out, prob_out, rows, vocab, k,
+                                            temperature, cs, stream, launched);
+    default:
+        *launched = false;
+        return cudaSuccess;
+    }
+}
+
+}  // namespace
+
 cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
                                float* prob_out, int64_t rows, int64_t vocab, int k,
                                float temperature, arops_dtype dtype, void* workspace,
                                cudaStream_t stream)
 {
-    const int slices = topk_slices(vocab);
-    const dim3 grid((unsigned)slices, (unsigned)rows);
     const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
     const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
+    if (topk_cluster_enabled()) {
+        const ClusterShape cs = cluster_shape(vocab);
+        bool launched = false;
+        cudaError_t err;
+        if (dtype == AROPS_BF16) {
+            const auto* lg = static_cast<const __nv_bfloat16*>(logits);
+            err = vec ? launch_cluster_m<__nv_bfloat16, true>(lg, gumbel, token_out, prob_out, rows,
+                                                              vocab, k, temperature, cs, stream,
+                                                              &launched)
+                      : launch_cluster_m<__nv_bfloat16, false>(lg, gumbel, token_out, prob_out,
+                                                               rows, vocab, k, temperature, cs,
+                                                               stream, &launched);
+        } else {
+            const auto* lg = static_cast<const float*>(logits);
+            err = vec ? launch_cluster_m<float, true>(lg, gumbel, token_out, prob_out, rows, vocab,
+                                                      k, temperature, cs, stream, &launched)
+                      : launch_cluster_m<float, false>(lg, gumbel, token_out, prob_out, rows, vocab,
+                                                       k, temperature, cs, stream, &launched);
+        }
+        if (launched)
+            return err;
+        // more rows than resident clusters, or no such clusters here: the slice kernel
+    }
+    const int slices = topk_slices(vocab);
+    const dim3 grid((unsigned)slices, (unsigned)rows);
     unsigned* counters = static_cast<unsigned*>(workspace);
     uint64_t* work = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(workspace) +
                                                  kCounterBytes);

@@ -25,7 +25,7 @@ import statistics
 import torch
 
 from . import (add_layernorm, add_rmsnorm, layernorm, mrope_qk, rmsnorm, set_pdl, set_streaming,
-               mrope_kv_append, swiglu, topk_sample, topk_sample_prepare,
+               set_topk_cluster, mrope_kv_append, swiglu, topk_sample, topk_sample_prepare,
                topk_sample_workspace)
 from . import inputs as I
 from .chain import DecodeChain
@@ -179,6 +179,8 @@ def main() -> None:
                     help="shared-memory streaming kernels instead of the default register kernels")
     ap.add_argument("--no-chain-pdl", action="store_true",
                     help="decode steps without programmatic dependent launch")
+    ap.add_argument("--topk-slice", action="store_true",
+                    help="top-k sampling on the slice kernel instead of the cluster kernel")
     ap.add_argument("--json", action="store_true")
     a = ap.parse_args()
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -186,6 +188,7 @@ def main() -> None:
     CHAIN_PDL = not a.no_chain_pdl
     set_pdl(a.pdl)
     set_streaming(a.streaming)
+    set_topk_cluster(not a.topk_slice)
     for op in (OPS if a.op == "all" else (a.op,)):
         fns, nbytes, desc = make_rotation(op, a.rows, dev, a.copies)
         us = time_op(fns, a.iters)

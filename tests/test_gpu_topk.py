@@ -1,6 +1,7 @@
 """Fused softmax + top-k sampling on the GPU against the oracle: the sampled
 token bit for bit (the decision is taken in fp32 on both sides), its
-probability within the fp32 bound."""
+probability within the fp32 bound.  Both kernels are run: the single-pass
+cluster kernel (the default) and the slice kernel."""
 import numpy as np
 import pytest
 import torch
@@ -12,6 +13,20 @@ from gpu_util import Guarded, dev
 from tolerance import to_f64
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["cluster", "slice"])
+def kernel(request):
+    old = ops.set_topk_cluster(request.param == "cluster")
+    yield request.param
+    ops.set_topk_cluster(old)
+
+
+@pytest.fixture
+def slice_kernel():
+    old = ops.set_topk_cluster(False)
+    yield
+    ops.set_topk_cluster(old)
 
 
 def _run(inp, k, temp):
@@ -30,18 +45,18 @@ def _check(inp, k, temp, what=""):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("vocab,k", [(1, 1), (63, 5), (4096, 50), (4097, 64), (3072, 1),
                                      (151936, 50), (262144, 64), (10000, 20)])
-def test_topk_sample_shapes(dtype, vocab, k):
+def test_topk_sample_shapes(dtype, vocab, k, kernel):
     inp = inputs.topk_inputs(5, vocab, k, dtype, seed=vocab + k)
     _check(inp, k, 0.8, f"{dtype} V={vocab} k={k}")
 
 
 @pytest.mark.parametrize("temp", [0.3, 1.0, 1.7])
-def test_topk_sample_temperatures_many_rows(temp):
+def test_topk_sample_temperatures_many_rows(temp, kernel):
     inp = inputs.topk_inputs(257, 20000, 40, "bf16", seed=int(temp * 10))
     _check(inp, 40, temp, f"T={temp}")
 
 
-def test_topk_sample_ties_go_to_lower_index():
+def test_topk_sample_ties_go_to_lower_index(kernel):
     """Coarse logits (multiples of 0.5) tie constantly; the candidates and ranks
     must follow (logit desc, index asc) exactly."""
     rng = np.random.default_rng(3)
@@ -55,7 +70,7 @@ def test_topk_sample_ties_go_to_lower_index():
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_topk_sample_flat_spread_and_outlier_rows(dtype):
+def test_topk_sample_flat_spread_and_outlier_rows(dtype, kernel):
     """Rows whose k largest values are not all near the largest one, and rows
     where one value repeats everywhere: constant logits (the k lowest indices
     win), three outliers far above N(0,1) noise (fewer than k values within
@@ -75,7 +90,7 @@ def test_topk_sample_flat_spread_and_outlier_rows(dtype):
     _check(inp, k, 1.0, f"flat/spread/outliers {dtype}")
 
 
-def test_topk_sample_winner_in_last_slice_and_greedy():
+def test_topk_sample_winner_in_last_slice_and_greedy(kernel):
     inp = inputs.topk_inputs(4, 151936, 8, "bf16", seed=9)
     lg = inp["logits"].clone()
     lg[0, -1] = 40.0
@@ -88,7 +103,7 @@ def test_topk_sample_winner_in_last_slice_and_greedy():
     _check(inp, 8, 1.0, "winners at slice edges")
 
 
-def test_topk_sample_distribution():
+def test_topk_sample_distribution(kernel):
     """Over 20,000 rows of one logit vector with fresh draws, the GPU's token
     frequencies match the top-k softmax (chi-square)."""
     rng = np.random.default_rng(11)
@@ -109,7 +124,7 @@ def test_topk_sample_distribution():
 COUNTER_BYTES = 1 << 18  # the workspace's arrival counters (one per row, up to 65535 rows)
 
 
-def test_topk_sample_workspace_is_exact_and_guarded():
+def test_topk_sample_workspace_is_exact_and_guarded(slice_kernel):
     rows, vocab, k = 5, 50000, 32
     need = ops.topk_sample_workspace(rows, vocab, k)
     assert need == COUNTER_BYTES + rows * ((vocab + 4095) // 4096) * k * 8
@@ -125,7 +140,7 @@ def test_topk_sample_workspace_is_exact_and_guarded():
     assert np.array_equal(tok.cpu().numpy(), t_ref)
 
 
-def test_topk_sample_one_workspace_for_many_shapes():
+def test_topk_sample_one_workspace_for_many_shapes(kernel):
     """The counters sit at a fixed place and every call leaves them at zero, so
     one prepared workspace serves calls of any shape in turn."""
     shapes = ((5, 151936, 50), (33, 70000, 64), (3, 4096, 7), (64, 151936, 50), (1, 100, 1))
@@ -140,7 +155,7 @@ def test_topk_sample_one_workspace_for_many_shapes():
     assert not w8[:COUNTER_BYTES].any()
 
 
-def test_topk_sample_flags_a_workspace_whose_counters_were_not_cleared():
+def test_topk_sample_flags_a_workspace_whose_counters_were_not_cleared(slice_kernel):
     """Counters left non-zero (a workspace never prepared) are reported in the
     device error word; the kernel still completes."""
     rows, vocab, k = 2, 10000, 8
@@ -152,8 +167,71 @@ def test_topk_sample_flags_a_workspace_whose_counters_were_not_cleared():
     assert ops.device_errors(clear=True) == 4  # AROPS_DEVICE_ERR_WORKSPACE
 
 
-def test_topk_sample_empty_rows():
+def test_topk_sample_empty_rows(kernel):
     lg = torch.empty(0, 100, dtype=torch.bfloat16, device="cuda")
     tok, prob = ops.topk_sample(lg, torch.empty(0, 4, device="cuda"), 4, 1.0)
     torch.cuda.synchronize()
     assert tok.numel() == 0
+
+
+# Cluster sizes 1 .. 16 and their edges (a CTA per 4096 logits up to 16 CTAs,
+# then up to 16384 logits a CTA), rows of 16-byte-aligned and unaligned starts.
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("vocab", [8, 4096, 4104, 8192, 8200, 16385, 32769, 65536, 65544,
+                                   131080, 196608, 262136])
+def test_topk_sample_cluster_sizes(dtype, vocab):
+    k = min(64, vocab)
+    inp = inputs.topk_inputs(3, vocab, k, dtype, seed=vocab)
+    _check(inp, k, 0.7, f"{dtype} V={vocab}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_topk_sample_unaligned_rows(kernel, dtype):
+    """Logits that start 2 or 4 bytes past a 16-byte boundary take the
+    element-by-element loads."""
+    rows, vocab = 4, 151936
+    inp = inputs.topk_inputs(rows, vocab, 50, "f32", seed=5)
+    lg = inp["logits"].to(dtype)
+    flat = torch.empty(rows * vocab + 1, dtype=dtype, device="cuda")
+    view = flat[1:].view(rows, vocab)  # contiguous rows, start one element past the boundary
+    view.copy_(dev(lg))
+    assert view.data_ptr() % 16 != 0
+    tok, prob = ops.topk_sample(view, dev(inp["gumbel"]), 50, 1.0)
+    t_ref, p_ref = oracle.get().topk_sample(lg, inp["gumbel"], 50, 1.0)
+    assert np.array_equal(tok.cpu().numpy(), t_ref)
+    np.testing.assert_allclose(to_f64(prob), p_ref, rtol=1e-5, atol=0)
+
+
+def test_topk_sample_cluster_kernel_leaves_the_workspace_alone():
+    """A few rows of up to 32768 logits always take the cluster kernel (clusters
+    of at most 8 CTAs, the portable size, dozens of which a B200 holds at
+    once); it reads no workspace byte and writes none."""
+    rows, vocab, k = 6, 32768, 64
+    w8 = torch.full((ops.topk_sample_workspace(rows, vocab, k),), 0x5A, dtype=torch.uint8,
+                    device="cuda")
+    inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=21)
+    tok, _ = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.0, workspace=w8)
+    torch.cuda.synchronize()
+    assert bool((w8 == 0x5A).all())
+    assert ops.device_errors(clear=True) == 0
+    t_ref, _ = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 1.0)
+    assert np.array_equal(tok.cpu().numpy(), t_ref)
+
+
+@pytest.mark.parametrize("rows", [1, 7, 64, 300])
+def test_topk_sample_kernels_agree_bit_for_bit(rows):
+    """The two kernels give the same tokens and the same probabilities, bit
+    for bit, over many rows."""
+    inp = inputs.topk_inputs(rows, 151936, 50, "bf16", seed=rows)
+    lg, g = dev(inp["logits"]), dev(inp["gumbel"])
+    out = {}
+    for mode in (True, False):
+        old = ops.set_topk_cluster(mode)
+        try:
+            tok, prob = ops.topk_sample(lg, g, 50, 0.8)
+            torch.cuda.synchronize()
+        finally:
+            ops.set_topk_cluster(old)
+        out[mode] = (tok.cpu(), prob.cpu())
+    assert torch.equal(out[True][0], out[False][0])
+    assert torch.equal(out[True][1], out[False][1])

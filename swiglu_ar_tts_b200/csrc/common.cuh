@@ -161,10 +161,6 @@ bool pdl_enabled();
 // Whether the shared-memory streaming (bulk-copy) kernels may be chosen.
 bool streaming_enabled();
 
-// Whether top-k sampling takes the single-pass cluster kernel (else the
-// slice-and-merge kernel).
-bool topk_cluster_enabled();
-
 // Counts one launch.
 void count_launch();
 

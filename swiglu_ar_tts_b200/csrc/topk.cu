@@ -35,6 +35,12 @@
 #include "common.cuh"
 
 namespace arops {
+// Whether calls may take the single-pass cluster kernel (api.cu,
+// arops_set_topk_cluster); otherwise always the slice kernel.
+bool topk_cluster_enabled();
+}  // namespace arops
+
+namespace arops {
 namespace {
 
 constexpr int kSlice = 4096;        // logits per slice

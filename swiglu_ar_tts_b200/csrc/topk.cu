@@ -1162,6 +1162,14 @@ cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* toke
     // B200; 8 rows: 18.4 against 14.7).
     if (rows > cluster_capacity<kernel>(cs.ncta))
         return cudaSuccess;
+    // The kernel attribute belongs to the current context, so it is set on
+    // every launch (a context created after the capacity lookup needs it too).
+    if (cs.ncta > 8) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess)
+            return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs.ncta, (unsigned)rows);
     cfg.blockDim = dim3(kClThreads);

@@ -235,3 +235,49 @@ def test_topk_sample_kernels_agree_bit_for_bit(rows):
         out[mode] = (tok.cpu(), prob.cpu())
     assert torch.equal(out[True][0], out[False][0])
     assert torch.equal(out[True][1], out[False][1])
+
+
+@pytest.mark.parametrize("rows", [5, 20])
+def test_topk_sample_in_a_graph_with_pdl(rows):
+    """Sampling captured in a CUDA graph behind another kernel, with
+    programmatic dependent launch (the end of a decode step): the cluster
+    kernel (5 rows) and the slice kernel (20 rows) replayed on new logits and
+    draws each time, every replay against the oracle."""
+    vocab, k = 151936, 50
+    lg = torch.empty(rows, vocab, dtype=torch.bfloat16, device="cuda")
+    g = torch.empty(rows, k, dtype=torch.float32, device="cuda")
+    x = torch.randn(rows, 2048, device="cuda").to(torch.bfloat16)
+    res = torch.randn(rows, 2048, device="cuda").to(torch.bfloat16)
+    gamma = torch.ones(2048, device="cuda").to(torch.bfloat16)
+    y = torch.empty_like(x)
+    tok = torch.empty(rows, dtype=torch.int32, device="cuda")
+    prob = torch.empty(rows, dtype=torch.float32, device="cuda")
+    ws = ops.topk_sample_prepare(torch.empty(ops.topk_sample_workspace(rows, vocab, k),
+                                             dtype=torch.uint8, device="cuda"))
+    old = ops.set_pdl(True)
+    try:
+        def step():
+            ops.add_rmsnorm(x, res, gamma, 1e-6, y=y)
+            ops.topk_sample(lg, g, k, 0.9, workspace=ws, token_out=tok, prob_out=prob)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            lg.zero_()
+            g.zero_()
+            step()  # warm-up outside the capture
+        torch.cuda.current_stream().wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for rep in range(3):
+            inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=100 + rep)
+            lg.copy_(inp["logits"])
+            g.copy_(inp["gumbel"])
+            graph.replay()
+            torch.cuda.synchronize()
+            t_ref, p_ref = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 0.9)
+            assert np.array_equal(tok.cpu().numpy(), t_ref), f"replay {rep}"
+            np.testing.assert_allclose(to_f64(prob), p_ref, rtol=1e-5, atol=0)
+        assert ops.device_errors(clear=True) == 0
+    finally:
+        ops.set_pdl(old)

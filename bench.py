@@ -55,7 +55,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from swiglu_ar_tts_b200.step import STEP_CONFIGS, Step, step_bytes  # noqa: E402
+from swiglu_ar_tts_b200.step import (STEP_CONFIGS, Step, run_e2e_pipelined,  # noqa: E402
+                                     step_bytes)
 
 METRIC = "fused-op HBM GB/s & % of B200 peak; µs per decode step (5 candidates)"
 UNIT = "GB/s"
@@ -488,7 +489,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-pdl", action="store_true", help="launch without programmatic dependent launch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -678,30 +679,37 @@ def main() -> None:
         run300[f"batch{batch}"] = {"graph_us_per_step": round(t["graph"], 2),
                                    "eager_us_per_step": round(t["eager"], 2)}
 
-    # end to end: pinned host buffers in and out, through the same public calls
+    # end to end: pinned host buffers in and out, through the same public
+    # calls, on two sets of device buffers so that one step's inputs cross
+    # PCIe while the previous step's results drain
     step.setup_e2e()
+    step_b = Step(device, pdl=not args.no_pdl, like=step)
+    step_b.setup_e2e(share=step)
+    sets = [step, step_b]
     torch.cuda.synchronize()
-    for _ in range(2):
-        step.run_e2e()
+    run_e2e_pipelined(sets, 2)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.e2e_steps):
-        step.run_e2e()
+    run_e2e_pipelined(sets, args.e2e_steps)
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    # the pipelined copies hand back exactly what the device holds
-    for g, _ in step.E2E_GROUPS:
-        for dst, src in step._e2e_out(g):
+    # the copies hand back exactly what the device holds (the last step's set)
+    last = sets[(args.e2e_steps - 1) % len(sets)]
+    for g, _ in last.E2E_GROUPS:
+        for dst, src in last._e2e_out(g):
             if not torch.equal(dst, src.cpu()):
                 raise SystemExit(f"e2e: host copy of {g} differs from the device result")
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
     e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
            "ms_per_step": e2e_ms, "h2d_bytes_per_step": step.h2d_bytes,
-           "d2h_bytes_per_step": step.d2h_bytes}
+           "d2h_bytes_per_step": step.d2h_bytes,
+           "pipeline": "two device buffer sets; each step's inputs cross while the previous "
+                       "step's results drain"}
+    del step_b, sets, last
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -44,7 +44,9 @@ class Step:
 
     OPS = ("rmsnorm", "add_rmsnorm", "swiglu", "mrope_qk", "decode_b5", "decode_b256")
 
-    def __init__(self, device: torch.device, pdl: bool = True):
+    def __init__(self, device: torch.device, pdl: bool = True, like: "Step | None" = None):
+        """``like``: take the host inputs of that step instead of drawing them
+        again (a second set of device buffers for the same workload)."""
         import swiglu_ar_tts_b200 as ops
 
         from . import inputs
@@ -52,7 +54,7 @@ class Step:
 
         self.ops = ops
         self.device = device
-        self.host = {
+        self.host = like.host if like is not None else {
             "rmsnorm": inputs.rmsnorm_inputs(64, 1024, "f32", 0),
             "add_rmsnorm": inputs.add_rmsnorm_inputs(4096, 2048, "bf16", 0),
             "swiglu": inputs.swiglu_inputs(8192, 6144, "bf16", 0),
@@ -70,8 +72,10 @@ class Step:
         self.mr = {k: v.to(d) for k, v in h["mrope_qk"].items()}
         self.mr["q_out"] = torch.empty_like(self.mr["q"])
         self.mr["k_out"] = torch.empty_like(self.mr["k"])
-        self.chain5 = DecodeChain(inputs.ChainShape(batch=5), device=d, pdl=pdl)
-        self.chain256 = DecodeChain(inputs.ChainShape(batch=256), device=d, seed=1000, pdl=pdl)
+        self.chain5 = DecodeChain(inputs.ChainShape(batch=5), device=d, pdl=pdl,
+                                  host_inputs=like.chain5.host_inputs if like else None)
+        self.chain256 = DecodeChain(inputs.ChainShape(batch=256), device=d, seed=1000, pdl=pdl,
+                                    host_inputs=like.chain256.host_inputs if like else None)
         self.chain5.capture()
         self.chain256.capture()
         self.pdl = pdl
@@ -169,7 +173,16 @@ class Step:
         self.decode_step_index += 1
 
     # -- end to end: host buffers in, results back to the host ------------------
-    def setup_e2e(self) -> None:
+    def setup_e2e(self, share: "Step | None" = None) -> None:
+        """Pinned host copies of every input and pinned host buffers for every
+        output, and the two copy streams.  With ``share`` (a step of the same
+        workload) this step becomes a second set of device buffers that uses
+        ``share``'s host buffers and copy streams (run_e2e_pipelined)."""
+        if share is not None:
+            self.h_in, self.h_out = share.h_in, share.h_out
+            self.h2d_bytes, self.d2h_bytes = share.h2d_bytes, share.d2h_bytes
+            self.s_h2d, self.s_d2h = share.s_h2d, share.s_d2h
+            return
         pin = lambda t: t.detach().cpu().pin_memory()  # noqa: E731
         self.h_in = {
             "rn": {k: pin(v) for k, v in self.host["rmsnorm"].items()},
@@ -231,18 +244,28 @@ class Step:
             srcs = dev[g]
         return list(zip(self.h_out[g], srcs))
 
-    def run_e2e(self) -> None:
+    def run_e2e(self, after: dict | None = None, serial: bool = True) -> dict:
         """Host->device copies of every input, the step, device->host copies of
         every output.  Three streams form a pipeline over the operators: the
         inputs of operator i+1 cross PCIe while operator i computes and the
         results of operator i-1 cross back (the two copy directions run at the
         same time).  Events order each operator's copy-in, compute and
-        copy-out; the step starts after the previous step's copy-outs."""
+        copy-out.  ``serial`` (one step at a time): the copies in wait for
+        everything enqueued before, and the compute stream ends waiting for
+        the copies back.  Otherwise (run_e2e_pipelined) the copies in of an
+        operator wait only for ``after[group]``, the end of the previous use
+        of this set's buffers of that operator.  Returns, per group, the event
+        that ends this step's use of them (its copy back, which followed its
+        compute)."""
         nb = dict(non_blocking=True)
         cur = torch.cuda.current_stream()
         h2d, d2h = self.s_h2d, self.s_d2h
-        h2d.wait_stream(cur)
+        if serial:
+            h2d.wait_stream(cur)
+        used = {}
         for g, name in self.E2E_GROUPS:
+            if after is not None:
+                h2d.wait_event(after[g])
             with torch.cuda.stream(h2d):
                 for dst, src in self._e2e_in(g):
                     dst.copy_(src, **nb)
@@ -257,8 +280,29 @@ class Step:
             with torch.cuda.stream(d2h):
                 for dst, src in self._e2e_out(g):
                     dst.copy_(src, **nb)
-        cur.wait_stream(d2h)
+            used[g] = torch.cuda.Event()
+            used[g].record(d2h)
+        if serial:
+            cur.wait_stream(d2h)
         self.decode_step_index += 1
+        return used
+
+
+def run_e2e_pipelined(sets: list, steps: int) -> None:
+    """``steps`` end-to-end steps on alternating sets of device buffers (Steps
+    of one workload sharing host buffers and copy streams; step i runs on set
+    i % len(sets)).  Each copy direction runs in order on its own stream, so
+    step i+1's inputs cross PCIe while step i computes and its results drain;
+    a set's buffers of an operator are refilled only after the previous step
+    on that set has computed and copied back that operator.  The compute
+    stream ends waiting for the last copy back."""
+    cur = torch.cuda.current_stream()
+    sets[0].s_h2d.wait_stream(cur)
+    after = [None] * len(sets)
+    for i in range(steps):
+        j = i % len(sets)
+        after[j] = sets[j].run_e2e(after[j], serial=False)
+    cur.wait_stream(sets[0].s_d2h)
 
 
 def main() -> None:

@@ -65,12 +65,23 @@ def test_noalloc_setup_call_launches_nothing():
     assert L.arops_launch_count() == before
 
 
+@pytest.mark.parametrize("kernel", ["slice", "cluster"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_noalloc_two_calls_match_workspace_entry_point_and_oracle(dtype):
+def test_noalloc_two_calls_match_workspace_entry_point_and_oracle(dtype, kernel):
     """Two calls in a row, each compared with the workspace entry point and with
-    the oracle.  The first call's logits sit 100 above the second's, so a key
-    the second call read from the first call's leftover scratch (instead of
-    writing it first) would outrank every real candidate and change the token."""
+    the oracle, on each kernel (these few-row calls take the cluster kernel by
+    default, which uses no scratch; the slice kernel is the one that does).
+    The first call's logits sit 100 above the second's, so a key the second
+    call read from the first call's leftover scratch (instead of writing it
+    first) would outrank every real candidate and change the token."""
+    old = ops.set_topk_cluster(kernel == "cluster")
+    try:
+        _two_calls(dtype)
+    finally:
+        ops.set_topk_cluster(old)
+
+
+def _two_calls(dtype):
     L = _lib()
     stream = torch.cuda.current_stream().cuda_stream
     orc = oracle.get()

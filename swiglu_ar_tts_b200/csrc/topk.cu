@@ -655,6 +655,19 @@ __device__ __forceinline__ void st_cluster_u64(uint32_t addr, uint64_t v)
     asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, const uint4& v)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_v2(uint32_t addr, uint32_t a, uint32_t b)
+{
+    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t atom_add_cluster_u32(uint32_t addr, uint32_t v)
 {
     uint32_t old;
@@ -689,18 +702,23 @@ __device__ __forceinline__ uint32_t cluster_nctarank()
 }
 
 struct ClusterSelect {
-    uint32_t hist[2][256];  // this CTA's histogram of a round (alternating buffers)
+    alignas(16) uint32_t hist[2][256];  // this CTA's histogram of a round (alternating buffers)
+    // first round: every CTA's histogram bins [0, span) as sent by that CTA,
+    // and its (largest leading bits, span)
+    alignas(16) uint32_t inbox[kClMaxCtas][256];
+    uint2 inbox_meta[kClMaxCtas];
     uint32_t ghist[256];    // the cluster's, summed from every CTA's
     uint32_t warp_top[32];  // per-warp counts of the push
     uint64_t warp_key[32];  // per-warp largest key
     uint64_t warp_floor[32];  // per-warp r-th largest lane maximum
-    uint32_t cta_top;       // this CTA's largest leading 16 bits
     uint64_t tau;           // bits of the boundary bin fixed so far (global-key layout)
     int shift;              // the bin is the keys with (key >> shift) == (tau >> shift)
     int need;               // keys still to take from the bin
     int binsz;              // keys in the bin, over the whole row
     int window;             // the first round found the bin
     int64_t first;          // the chunk's first vocabulary index
+    uint32_t ctop;          // the row's largest leading bits
+    uint32_t push_cnt[kClMaxCtas];  // keys each CTA pushes (when the first round decides)
     uint32_t push_base;
     // the first CTA's: keys pushed by the cluster, their count, their ranking
     uint32_t push_count;
@@ -805,22 +823,16 @@ __device__ __forceinline__ void cluster_digit_scan(ClusterSelect& st, int shift)
     }
 }
 
-// Sums this round's histogram buffer `h` over the cluster's CTAs into ghist
-// (threads 0..255; `delta` shifts each CTA's bins, zero after the first round).
-template <bool SHIFTED>
-__device__ __forceinline__ uint32_t cluster_hist_sum(const uint32_t* h, uint32_t ncta, uint32_t tc,
-                                                     uint32_t ctop)
+// Sum over the cluster's CTAs of bin threadIdx.x of a digit round's
+// histogram buffer `h` (read from every CTA's shared memory; threads 0..255).
+__device__ __forceinline__ uint32_t cluster_hist_sum(const uint32_t* h, uint32_t ncta)
 {
     const uint32_t bin = threadIdx.x;
     // all remote loads first, then the sum: one round trip in all
     uint32_t v[kClMaxCtas];
 #pragma unroll
-    for (uint32_t c = 0; c < (uint32_t)kClMaxCtas; ++c) {
-        uint32_t delta = 0;
-        if constexpr (SHIFTED)
-            delta = ctop - __shfl_sync(0xFFFFFFFFu, tc, c & 31u);
-        v[c] = (c < ncta && bin >= delta) ? ld_cluster_u32(cluster_addr(h + (bin - delta), c)) : 0u;
-    }
+    for (uint32_t c = 0; c < (uint32_t)kClMaxCtas; ++c)
+        v[c] = c < ncta ? ld_cluster_u32(cluster_addr(h + bin, c)) : 0u;
     uint32_t tot = 0;
 #pragma unroll
     for (int c = 0; c < kClMaxCtas; ++c)
@@ -953,20 +965,46 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
                 atomicAdd(&st.hist[0][d], 1u);
         }
     }
-    if (tid == 0)
-        st.cta_top = top;
-    cluster_barrier();  // every CTA's histogram and largest bits are published
+    // Send the histogram to every CTA of the cluster (its row `crank` of their
+    // inboxes) before the barrier, so that the sum after it reads only this
+    // CTA's own shared memory.  The keys that take part lie within `span` bins
+    // of the CTA's largest leading bits (the floor's are the lowest), so only
+    // those bins go out, four to a store: a few dozen for logit-like rows.
+    __syncthreads();  // the CTA's histogram is complete
+    {
+        const uint32_t flead = (uint32_t)(floor >> VS);
+        const uint32_t span = floor ? min(256u, top - flead + 1u) : 256u;
+        const uint32_t nv = (span + 3u) / 4u;
+        for (uint32_t i = tid; i < nv * ncta; i += kClThreads) {
+            const uint32_t c = i / nv;
+            const uint32_t v = i - c * nv;
+            st_cluster_v4(cluster_addr(&st.inbox[crank][4u * v], c),
+                          *reinterpret_cast<const uint4*>(&st.hist[0][4u * v]));
+        }
+        if ((uint32_t)tid < ncta)
+            st_cluster_v2(cluster_addr(&st.inbox_meta[crank], (uint32_t)tid), top, span);
+    }
+    cluster_barrier();  // every CTA's histogram has arrived everywhere
 
     // The row's histogram of distances below its largest leading bits: a CTA
     // whose own largest bits are delta below the row's contributes its bin
     // d - delta to bin d (its window covers the row's, from below).
     if (tid < 256) {
-        const uint32_t tc =
-            (uint32_t)lane < ncta ? ld_cluster_u32(cluster_addr(&st.cta_top, lane)) : 0u;
-        const uint32_t ctop = __reduce_max_sync(0xFFFFFFFFu, tc);
-        st.ghist[tid] = cluster_hist_sum<true>(st.hist[0], ncta, tc, ctop);
-        if (tid == 0)
+        const uint2 meta = (uint32_t)lane < ncta ? st.inbox_meta[lane] : make_uint2(0u, 0u);
+        const uint32_t ctop = __reduce_max_sync(0xFFFFFFFFu, meta.x);
+        uint32_t tot = 0;
+#pragma unroll
+        for (uint32_t c = 0; c < (uint32_t)kClMaxCtas; ++c) {
+            const uint32_t delta = ctop - __shfl_sync(0xFFFFFFFFu, meta.x, c);
+            const uint32_t span = __shfl_sync(0xFFFFFFFFu, meta.y, c);
+            if (c < ncta && (uint32_t)tid >= delta && (uint32_t)tid - delta < span)
+                tot += st.inbox[c][tid - delta];
+        }
+        st.ghist[tid] = tot;
+        if (tid == 0) {
             st.tau = ctop;  // kept for warp 0's scan below
+            st.ctop = ctop;
+        }
     }
     __syncthreads();
     if (warp == 0)
@@ -976,6 +1014,7 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
     // Digit rounds, only while the boundary bin is large and not taken whole
     // (or when the 256 nearest values held fewer than k keys).
     bool more = !st.window || (st.need != st.binsz && st.binsz > kSmallBin);
+    const bool rounds = more;
     int shift = st.window ? GS - 8 : GB - 8;
     __syncthreads();  // every thread has read the first round's outcome
     if (tid == 0 && !st.window) {
@@ -1002,7 +1041,7 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
         }
         cluster_barrier();
         if (tid < 256)
-            st.ghist[tid] = cluster_hist_sum<false>(h, ncta, 0u, 0u);
+            st.ghist[tid] = cluster_hist_sum(h, ncta);
         __syncthreads();
         if (warp == 0)
             cluster_digit_scan(st, shift);
@@ -1012,22 +1051,69 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
 
     // Push: every key from the boundary bin up (k - need above the bin, binsz
     // in it: at most k - 1 + kSmallBin, or exactly k when the bin is taken
-    // whole) into the first CTA's shared memory, at a range reserved with one
-    // remote atomic per CTA.
+    // whole) into the first CTA's shared memory, CTA by CTA.  When the first
+    // round decided, every CTA knows how many keys each CTA pushes (its bins
+    // from the row's top down to the boundary bin, in the histograms it
+    // received), so it finds its range without any exchange; after digit
+    // rounds the range is reserved with one remote atomic per CTA.
     uint64_t lthr = local_threshold<T>(st.tau, first);  // the bin's low bits are 0
     lthr = max(lthr, (uint64_t)floor);
     int cnt = 0;
 #pragma unroll
     for (int m = 0; m < M; ++m)
         cnt += key[m] && (uint64_t)key[m] >= lthr;
-    const int off = selected_offset(cnt, reinterpret_cast<int*>(st.warp_top));
-    if (tid == kClThreads - 1) {
-        const uint32_t total = (uint32_t)(off + cnt);
-        st.push_base = total ? atom_add_cluster_u32(cluster_addr(&st.push_count, 0), total) : 0u;
+    int incl = cnt;  // warp-inclusive count: the thread's keys go after the lower lanes'
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o)
+            incl += v;
+    }
+    if (lane == 31)
+        st.warp_top[warp] = (uint32_t)incl;
+    if (!rounds && (uint32_t)warp < ncta) {
+        const uint32_t dbin = st.ctop - (uint32_t)(st.tau >> GS);
+        const uint2 meta = st.inbox_meta[warp];
+        const uint32_t delta = st.ctop - meta.x;
+        uint32_t c = 0;
+        if (dbin >= delta) {
+            const uint32_t last = min(dbin - delta, meta.y - 1u);
+            for (uint32_t i = lane; i <= last; i += 32)
+                c += st.inbox[warp][i];
+        }
+        c = __reduce_add_sync(0xFFFFFFFFu, c);
+        if (lane == 0)
+            st.push_cnt[warp] = c;
     }
     __syncthreads();
+    int off = incl - cnt;
+    for (int w = 0; w < warp; ++w)
+        off += (int)st.warp_top[w];
+    uint32_t base;
+    if (!rounds) {
+        uint32_t b = 0, total = 0;
+#pragma unroll
+        for (uint32_t c = 0; c < (uint32_t)kClMaxCtas; ++c) {
+            if (c < ncta) {
+                total += st.push_cnt[c];
+                if (c < crank)
+                    b += st.push_cnt[c];
+            }
+        }
+        base = b;
+        if (crank == 0 && tid == 0)
+            st.push_count = total;  // no CTA adds to it on this path
+    } else {
+        if (tid == kClThreads - 1) {
+            const uint32_t total = (uint32_t)(off + cnt);
+            st.push_base =
+                total ? atom_add_cluster_u32(cluster_addr(&st.push_count, 0), total) : 0u;
+        }
+        __syncthreads();
+        base = st.push_base;
+    }
     {
-        uint32_t slot = st.push_base + (uint32_t)off;
+        uint32_t slot = base + (uint32_t)off;
         const uint32_t cand0 = cluster_addr(&st.cand[0], 0);
 #pragma unroll
         for (int m = 0; m < M; ++m) {

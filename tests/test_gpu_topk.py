@@ -281,3 +281,43 @@ def test_topk_sample_in_a_graph_with_pdl(rows):
         assert ops.device_errors(clear=True) == 0
     finally:
         ops.set_pdl(old)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_topk_sample_ties_across_cta_boundaries(kernel, dtype):
+    """Equal maxima that straddle the boundary between two CTAs' chunks (the
+    cluster kernel cuts a 151,936-logit row into chunks of 9,496): the
+    candidates must be the lowest indices, crossing the boundary in order.  A
+    run of 11 ties is taken whole by the first round; a run of 100 with k = 50
+    splits the boundary bin and takes the digit rounds."""
+    rng = np.random.default_rng(23)
+    vocab, rows = 151936, 4
+    lg = rng.standard_normal((rows, vocab))
+    lg[0, 9490:9501] = 50.0   # 11 ties over the boundary at 9,496
+    lg[1, 9446:9546] = 50.0   # 100 ties, 50 on each side
+    lg[2, 18980:19000] = 50.0  # 20 ties over the boundary at 18,992
+    lg[3, 151900:] = 50.0     # ties at the end of the last chunk
+    for k in (8, 50):
+        g = rng.gumbel(size=(rows, k)).astype(np.float32)
+        inp = {"logits": torch.from_numpy(lg).float().to(dtype), "gumbel": torch.from_numpy(g)}
+        _check(inp, k, 1.0, f"boundary ties k={k} {dtype}")
+        tok, _ = _run({"logits": inp["logits"], "gumbel": torch.zeros(rows, k)}, k, 1.0)
+        assert list(tok) == [9490, 9446, 18980, 151900]  # greedy: the first index of the maximum
+
+
+def test_topk_sample_dispatch_by_rows():
+    """A call of one row takes the cluster kernel (the workspace stays as it
+    was); one of 64 rows, more than a B200 holds clusters of 16 CTAs at once,
+    takes the slice kernel (its candidates land in the workspace)."""
+    vocab, k = 151936, 50
+    for rows, touched in ((1, False), (64, True)):
+        n = ops.topk_sample_workspace(rows, vocab, k)
+        w8 = torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
+        w8[:COUNTER_BYTES] = 0
+        inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=rows)
+        tok, _ = ops.topk_sample(dev(inp["logits"]), dev(inp["gumbel"]), k, 1.0, workspace=w8)
+        torch.cuda.synchronize()
+        assert bool((w8[COUNTER_BYTES:] != 0xA5).any()) == touched, rows
+        assert not w8[:COUNTER_BYTES].any()
+        t_ref, _ = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 1.0)
+        assert np.array_equal(tok.cpu().numpy(), t_ref)

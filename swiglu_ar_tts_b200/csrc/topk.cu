@@ -1250,11 +1250,13 @@ cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* toke
         return cudaSuccess;
     // The kernel attribute belongs to the current context, so it is set on
     // every launch (a context created after the capacity lookup needs it too).
-    if (cs.ncta > 8) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess)
-            return e;
+    // If it is refused the call falls back to the slice kernel, with the
+    // runtime's last-error state cleared.
+    if (cs.ncta > 8 &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess) {
+        (void)cudaGetLastError();
+        return cudaSuccess;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs.ncta, (unsigned)rows);

@@ -211,18 +211,19 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  *              KiB); every call leaves them zero again, for any later shape.
  *              The rest holds candidates and needs no initialisation.  Two
  *              calls in flight at once must not share one workspace.
- * One kernel is enqueued on `stream`.  When every row's cluster fits on the
- * device at once (a few rows: 7 of 151936 logits on a B200) and the cluster
- * kernel is enabled (arops_set_topk_cluster, the default), it is the
- * single-pass cluster kernel: a thread-block cluster of up to 16 CTAs per row
- * holds the row's logits in registers, the CTAs select the row's top_k
- * together through each other's shared memory, and the cluster's first CTA
- * ranks them and takes the decision; it does not touch the workspace.
- * Otherwise it is the slice kernel: each 4096-logit
- * slice's CTA writes its top_k candidates to the workspace, and the last CTA
- * of a row to finish (counted on the row's arrival counter) merges them and
- * takes the decision; no CTA waits for another.  The two give identical
- * results.  A counter found non-zero at the start of a slice-kernel call (a
+ * One kernel is enqueued on `stream`, by default (arops_set_topk_cluster) a
+ * single-pass cluster kernel: a thread-block cluster per row whose CTAs
+ * select the row's top_k together through each other's shared memory, the
+ * cluster's first CTA ranking them and taking the decision, touching no
+ * workspace byte.  A call whose rows' clusters of up to 16 CTAs all fit on
+ * the device at once (a few rows: 7 of 151936 logits on a B200) holds the
+ * logits in registers; larger calls use clusters of up to 8 CTAs holding
+ * chunks of up to ~76 KB of logits in shared memory, many rows at once.
+ * Where neither can run (or arops_set_topk_cluster(0)) it is the slice
+ * kernel: each 4096-logit slice's CTA writes its top_k candidates to the
+ * workspace, and the last CTA of a row to finish (counted on the row's
+ * arrival counter) merges them and takes the decision; no CTA waits for
+ * another.  All three give identical results.  A counter found non-zero at the start of a slice-kernel call (a
  * workspace that was not cleared) sets AROPS_DEVICE_ERR_WORKSPACE in the
  * device error word, and that row's outputs are then undefined.
  */
@@ -317,13 +318,14 @@ AROPS_API int arops_set_pdl(int enable);
 AROPS_API int arops_set_streaming(int enable);
 
 /*
- * Top-k sampling kernel selection (process-wide).  Enabled (the default),
- * arops_topk_sample and arops_topk_sample_noalloc take the single-pass cluster
- * kernel for calls whose rows' clusters the device holds at once; disabled,
- * always the slice kernel.  Both give identical results; the control exists
- * for measurement and testing.  Returns the old setting.
+ * Top-k sampling kernel selection (process-wide): 0 = the slice kernel for
+ * every call; 1 (the default) = the cluster kernels as described at
+ * arops_topk_sample (registers for few rows, shared memory for many); 2 = the
+ * shared-memory cluster kernel for every call.  Other values are clamped.
+ * Every kernel gives identical results; the control exists for measurement
+ * and testing.  Returns the old setting.
  */
-AROPS_API int arops_set_topk_cluster(int enable);
+AROPS_API int arops_set_topk_cluster(int mode);
 
 /*
  * Device-side error bits of the current device, OR-ed by kernels that abandon

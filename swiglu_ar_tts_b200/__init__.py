@@ -366,11 +366,13 @@ def set_streaming(enable: bool) -> bool:
     return bool(lib().arops_set_streaming(1 if enable else 0))
 
 
-def set_topk_cluster(enable: bool) -> bool:
-    """Choose the single-pass cluster kernel for top-k sampling (the default,
-    where the device can hold its clusters) or the slice kernel; returns the
-    old setting.  Both give identical results."""
-    return bool(lib().arops_set_topk_cluster(1 if enable else 0))
+def set_topk_cluster(mode) -> int:
+    """Which kernels top-k sampling may take: 0 (or False) the slice kernel
+    only; 1 (or True, the default) the cluster kernels, registers for calls
+    whose rows' 16-CTA clusters are all resident at once and shared memory for
+    the rest; 2 the shared-memory cluster kernel for every call.  Returns the
+    old mode.  Every kernel gives identical results."""
+    return int(lib().arops_set_topk_cluster(int(mode)))
 
 
 def device_errors(clear: bool = True) -> int:

@@ -92,9 +92,9 @@ bool streaming_enabled()
     return g_streaming.load(std::memory_order_relaxed) != 0;
 }
 
-bool topk_cluster_enabled()
+int topk_cluster_mode()
 {
-    return g_topk_cluster.load(std::memory_order_relaxed) != 0;
+    return g_topk_cluster.load(std::memory_order_relaxed);
 }
 
 void count_launch()
@@ -443,9 +443,9 @@ AROPS_API int arops_set_streaming(int enable)
     return g_streaming.exchange(enable ? 1 : 0);
 }
 
-AROPS_API int arops_set_topk_cluster(int enable)
+AROPS_API int arops_set_topk_cluster(int mode)
 {
-    return g_topk_cluster.exchange(enable ? 1 : 0);
+    return g_topk_cluster.exchange(mode < 0 ? 0 : (mode > 2 ? 2 : mode));
 }
 
 AROPS_API uint64_t arops_launch_count(void)

@@ -35,9 +35,10 @@
 #include "common.cuh"
 
 namespace arops {
-// Whether calls may take the single-pass cluster kernel (api.cu,
-// arops_set_topk_cluster); otherwise always the slice kernel.
-bool topk_cluster_enabled();
+// Which kernels sampling calls may take (api.cu, arops_set_topk_cluster): 0
+// the slice kernel only; 1 the cluster kernels (registers for few rows, shared
+// memory for many); 2 the shared-memory cluster kernel for every call.
+int topk_cluster_mode();
 }  // namespace arops
 
 namespace arops {
@@ -717,6 +718,7 @@ struct ClusterSelect {
     int binsz;              // keys in the bin, over the whole row
     int window;             // the first round found the bin
     int64_t first;          // the chunk's first vocabulary index
+    uint32_t ncomp;         // keys listed by the shared-memory kernel
     uint32_t ctop;          // the row's largest leading bits
     uint32_t push_cnt[kClMaxCtas];  // keys each CTA pushes (when the first round decides)
     uint32_t push_base;
@@ -840,137 +842,208 @@ __device__ __forceinline__ uint32_t cluster_hist_sum(const uint32_t* h, uint32_t
     return tot;
 }
 
-// Grid (ncta, rows), clusters of ncta CTAs along x; CTA c of a row holds the
-// row's logits [c * chunk, (c + 1) * chunk), M per thread (chunk <= 512 M).
-// VEC: the chunk starts on a 16-byte boundary and thread t loads the 16-byte
-// vectors at chunk positions (v * 512 + t) * E; otherwise one element at a time.
-template <typename T, bool VEC, int M>
-__global__ void __launch_bounds__(kClThreads, (sizeof(T) == 2 && M <= 16) ? 2 : 1)
-topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int k,
-                    const float* __restrict__ gumbel, float temperature,
-                    int32_t* __restrict__ token_out, float* __restrict__ prob_out)
+// This thread's keys of its chunk, as the select walks them:
+//   max_key()        a key no smaller than the smallest key of the thread's
+//                    largest value and no larger than its largest key (0 if
+//                    the thread holds no position of the chunk);
+//   each_from(lo, f) f(key) for every key >= lo (lo > 0).
+// RegKeys holds the keys in registers (M a thread).  SmemKeys forms them from
+// the chunk's values in shared memory (16-byte vectors tid, tid + 512, ...: a
+// chunk too large for registers), testing the values first, two bf16 at a
+// time, so that only the few keys at or above a threshold are ever formed.
+template <typename K, int M>
+struct RegKeys {
+    static constexpr bool kCompact = false;
+    K key[M];  // 0 marks a position past the chunk; no real key is 0
+    __device__ __forceinline__ K max_key() const
+    {
+        K m = 0;
+#pragma unroll
+        for (int i = 0; i < M; ++i)
+            m = max(m, key[i]);
+        return m;
+    }
+    template <class F>
+    __device__ __forceinline__ void each_from(uint64_t lo, F&& f) const
+    {
+#pragma unroll
+        for (int i = 0; i < M; ++i)
+            if ((uint64_t)key[i] >= lo)
+                f(key[i]);
+    }
+};
+
+// The keys of a CTA listed in shared memory (the compacted ones): thread tid
+// takes entries tid, tid + 512, ...
+template <typename K>
+struct ListKeys {
+    const K* list;
+    int n;
+    template <class F>
+    __device__ __forceinline__ void each_from(uint64_t lo, F&& f) const
+    {
+        for (int i = (int)threadIdx.x; i < n; i += kClThreads) {
+            const K x = list[i];
+            if ((uint64_t)x >= lo)
+                f(x);
+        }
+    }
+};
+
+// Keys from the floor up that the shared-memory kernel lists for its later
+// passes (~130 a CTA for logit-like rows; a row that has more keeps walking
+// its whole chunk).
+constexpr int kCompactKeys = 2048;
+
+template <typename T>
+struct SmemKeys;
+
+// Largest of each 16-bit half (a single instruction on sm_90 and later).
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Two bf16 in a 32-bit word, each turned into the 16 bits KeyBits orders by.
+__device__ __forceinline__ uint32_t ordered_bf16x2(uint32_t w)
+{
+    const uint32_t sign = (w >> 15) & 0x00010001u;
+    return w ^ 0x80008000u ^ (sign * 0x7FFFu);
+}
+
+template <>
+struct SmemKeys<__nv_bfloat16> {
+    static constexpr bool kCompact = true;
+    const __nv_bfloat16* vals;  // 16-byte aligned, padded to whole vectors
+    int n;
+    uint32_t* list;             // kCompactKeys entries for the compacted keys
+    __device__ __forceinline__ uint32_t max_key() const
+    {
+        const int nv = (n + 7) / 8;
+        uint32_t acc = 0;
+        bool any = false;
+        for (int v = (int)threadIdx.x; v < nv; v += kClThreads) {
+            const uint4 x = reinterpret_cast<const uint4*>(vals)[v];
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            if (v * 8 + 8 <= n) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    acc = max_u16x2(acc, ordered_bf16x2(w[i]));
+            } else {  // the ragged last vector
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t o = ordered_bf16x2(w[i]);
+                    if (v * 8 + 2 * i < n)
+                        acc = max_u16x2(acc, o & 0xFFFFu);
+                    if (v * 8 + 2 * i + 1 < n)
+                        acc = max_u16x2(acc, o & 0xFFFF0000u);
+                }
+            }
+            any = true;
+        }
+        const uint32_t m = max(acc & 0xFFFFu, acc >> 16);
+        return any ? (m << 16) : 0u;  // (value, inverted position 0): the value's smallest key
+    }
+    template <class F>
+    __device__ __forceinline__ void each_from(uint64_t lo, F&& f) const
+    {
+        if (lo > 0xFFFFFFFFull)
+            return;
+        const uint32_t lov = (uint32_t)(lo >> 16);
+        // a half is at least lov when max(half, lov - 1) moves off lov - 1
+        const uint32_t below2 = (lov ? lov - 1u : 0u) * 0x00010001u;
+        const int nv = (n + 7) / 8;
+        for (int v = (int)threadIdx.x; v < nv; v += kClThreads) {
+            const uint4 x = reinterpret_cast<const uint4*>(vals)[v];
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t o = ordered_bf16x2(w[i]);
+                if (lov == 0u || max_u16x2(o, below2) != below2) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int p = v * 8 + 2 * i + h;
+                        if (((o >> (16 * h)) & 0xFFFFu) >= lov && p < n) {
+                            const uint32_t key = (((o >> (16 * h)) & 0xFFFFu) << 16) |
+                                                 (0xFFFFu - (uint32_t)p);
+                            if (key >= (uint32_t)lo)
+                                f(key);
+                        }
+                    }
+                }
+            }
+        }
+    }
+};
+
+template <>
+struct SmemKeys<float> {
+    static constexpr bool kCompact = true;
+    const float* vals;  // 16-byte aligned, padded to whole vectors
+    int n;
+    uint64_t* list;     // kCompactKeys entries for the compacted keys
+    __device__ __forceinline__ uint64_t max_key() const
+    {
+        uint32_t m = 0;
+        bool any = false;
+        for (int p = (int)threadIdx.x * 4; p < n; p += kClThreads * 4) {
+            const float4 x = *reinterpret_cast<const float4*>(vals + p);
+            const float e[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (p + j < n)
+                    m = max(m, order_bits(e[j]));
+            any = true;
+        }
+        return any ? ((uint64_t)m << 16) : 0ull;
+    }
+    template <class F>
+    __device__ __forceinline__ void each_from(uint64_t lo, F&& f) const
+    {
+        if (lo > 0xFFFFFFFFFFFFull)
+            return;
+        const uint32_t lov = (uint32_t)(lo >> 16);
+        for (int p = (int)threadIdx.x * 4; p < n; p += kClThreads * 4) {
+            const float4 x = *reinterpret_cast<const float4*>(vals + p);
+            const float e[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t o = order_bits(e[j]);
+                if (o >= lov && p + j < n) {
+                    const uint64_t key = ((uint64_t)o << 16) | (0xFFFFu - (uint32_t)(p + j));
+                    if (key >= lo)
+                        f(key);
+                }
+            }
+        }
+    }
+};
+
+// The rest of the select, from the histogram exchange on, and the sampling
+// decision; `keys` walks this thread's keys from `floor` up.
+template <typename T, class Keys>
+__device__ __forceinline__ void cluster_finish(const Keys& keys, ClusterSelect& st,
+                                               typename LocalKey<T>::type floor, uint32_t top,
+                                               int64_t row, int64_t first, int k,
+                                               const float (&gdraw)[2], float temperature,
+                                               int32_t* token_out, float* prob_out)
 {
     using K = typename LocalKey<T>::type;
-    constexpr int E = Vec<T>::N;
     constexpr int VS = LocalKey<T>::BITS - 16;  // leading 16 bits of a local key
     constexpr int GB = KeyBits<T>::V + kIndexBits;
     constexpr int GS = GB - 16;                 // leading 16 bits of a row key
-    static_assert(!VEC || M % E == 0, "whole vectors per thread");
-    __shared__ ClusterSelect st;
     const int tid = (int)threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const uint32_t crank = cluster_ctarank();
     const uint32_t ncta = cluster_nctarank();
-    const int64_t row = blockIdx.y;
-    const int64_t first = (int64_t)crank * chunk;
-    const int n = (int)(vocab - first < (int64_t)chunk ? (vocab - first > 0 ? vocab - first : 0)
-                                                       : (int64_t)chunk);
-    const T* src = logits + row * vocab + first;
-    // the chunk into L2 while the previous kernel drains, one line per thread
-    {
-        constexpr int kPerLine = 128 / sizeof(T);
-        for (int i = tid * kPerLine; i < n; i += kClThreads * kPerLine)
-            prefetch_l2_line(src + i);
-    }
-    for (int i = tid; i < 256; i += kClThreads)
-        st.hist[0][i] = 0;
-    if (tid == 0) {
-        st.push_count = 0;
-        st.window = 0;
-        st.first = first;
-    }
-    pdl_wait();
-    pdl_allow_dependents();
-
-    float gdraw[2] = {0.f, 0.f};  // the first CTA's warp 0: draws of ranks lane, lane + 32
-    if (crank == 0 && tid < 32) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-            if (tid + 32 * r < k)
-                gdraw[r] = __ldg(gumbel + row * k + tid + 32 * r);
-    }
-    K key[M];  // local keys; 0 marks a position past the chunk (no real key is 0)
-    if constexpr (VEC) {
-#pragma unroll
-        for (int v = 0; v < M / E; ++v) {
-            const int p0 = (v * kClThreads + tid) * E;
-            float f[E];
-            if (p0 + E <= n) {
-                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(src + p0)), f);
-            } else {
-#pragma unroll
-                for (int j = 0; j < E; ++j)
-                    f[j] = (p0 + j < n) ? load_elem(src + p0 + j) : 0.f;
-            }
-#pragma unroll
-            for (int j = 0; j < E; ++j)
-                key[v * E + j] = (p0 + j < n) ? (((K)KeyBits<T>::of(f[j]) << 16) |
-                                                 (K)(0xFFFFu - (uint32_t)(p0 + j)))
-                                              : K(0);
-        }
-    } else {
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const int p = tid + m * kClThreads;
-            key[m] = (p < n) ? (((K)KeyBits<T>::of(load_elem(src + p)) << 16) |
-                                (K)(0xFFFFu - (uint32_t)p))
-                             : K(0);
-        }
-    }
-
-    // First round.  Each warp finds the r = ceil(k / 16) largest of its lanes'
-    // largest keys; the smallest of the 16 warps' r-th values, `floor`, has at
-    // least 16 r >= k of the CTA's keys at or above it, so the CTA's k-th
-    // largest key, and with it the row's, is not below it: keys under `floor`
-    // take no further part (typically all but a few dozen of the chunk's).
-    // Then the CTA's largest leading 16 bits and its histogram of the
-    // distances below them (the 256 nearest values) over the remaining keys.
-    K floor;
-    uint32_t top;
-    {
-        K cur = 0;
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-            cur = max(cur, key[m]);
-        const int r = (k + kClWarps - 1) / kClWarps;
-        K wtop = 0, rth = 0;
-        for (int i = 0; i < r; ++i) {
-            const K w = warp_max(cur);
-            if (i == 0)
-                wtop = w;
-            rth = w;
-            if (cur == w)  // keys are distinct: the lane that holds it drops out
-                cur = 0;
-        }
-        if (lane == 0) {
-            st.warp_key[warp] = (uint64_t)wtop;
-            st.warp_floor[warp] = (uint64_t)rth;
-        }
-        __syncthreads();
-        uint64_t t = 0, f = ~0ull;
-#pragma unroll
-        for (int w = 0; w < kClWarps; ++w) {
-            t = max(t, st.warp_key[w]);
-            f = min(f, st.warp_floor[w]);
-        }
-        floor = (K)f;
-        top = (uint32_t)(t >> VS);
-    }
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-        if (key[m] && key[m] >= floor) {
-            const uint32_t d = top - (uint32_t)(key[m] >> VS);
-            if (d < 256u)
-                atomicAdd(&st.hist[0][d], 1u);
-        }
-    }
     // Send the histogram to every CTA of the cluster (its row `crank` of their
     // inboxes) before the barrier, so that the sum after it reads only this
     // CTA's own shared memory.  The keys that take part lie within `span` bins
     // of the CTA's largest leading bits (the floor's are the lowest), so only
     // those bins go out, four to a store: a few dozen for logit-like rows.
-    __syncthreads();  // the CTA's histogram is complete
     {
         const uint32_t flead = (uint32_t)(floor >> VS);
         const uint32_t span = floor ? min(256u, top - flead + 1u) : 256u;
@@ -1031,14 +1104,11 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
         // re-read each round, so that the row keys are formed here and not
         // kept in registers across rounds
         const int64_t f = *reinterpret_cast<volatile int64_t*>(&st.first);
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            if (key[m] && key[m] >= floor) {
-                const uint64_t g = row_key<T>(key[m], f);
-                if ((g & high_mask) == prefix)
-                    atomicAdd(&h[(uint32_t)(g >> shift) & 255u], 1u);
-            }
-        }
+        keys.each_from(floor ? (uint64_t)floor : 1ull, [&](K x) {
+            const uint64_t g = row_key<T>(x, f);
+            if ((g & high_mask) == prefix)
+                atomicAdd(&h[(uint32_t)(g >> shift) & 255u], 1u);
+        });
         cluster_barrier();
         if (tid < 256)
             st.ghist[tid] = cluster_hist_sum(h, ncta);
@@ -1059,9 +1129,7 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
     uint64_t lthr = local_threshold<T>(st.tau, first);  // the bin's low bits are 0
     lthr = max(lthr, (uint64_t)floor);
     int cnt = 0;
-#pragma unroll
-    for (int m = 0; m < M; ++m)
-        cnt += key[m] && (uint64_t)key[m] >= lthr;
+    keys.each_from(lthr ? lthr : 1ull, [&](K) { ++cnt; });
     int incl = cnt;  // warp-inclusive count: the thread's keys go after the lower lanes'
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1115,14 +1183,11 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
     {
         uint32_t slot = base + (uint32_t)off;
         const uint32_t cand0 = cluster_addr(&st.cand[0], 0);
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            if (key[m] && (uint64_t)key[m] >= lthr) {
-                if (slot < (uint32_t)kClPushSlots)  // never reached: the bound only guards
-                    st_cluster_u64(cand0 + 8u * slot, row_key<T>(key[m], first));
-                ++slot;
-            }
-        }
+        keys.each_from(lthr ? lthr : 1ull, [&](K x) {
+            if (slot < (uint32_t)kClPushSlots)  // never reached: the bound only guards
+                st_cluster_u64(cand0 + 8u * slot, row_key<T>(x, first));
+            ++slot;
+        });
     }
     cluster_barrier();  // every push has landed; no CTA touches another's memory after this
     if (crank != 0)
@@ -1147,6 +1212,221 @@ topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int 
     }
     __syncthreads();
     sample_decision<T>(st.ranked, k, gdraw, temperature, token_out + row, prob_out + row);
+}
+
+// The select and the sampling decision of one row's cluster, shared by the
+// cluster kernels: `keys` walks this thread's keys of the chunk (KeySource
+// below), `st` is the CTA's shared state (its first round's histogram zeroed
+// and push_count, window and first set before the dependency wait).
+template <typename T, class Keys>
+__device__ __forceinline__ void cluster_select_sample(const Keys& keys, ClusterSelect& st,
+                                                      int64_t row, int64_t first, int k,
+                                                      const float (&gdraw)[2], float temperature,
+                                                      int32_t* token_out, float* prob_out)
+{
+    using K = typename LocalKey<T>::type;
+    constexpr int VS = LocalKey<T>::BITS - 16;  // leading 16 bits of a local key
+    const int tid = (int)threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+
+    // First round.  Each warp finds the r = ceil(k / 16) largest of its lanes'
+    // largest keys; the smallest of the 16 warps' r-th values, `floor`, has at
+    // least 16 r >= k of the CTA's keys at or above it, so the CTA's k-th
+    // largest key, and with it the row's, is not below it: keys under `floor`
+    // take no further part (typically all but a few dozen of the chunk's).
+    // Then the CTA's largest leading 16 bits and its histogram of the
+    // distances below them (the 256 nearest values) over the remaining keys.
+    K floor;
+    uint32_t top;
+    {
+        K cur = keys.max_key();
+        const int r = (k + kClWarps - 1) / kClWarps;
+        K wtop = 0, rth = 0;
+        for (int i = 0; i < r; ++i) {
+            const K w = warp_max(cur);
+            if (i == 0)
+                wtop = w;
+            rth = w;
+            if (cur == w)  // keys are distinct: the lane that holds it drops out
+                cur = 0;
+        }
+        if (lane == 0) {
+            st.warp_key[warp] = (uint64_t)wtop;
+            st.warp_floor[warp] = (uint64_t)rth;
+        }
+        __syncthreads();
+        uint64_t t = 0, f = ~0ull;
+#pragma unroll
+        for (int w = 0; w < kClWarps; ++w) {
+            t = max(t, st.warp_key[w]);
+            f = min(f, st.warp_floor[w]);
+        }
+        floor = (K)f;
+        top = (uint32_t)(t >> VS);
+    }
+    keys.each_from(floor ? (uint64_t)floor : 1ull, [&](K x) {
+        const uint32_t d = top - (uint32_t)(x >> VS);
+        if (d < 256u)
+            atomicAdd(&st.hist[0][d], 1u);
+        if constexpr (Keys::kCompact) {  // the keys that take part, listed for the later passes
+            const uint32_t slot = atomicAdd(&st.ncomp, 1u);
+            if (slot < (uint32_t)kCompactKeys)
+                keys.list[slot] = x;
+        }
+    });
+    __syncthreads();  // the CTA's histogram (and list) is complete
+    if constexpr (Keys::kCompact) {
+        if (st.ncomp <= (uint32_t)kCompactKeys) {
+            const ListKeys<K> listed{keys.list, (int)st.ncomp};
+            cluster_finish<T>(listed, st, floor, top, row, first, k, gdraw, temperature,
+                              token_out, prob_out);
+            return;
+        }
+    }
+    cluster_finish<T>(keys, st, floor, top, row, first, k, gdraw, temperature, token_out,
+                      prob_out);
+}
+
+// What both cluster kernels do first: this CTA's chunk of its row into L2
+// while the previous kernel drains, the first round's histogram zeroed and the
+// shared state set, the dependency wait, and the first CTA's warp 0 loads the
+// Gumbel draws of ranks lane and lane + 32.  Returns the chunk's first logit.
+template <typename T>
+__device__ __forceinline__ const T* cluster_prologue(ClusterSelect& st, const T* logits,
+                                                     int64_t vocab, int chunk, int k,
+                                                     const float* __restrict__ gumbel,
+                                                     int64_t& first, int& n, float (&gdraw)[2])
+{
+    const int tid = (int)threadIdx.x;
+    const uint32_t crank = cluster_ctarank();
+    const int64_t row = blockIdx.y;
+    first = (int64_t)crank * chunk;
+    n = (int)(vocab - first < (int64_t)chunk ? (vocab - first > 0 ? vocab - first : 0)
+                                              : (int64_t)chunk);
+    const T* src = logits + row * vocab + first;
+    {
+        constexpr int kPerLine = 128 / sizeof(T);
+        for (int i = tid * kPerLine; i < n; i += kClThreads * kPerLine)
+            prefetch_l2_line(src + i);
+    }
+    for (int i = tid; i < 256; i += kClThreads)
+        st.hist[0][i] = 0;
+    if (tid == 0) {
+        st.push_count = 0;
+        st.window = 0;
+        st.first = first;
+        st.ncomp = 0;
+    }
+    pdl_wait();
+    pdl_allow_dependents();
+    gdraw[0] = gdraw[1] = 0.f;
+    if (crank == 0 && tid < 32) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if (tid + 32 * r < k)
+                gdraw[r] = __ldg(gumbel + row * k + tid + 32 * r);
+    }
+    return src;
+}
+
+// Grid (ncta, rows), clusters of ncta CTAs along x; CTA c of a row holds the
+// row's logits [c * chunk, (c + 1) * chunk), M per thread in registers (chunk
+// <= 512 M).  VEC: the chunk starts on a 16-byte boundary and thread t loads
+// the 16-byte vectors at chunk positions (v * 512 + t) * E; otherwise one
+// element at a time.
+template <typename T, bool VEC, int M>
+__global__ void __launch_bounds__(kClThreads, (sizeof(T) == 2 && M <= 16) ? 2 : 1)
+topk_cluster_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int k,
+                    const float* __restrict__ gumbel, float temperature,
+                    int32_t* __restrict__ token_out, float* __restrict__ prob_out)
+{
+    using K = typename LocalKey<T>::type;
+    constexpr int E = Vec<T>::N;
+    static_assert(!VEC || M % E == 0, "whole vectors per thread");
+    __shared__ ClusterSelect st;
+    const int tid = (int)threadIdx.x;
+    int64_t first;
+    int n;
+    float gdraw[2];
+    const T* src = cluster_prologue<T>(st, logits, vocab, chunk, k, gumbel, first, n, gdraw);
+    RegKeys<K, M> keys;
+    if constexpr (VEC) {
+#pragma unroll
+        for (int v = 0; v < M / E; ++v) {
+            const int p0 = (v * kClThreads + tid) * E;
+            float f[E];
+            if (p0 + E <= n) {
+                Vec<T>::unpack(__ldg(reinterpret_cast<const uint4*>(src + p0)), f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < E; ++j)
+                    f[j] = (p0 + j < n) ? load_elem(src + p0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < E; ++j)
+                keys.key[v * E + j] = (p0 + j < n) ? (((K)KeyBits<T>::of(f[j]) << 16) |
+                                                      (K)(0xFFFFu - (uint32_t)(p0 + j)))
+                                                   : K(0);
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const int p = tid + m * kClThreads;
+            keys.key[m] = (p < n) ? (((K)KeyBits<T>::of(load_elem(src + p)) << 16) |
+                                     (K)(0xFFFFu - (uint32_t)p))
+                                  : K(0);
+        }
+    }
+    cluster_select_sample<T>(keys, st, blockIdx.y, first, k, gdraw, temperature, token_out,
+                             prob_out);
+}
+
+// Many-row variant: smaller clusters (up to 8 CTAs, so that many rows' clusters
+// are resident at once) whose CTAs hold chunks too large for registers (up to
+// ~76 KB of logits, 16-bit positions) in shared memory; the select walks them
+// from there (SmemKeys).  VEC: 16-byte-aligned chunks copied with 16-byte
+// loads, eight in flight per thread; otherwise one element at a time.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kClThreads, 2)
+topk_cluster_smem_kernel(const T* __restrict__ logits, int64_t vocab, int chunk, int k,
+                         const float* __restrict__ gumbel, float temperature,
+                         int32_t* __restrict__ token_out, float* __restrict__ prob_out)
+{
+    constexpr int E = Vec<T>::N;
+    extern __shared__ uint4 topk_chunk_smem[];  // the chunk, padded to whole vectors
+    __shared__ ClusterSelect st;
+    const int tid = (int)threadIdx.x;
+    int64_t first;
+    int n;
+    float gdraw[2];
+    const T* src = cluster_prologue<T>(st, logits, vocab, chunk, k, gumbel, first, n, gdraw);
+    T* vals = reinterpret_cast<T*>(topk_chunk_smem);
+    if constexpr (VEC) {
+        constexpr int B = 8;
+        const int nv = n / E;  // n is a multiple of E when rows are 16-byte aligned
+        const uint4* s4 = reinterpret_cast<const uint4*>(src);
+        for (int v0 = tid; v0 < nv; v0 += B * kClThreads) {
+            uint4 r[B];
+#pragma unroll
+            for (int b = 0; b < B; ++b)
+                if (v0 + b * kClThreads < nv)
+                    r[b] = __ldg(s4 + v0 + b * kClThreads);
+#pragma unroll
+            for (int b = 0; b < B; ++b)
+                if (v0 + b * kClThreads < nv)
+                    topk_chunk_smem[v0 + b * kClThreads] = r[b];
+        }
+    } else {
+        for (int p = tid; p < n; p += kClThreads)
+            vals[p] = src[p];
+    }
+    __syncthreads();
+    using K = typename LocalKey<T>::type;
+    K* list = reinterpret_cast<K*>(topk_chunk_smem + (chunk * sizeof(T) + 15) / 16);
+    const SmemKeys<T> keys{vals, n, list};
+    cluster_select_sample<T>(keys, st, blockIdx.y, first, k, gdraw, temperature, token_out,
+                             prob_out);
 }
 
 }  // namespace
@@ -1193,11 +1473,13 @@ ClusterShape cluster_shape(int64_t vocab)
     return {ncta, (int)chunk, m};
 }
 
-// Clusters of `ncta` CTAs of `Kernel` that the current device holds at once
-// (0 if it cannot run them; above 8 CTAs it first allows the non-portable
-// cluster size on the kernel).  Looked up once per device and cluster size.
+// Clusters of `ncta` CTAs of `Kernel` (with `smem` bytes of dynamic shared
+// memory a CTA) that the current device holds at once (0 if it cannot run
+// them; above 8 CTAs it first allows the non-portable cluster size on the
+// kernel).  Looked up once per device and cluster size: every launcher passes
+// one `smem` per kernel (its largest).
 template <auto Kernel>
-int cluster_capacity(int ncta)
+int cluster_capacity(int ncta, size_t smem = 0)
 {
     constexpr int kMaxDevices = 64;
     constexpr int kSizes = 5;  // 1, 2, 4, 8, 16 CTAs
@@ -1211,12 +1493,18 @@ int cluster_capacity(int ncta)
     int v = cache[dev][slot].load(std::memory_order_relaxed);
     if (v == 0) {
         int clusters = 0;
-        if (ncta <= 8 ||
-            cudaFuncSetAttribute(Kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                cudaSuccess) {
+        const bool attrs_ok =
+            (ncta <= 8 ||
+             cudaFuncSetAttribute(Kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                 cudaSuccess) &&
+            (smem <= 48 * 1024 ||
+             cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem) == cudaSuccess);
+        if (attrs_ok) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)ncta, 1);
             cfg.blockDim = dim3(kClThreads);
+            cfg.dynamicSmemBytes = smem;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
             attr[0].val.clusterDim.x = (unsigned)ncta;
@@ -1234,6 +1522,35 @@ int cluster_capacity(int ncta)
     return v - 1;
 }
 
+// Kernel attributes a cluster launch needs (the non-portable cluster size
+// above 8 CTAs, dynamic shared memory above 48 KB), set once per device: a
+// call costs several microseconds on the host, as much as the kernel.  They
+// belong to a CUDA context, so a launch that is refused (a context created
+// after they were set) sets them again and retries once (launch_with_attrs).
+template <auto Kernel>
+cudaError_t set_cluster_attrs(int ncta, size_t smem, bool force)
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];  // 1: set on that device
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices)
+        dev = -1;
+    if (!force && dev >= 0 && done[dev].load(std::memory_order_relaxed))
+        return cudaSuccess;
+    cudaError_t e = cudaSuccess;
+    if (ncta > 8)
+        e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess && smem > 48 * 1024)
+        e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return e;
+    }
+    if (dev >= 0)
+        done[dev].store(1, std::memory_order_relaxed);
+    return cudaSuccess;
+}
+
 template <typename T, bool VEC, int M>
 cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* token_out,
                              float* prob_out, int64_t rows, int64_t vocab, int k,
@@ -1248,16 +1565,9 @@ cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* toke
     // B200; 8 rows: 18.4 against 14.7).
     if (rows > cluster_capacity<kernel>(cs.ncta))
         return cudaSuccess;
-    // The kernel attribute belongs to the current context, so it is set on
-    // every launch (a context created after the capacity lookup needs it too).
-    // If it is refused the call falls back to the slice kernel, with the
-    // runtime's last-error state cleared.
-    if (cs.ncta > 8 &&
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess) {
-        (void)cudaGetLastError();
+    // refused attributes: the slice kernel takes the call
+    if (set_cluster_attrs<kernel>(kClMaxCtas, 0, false) != cudaSuccess)
         return cudaSuccess;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs.ncta, (unsigned)rows);
     cfg.blockDim = dim3(kClThreads);
@@ -1275,8 +1585,14 @@ cudaError_t launch_cluster_t(const T* logits, const float* gumbel, int32_t* toke
         cfg.numAttrs = 2;
     }
     *launched = true;
-    const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, cs.chunk, k, gumbel,
-                                               temperature, token_out, prob_out);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, cs.chunk, k, gumbel,
+                                         temperature, token_out, prob_out);
+    if (err != cudaSuccess && cs.ncta > 8) {  // attributes of another context: set, retry
+        (void)cudaGetLastError();
+        if (set_cluster_attrs<kernel>(kClMaxCtas, 0, true) == cudaSuccess)
+            err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, cs.chunk, k, gumbel,
+                                     temperature, token_out, prob_out);
+    }
     if (err == cudaSuccess)
         count_launch();
     return err;
@@ -1307,6 +1623,77 @@ cudaError_t launch_cluster_m(const T* logits, const float* gumbel, int32_t* toke
     }
 }
 
+// Shape of the many-row launch: the fewest CTAs per cluster (a power of two
+// up to 8, the portable size) whose chunks hold at most ~76 KB of logits and
+// 65,528 positions (16-bit local positions, multiples of 8 logits), so that
+// two CTAs share an SM and many rows' clusters are resident at once.  ncta = 0
+// when no such shape exists.
+struct SmemShape {
+    int ncta;
+    int chunk;
+    size_t smem;  // dynamic shared memory a CTA: the chunk's values
+};
+
+constexpr size_t kSmemChunkTarget = 76 * 1024;
+constexpr int kSmemMaxChunk = 65528;
+constexpr size_t kSmemMaxBytes = 144 * 1024;  // fp32 rows of 262,144 logits over 8 CTAs
+
+SmemShape smem_shape(int64_t vocab, size_t esize)
+{
+    int ncta = 1;
+    while (ncta < 8 && ((size_t)ceil_div(vocab, ncta) * esize > kSmemChunkTarget ||
+                        ceil_div(vocab, ncta) > kSmemMaxChunk))
+        ncta *= 2;
+    const int64_t chunk = (int64_t)round_up((uint32_t)ceil_div(vocab, ncta), 8u);
+    if (chunk > kSmemMaxChunk || (size_t)chunk * esize + kCompactKeys * 8 > kSmemMaxBytes)
+        return {0, 0, 0};
+    const size_t key_bytes = esize == 2 ? 4 : 8;
+    return {ncta, (int)chunk, (size_t)chunk * esize + kCompactKeys * key_bytes};
+}
+
+template <typename T, bool VEC>
+cudaError_t launch_cluster_smem(const T* logits, const float* gumbel, int32_t* token_out,
+                                float* prob_out, int64_t rows, int64_t vocab, int k,
+                                float temperature, cudaStream_t stream, bool* launched)
+{
+    constexpr auto kernel = topk_cluster_smem_kernel<T, VEC>;
+    *launched = false;
+    const SmemShape ss = smem_shape(vocab, sizeof(T));
+    if (ss.ncta == 0 || cluster_capacity<kernel>(ss.ncta, kSmemMaxBytes) < 1)
+        return cudaSuccess;
+    if (set_cluster_attrs<kernel>(8, kSmemMaxBytes, false) != cudaSuccess)
+        return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ss.ncta, (unsigned)rows);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = ss.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ss.ncta;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (pdl_enabled()) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
+    }
+    *launched = true;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, ss.chunk, k, gumbel,
+                                         temperature, token_out, prob_out);
+    if (err != cudaSuccess && ss.smem > 48 * 1024) {  // attributes of another context
+        (void)cudaGetLastError();
+        if (set_cluster_attrs<kernel>(8, kSmemMaxBytes, true) == cudaSuccess)
+            err = cudaLaunchKernelEx(&cfg, kernel, logits, vocab, ss.chunk, k, gumbel,
+                                     temperature, token_out, prob_out);
+    }
+    if (err == cudaSuccess)
+        count_launch();
+    return err;
+}
+
 }  // namespace
 
 cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
@@ -1316,28 +1703,56 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
 {
     const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
     const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
-    if (topk_cluster_enabled()) {
-        const ClusterShape cs = cluster_shape(vocab);
+    const int mode = topk_cluster_mode();
+    if (mode != 0) {
         bool launched = false;
-        cudaError_t err;
-        if (dtype == AROPS_BF16) {
-            const auto* lg = static_cast<const __nv_bfloat16*>(logits);
-            err = vec ? launch_cluster_m<__nv_bfloat16, true>(lg, gumbel, token_out, prob_out, rows,
-                                                              vocab, k, temperature, cs, stream,
-                                                              &launched)
-                      : launch_cluster_m<__nv_bfloat16, false>(lg, gumbel, token_out, prob_out,
-                                                               rows, vocab, k, temperature, cs,
-                                                               stream, &launched);
-        } else {
-            const auto* lg = static_cast<const float*>(logits);
-            err = vec ? launch_cluster_m<float, true>(lg, gumbel, token_out, prob_out, rows, vocab,
-                                                      k, temperature, cs, stream, &launched)
-                      : launch_cluster_m<float, false>(lg, gumbel, token_out, prob_out, rows, vocab,
-                                                       k, temperature, cs, stream, &launched);
+        cudaError_t err = cudaSuccess;
+        // few rows: the register cluster kernel, while every row's cluster is
+        // resident at once (mode 1); otherwise the shared-memory one
+        if (mode == 1) {
+            const ClusterShape cs = cluster_shape(vocab);
+            if (dtype == AROPS_BF16) {
+                const auto* lg = static_cast<const __nv_bfloat16*>(logits);
+                err = vec ? launch_cluster_m<__nv_bfloat16, true>(lg, gumbel, token_out, prob_out,
+                                                                  rows, vocab, k, temperature, cs,
+                                                                  stream, &launched)
+                          : launch_cluster_m<__nv_bfloat16, false>(lg, gumbel, token_out, prob_out,
+                                                                   rows, vocab, k, temperature,
+                                                                   cs, stream, &launched);
+            } else {
+                const auto* lg = static_cast<const float*>(logits);
+                err = vec ? launch_cluster_m<float, true>(lg, gumbel, token_out, prob_out, rows,
+                                                          vocab, k, temperature, cs, stream,
+                                                          &launched)
+                          : launch_cluster_m<float, false>(lg, gumbel, token_out, prob_out, rows,
+                                                           vocab, k, temperature, cs, stream,
+                                                           &launched);
+            }
+        }
+        if (!launched) {
+            if (dtype == AROPS_BF16) {
+                const auto* lg = static_cast<const __nv_bfloat16*>(logits);
+                err = vec ? launch_cluster_smem<__nv_bfloat16, true>(lg, gumbel, token_out,
+                                                                     prob_out, rows, vocab, k,
+                                                                     temperature, stream,
+                                                                     &launched)
+                          : launch_cluster_smem<__nv_bfloat16, false>(lg, gumbel, token_out,
+                                                                      prob_out, rows, vocab, k,
+                                                                      temperature, stream,
+                                                                      &launched);
+            } else {
+                const auto* lg = static_cast<const float*>(logits);
+                err = vec ? launch_cluster_smem<float, true>(lg, gumbel, token_out, prob_out, rows,
+                                                             vocab, k, temperature, stream,
+                                                             &launched)
+                          : launch_cluster_smem<float, false>(lg, gumbel, token_out, prob_out,
+                                                              rows, vocab, k, temperature, stream,
+                                                              &launched);
+            }
         }
         if (launched)
             return err;
-        // more rows than resident clusters, or no such clusters here: the slice kernel
+        // no cluster launch possible here: the slice kernel
     }
     const int slices = topk_slices(vocab);
     const dim3 grid((unsigned)slices, (unsigned)rows);

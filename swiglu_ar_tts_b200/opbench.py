@@ -179,8 +179,8 @@ def main() -> None:
                     help="shared-memory streaming kernels instead of the default register kernels")
     ap.add_argument("--no-chain-pdl", action="store_true",
                     help="decode steps without programmatic dependent launch")
-    ap.add_argument("--topk-slice", action="store_true",
-                    help="top-k sampling on the slice kernel instead of the cluster kernel")
+    ap.add_argument("--topk-mode", type=int, default=1, choices=(0, 1, 2),
+                    help="top-k kernels: 0 slice, 1 cluster (default), 2 shared-memory cluster")
     ap.add_argument("--json", action="store_true")
     a = ap.parse_args()
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -188,7 +188,7 @@ def main() -> None:
     CHAIN_PDL = not a.no_chain_pdl
     set_pdl(a.pdl)
     set_streaming(a.streaming)
-    set_topk_cluster(not a.topk_slice)
+    set_topk_cluster(a.topk_mode)
     for op in (OPS if a.op == "all" else (a.op,)):
         fns, nbytes, desc = make_rotation(op, a.rows, dev, a.copies)
         us = time_op(fns, a.iters)

@@ -15,9 +15,12 @@ from tolerance import to_f64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["cluster", "slice"])
+MODES = {"slice": 0, "cluster": 1, "smem": 2}  # arops_set_topk_cluster
+
+
+@pytest.fixture(params=["cluster", "smem", "slice"])
 def kernel(request):
-    old = ops.set_topk_cluster(request.param == "cluster")
+    old = ops.set_topk_cluster(MODES[request.param])
     yield request.param
     ops.set_topk_cluster(old)
 
@@ -220,12 +223,12 @@ def test_topk_sample_cluster_kernel_leaves_the_workspace_alone():
 
 @pytest.mark.parametrize("rows", [1, 7, 64, 300])
 def test_topk_sample_kernels_agree_bit_for_bit(rows):
-    """The two kernels give the same tokens and the same probabilities, bit
+    """The three kernels give the same tokens and the same probabilities, bit
     for bit, over many rows."""
     inp = inputs.topk_inputs(rows, 151936, 50, "bf16", seed=rows)
     lg, g = dev(inp["logits"]), dev(inp["gumbel"])
     out = {}
-    for mode in (True, False):
+    for mode in (1, 2, 0):
         old = ops.set_topk_cluster(mode)
         try:
             tok, prob = ops.topk_sample(lg, g, 50, 0.8)
@@ -233,16 +236,17 @@ def test_topk_sample_kernels_agree_bit_for_bit(rows):
         finally:
             ops.set_topk_cluster(old)
         out[mode] = (tok.cpu(), prob.cpu())
-    assert torch.equal(out[True][0], out[False][0])
-    assert torch.equal(out[True][1], out[False][1])
+    for mode in (1, 2):
+        assert torch.equal(out[mode][0], out[0][0]), mode
+        assert torch.equal(out[mode][1], out[0][1]), mode
 
 
 @pytest.mark.parametrize("rows", [5, 20])
 def test_topk_sample_in_a_graph_with_pdl(rows):
     """Sampling captured in a CUDA graph behind another kernel, with
-    programmatic dependent launch (the end of a decode step): the cluster
-    kernel (5 rows) and the slice kernel (20 rows) replayed on new logits and
-    draws each time, every replay against the oracle."""
+    programmatic dependent launch (the end of a decode step): the register
+    cluster kernel (5 rows) and the shared-memory one (20 rows) replayed on
+    new logits and draws each time, every replay against the oracle."""
     vocab, k = 151936, 50
     lg = torch.empty(rows, vocab, dtype=torch.bfloat16, device="cuda")
     g = torch.empty(rows, k, dtype=torch.float32, device="cuda")
@@ -305,12 +309,21 @@ def test_topk_sample_ties_across_cta_boundaries(kernel, dtype):
         assert list(tok) == [9490, 9446, 18980, 151900]  # greedy: the first index of the maximum
 
 
-def test_topk_sample_dispatch_by_rows():
-    """A call of one row takes the cluster kernel (the workspace stays as it
-    was); one of 64 rows, more than a B200 holds clusters of 16 CTAs at once,
-    takes the slice kernel (its candidates land in the workspace)."""
+@pytest.mark.parametrize("mode,touched", [(1, False), (2, False), (0, True)])
+def test_topk_sample_workspace_use_by_kernel(mode, touched):
+    """The cluster kernels (one row: registers; 64 rows, more than a B200 holds
+    clusters of 16 CTAs at once: shared memory) leave the workspace as it was;
+    the slice kernel's candidates land in it."""
     vocab, k = 151936, 50
-    for rows, touched in ((1, False), (64, True)):
+    old = ops.set_topk_cluster(mode)
+    try:
+        _workspace_use(vocab, k, touched)
+    finally:
+        ops.set_topk_cluster(old)
+
+
+def _workspace_use(vocab, k, touched):
+    for rows in (1, 64):
         n = ops.topk_sample_workspace(rows, vocab, k)
         w8 = torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
         w8[:COUNTER_BYTES] = 0

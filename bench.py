@@ -303,6 +303,39 @@ ISOLATED = (("rmsnorm", "rmsnorm"), ("add_rmsnorm", "add_rmsnorm"), ("swiglu", "
             ("mrope_qk", "mrope_qk"), ("decode5", "decode_b5"), ("decode256", "decode_b256"))
 
 
+def _time_alone(op: str, rows, device, peak: float, peak_kind: str, launches: int) -> dict:
+    """One operator on its own (see isolated_ops)."""
+    import swiglu_ar_tts_b200 as ops
+    from swiglu_ar_tts_b200 import opbench
+
+    fns, nbytes, desc = opbench.make_rotation(op, rows, device, None)
+    ops.set_pdl(False)
+    us = opbench.time_op(fns, launches)
+    ops.set_pdl(True)
+    for f in fns:
+        f()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(1e7))
+    e0.record()
+    for i in range(launches):
+        fns[i % len(fns)]()
+    e1.record()
+    torch.cuda.synchronize()
+    b2b = 1e3 * e0.elapsed_time(e1) / launches
+    med = statistics.median(us)
+    gbs = nbytes / (med * 1e-6) / 1e9
+    gbs_b2b = nbytes / (b2b * 1e-6) / 1e9
+    del fns
+    torch.cuda.empty_cache()
+    return {"shape": desc, "bytes": nbytes, "launches": launches,
+            "us_median": round(med, 3), "us_min": round(min(us), 3),
+            "gbs_median": round(gbs, 1),
+            "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
+            "us_back_to_back": round(b2b, 3), "gbs_back_to_back": round(gbs_b2b, 1),
+            "frac_back_to_back": round(gbs_b2b / peak, 4)}
+
+
 def isolated_ops(device, peak: float, peak_kind: str, launches: int = 100) -> dict:
     """Each operator on its own, outside the timed steps: enough copies of its
     buffers to cover 512 MB (4x L2; a decode step at batch 256 is 588 MB in one
@@ -314,38 +347,28 @@ def isolated_ops(device, peak: float, peak_kind: str, launches: int = 100) -> di
     programmatic dependent launch between one pair of events, per launch (each
     launch overlaps its predecessor's drain, as inside a step)."""
     import swiglu_ar_tts_b200 as ops
-    from swiglu_ar_tts_b200 import opbench
 
     out = {}
     old = ops.set_pdl(False)
     try:
         for op, key in ISOLATED:
-            fns, nbytes, desc = opbench.make_rotation(op, None, device, None)
-            ops.set_pdl(False)
-            us = opbench.time_op(fns, launches)
-            ops.set_pdl(True)
-            for f in fns:
-                f()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize()
-            torch.cuda._sleep(int(1e7))
-            e0.record()
-            for i in range(launches):
-                fns[i % len(fns)]()
-            e1.record()
-            torch.cuda.synchronize()
-            b2b = 1e3 * e0.elapsed_time(e1) / launches
-            med = statistics.median(us)
-            gbs = nbytes / (med * 1e-6) / 1e9
-            gbs_b2b = nbytes / (b2b * 1e-6) / 1e9
-            out[key] = {"shape": desc, "bytes": nbytes, "launches": launches,
-                        "us_median": round(med, 3), "us_min": round(min(us), 3),
-                        "gbs_median": round(gbs, 1),
-                        "frac_of_" + peak_kind + "_hbm": round(gbs / peak, 4),
-                        "us_back_to_back": round(b2b, 3), "gbs_back_to_back": round(gbs_b2b, 1),
-                        "frac_back_to_back": round(gbs_b2b / peak, 4)}
-            del fns
-            torch.cuda.empty_cache()
+            out[key] = _time_alone(op, None, device, peak, peak_kind, launches)
+    finally:
+        ops.set_pdl(old)
+    return out
+
+
+def sampling_ops(device, peak: float, peak_kind: str, launches: int = 100) -> dict:
+    """The fused softmax + top-k sampler (top 50 of 151,936 bf16 logits a row)
+    timed the same way, at the decode step's two batch sizes: 5 candidates
+    (the register cluster kernel) and 256 rows (the shared-memory one)."""
+    import swiglu_ar_tts_b200 as ops
+
+    out = {}
+    old = ops.set_pdl(False)
+    try:
+        for rows in (5, 256):
+            out[f"rows{rows}"] = _time_alone("topk_sample", rows, device, peak, peak_kind, launches)
     finally:
         ops.set_pdl(old)
     return out
@@ -575,6 +598,7 @@ def main() -> None:
                             "rows_per_s": round(step.rows[name] / (us * 1e-6)),
                             "us_marginal": round(marg[name], 3)}
     iso = isolated_ops(device, peak, peak_kind)
+    sampling = sampling_ops(device, peak, peak_kind)
     # time per kernel type in the step: prefill operators are one launch each;
     # each decode step is split across its operators' kernels (decode_split)
     kernels: dict[str, dict] = {}
@@ -746,6 +770,7 @@ def main() -> None:
                                "batch256": ops_report["decode_b256"]["us"]},
         "ops": ops_report,
         "ops_isolated": iso,
+        "sampling": sampling,
         "roofline": roofline,
         "roofline_swiglu": roofline_swiglu,
         "kernels": kernels,

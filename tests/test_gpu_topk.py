@@ -334,3 +334,42 @@ def _workspace_use(vocab, k, touched):
         assert not w8[:COUNTER_BYTES].any()
         t_ref, _ = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 1.0)
         assert np.array_equal(tok.cpu().numpy(), t_ref)
+
+
+_FIRST_CALL_CAPTURED = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+import oracle, swiglu_ar_tts_b200 as ops
+from swiglu_ar_tts_b200 import inputs
+rows, vocab, k = {rows}, 151936, 50
+inp = inputs.topk_inputs(rows, vocab, k, "bf16", seed=rows)
+lg, g = inp["logits"].cuda(), inp["gumbel"].cuda()
+tok = torch.empty(rows, dtype=torch.int32, device="cuda")
+prob = torch.empty(rows, dtype=torch.float32, device="cuda")
+ws = ops.topk_sample_prepare(torch.empty(ops.topk_sample_workspace(rows, vocab, k), dtype=torch.uint8, device="cuda"))
+torch.cuda.synchronize()
+graph = torch.cuda.CUDAGraph()
+with torch.cuda.graph(graph):  # the process's first sampling call
+    ops.topk_sample(lg, g, k, 0.9, workspace=ws, token_out=tok, prob_out=prob)
+graph.replay()
+torch.cuda.synchronize()
+t_ref, _ = oracle.get().topk_sample(inp["logits"], inp["gumbel"], k, 0.9)
+assert np.array_equal(tok.cpu().numpy(), t_ref)
+print("ok")
+"""
+
+
+@pytest.mark.parametrize("rows", [5, 40])
+def test_topk_sample_first_call_inside_a_graph_capture(rows):
+    """A fresh process whose first sampling call is made while a CUDA graph is
+    being captured (the one-time occupancy lookup and kernel attributes of the
+    cluster kernels run inside the capture): register kernel (5 rows) and
+    shared-memory kernel (40 rows)."""
+    import os
+    import subprocess
+    import sys
+
+    tests = os.path.dirname(os.path.abspath(__file__))
+    code = _FIRST_CALL_CAPTURED.format(root=os.path.dirname(tests), tests=tests, rows=rows)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stderr[-2000:]

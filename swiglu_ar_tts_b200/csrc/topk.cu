@@ -1626,8 +1626,8 @@ cudaError_t launch_cluster_m(const T* logits, const float* gumbel, int32_t* toke
 // Shape of the many-row launch: the fewest CTAs per cluster (a power of two
 // up to 8, the portable size) whose chunks hold at most ~76 KB of logits and
 // 65,528 positions (16-bit local positions, multiples of 8 logits), so that
-// two CTAs share an SM and many rows' clusters are resident at once.  ncta = 0
-// when no such shape exists.
+// two CTAs share an SM and many rows' clusters are resident at once; more
+// CTAs when there are few rows.  ncta = 0 when no such shape exists.
 struct SmemShape {
     int ncta;
     int chunk;
@@ -1638,11 +1638,17 @@ constexpr size_t kSmemChunkTarget = 76 * 1024;
 constexpr int kSmemMaxChunk = 65528;
 constexpr size_t kSmemMaxBytes = 144 * 1024;  // fp32 rows of 262,144 logits over 8 CTAs
 
-SmemShape smem_shape(int64_t vocab, size_t esize)
+SmemShape smem_shape(int64_t vocab, size_t esize, int64_t rows, int sm_count)
 {
     int ncta = 1;
     while (ncta < 8 && ((size_t)ceil_div(vocab, ncta) * esize > kSmemChunkTarget ||
                         ceil_div(vocab, ncta) > kSmemMaxChunk))
+        ncta *= 2;
+    // Few rows: twice the CTAs on half the chunk while the rows' CTAs would
+    // fill at most half the SMs (8 rows of 151,936 bf16 logits: 10.9 against
+    // 13.0 us back to back on B200 with 8 CTAs instead of 4; equal at 16
+    // rows, slower at 32).
+    while (ncta < 8 && rows * ncta * 2 <= sm_count && ceil_div(vocab, 2 * ncta) >= 4096)
         ncta *= 2;
     const int64_t chunk = (int64_t)round_up((uint32_t)ceil_div(vocab, ncta), 8u);
     if (chunk > kSmemMaxChunk || (size_t)chunk * esize + kCompactKeys * 8 > kSmemMaxBytes)
@@ -1658,7 +1664,10 @@ cudaError_t launch_cluster_smem(const T* logits, const float* gumbel, int32_t* t
 {
     constexpr auto kernel = topk_cluster_smem_kernel<T, VEC>;
     *launched = false;
-    const SmemShape ss = smem_shape(vocab, sizeof(T));
+    DeviceInfo di;
+    if (current_device_info(&di) != cudaSuccess)
+        return cudaSuccess;
+    const SmemShape ss = smem_shape(vocab, sizeof(T), rows, di.sm_count);
     if (ss.ncta == 0 || cluster_capacity<kernel>(ss.ncta, kSmemMaxBytes) < 1)
         return cudaSuccess;
     if (set_cluster_attrs<kernel>(8, kSmemMaxBytes, false) != cudaSuccess)

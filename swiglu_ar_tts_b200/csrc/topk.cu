@@ -8,11 +8,13 @@
 // rank): Gumbel-max sampling from softmax(logits / T) restricted to the top k.
 // prob_out is that token's probability under the same restricted softmax.
 //
-// Two kernels give the same results.  The cluster kernel (second half of this
-// file) runs a row per thread-block cluster with the selection exchanged
-// through distributed shared memory; it is taken while every row's cluster is
-// resident at once (a few rows).  The slice kernel serves every other call:
-// grid (slices, rows).  A CTA turns its 4096-logit slice into
+// Three kernels give the same results.  The cluster kernels (second half of
+// this file) run a row per thread-block cluster with the selection exchanged
+// through distributed shared memory: logits in registers on clusters of up
+// to 16 CTAs while every row's cluster is resident at once (a few rows), in
+// shared memory on clusters of up to 8 for more rows.  The slice kernel serves
+// calls where no cluster launch is possible: grid (slices, rows).  A CTA turns
+// its 4096-logit slice into
 // keys (order-preserving bits of the value, then the inverted position, so
 // that larger keys are larger logits and, among equal logits, lower indices:
 // every key is distinct; 32 bits for bf16, 48 for fp32), finds its k largest
@@ -591,15 +593,15 @@ topk_sample_kernel(const T* __restrict__ logits, int64_t vocab, int k, int slice
 }
 
 // ---------------------------------------------------------------------------
-// Single-pass variant on a thread-block cluster: one cluster of `ncta` CTAs
-// (up to 16) per row, each CTA holding a contiguous chunk of the row's logits
-// in registers.  The select runs over the whole row at once: every CTA first
-// drops the keys below a floor that at least k of its keys reach (so none of
-// the dropped ones can be among the row's k largest), histograms the rest in
-// its shared memory, the cluster barrier publishes
-// the histograms, and every CTA sums the cluster's from its peers' shared
-// memory (distributed shared memory), so all CTAs reach the same decision
-// without any exchange through global memory.  Once the boundary bin holds at
+// Single-pass variants on a thread-block cluster: one cluster of `ncta` CTAs
+// per row, each CTA holding a contiguous chunk of the row's logits, in
+// registers (up to 16 CTAs) or in shared memory (up to 8).  The select runs
+// over the whole row at once: every CTA first drops the keys below a floor
+// that at least k of its keys reach (so none of the dropped ones can be among
+// the row's k largest), histograms the rest in its shared memory and sends
+// the histogram to its peers' shared memory (distributed shared memory)
+// before a cluster barrier, and every CTA sums the cluster's, so all CTAs
+// reach the same decision without any exchange through global memory.  Once the boundary bin holds at
 // most kSmallBin keys, every CTA pushes its keys from that bin up (at most
 // k - 1 + kSmallBin in all, the row's k largest among them) into the shared
 // memory of the cluster's first CTA, which ranks them by counting and takes

@@ -374,3 +374,22 @@ def test_topk_sample_first_call_inside_a_graph_capture(rows):
     code = _FIRST_CALL_CAPTURED.format(root=os.path.dirname(tests), tests=tests, rows=rows)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "ok" in r.stdout, r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("offset", [0, 1])
+def test_topk_sample_ten_rows(dtype, offset):
+    """Ten rows of 151,936 logits, 16-byte-aligned or one element past the
+    boundary: more rows than a B200 holds 16-CTA clusters of the register
+    kernel at once, so the default takes it on 8-CTA clusters (40 logits a
+    thread)."""
+    rows, vocab, k = 10, 151936, 50
+    inp = inputs.topk_inputs(rows, vocab, k, "f32", seed=77 + offset)
+    lg = inp["logits"].to(dtype)
+    flat = torch.empty(rows * vocab + offset, dtype=dtype, device="cuda")
+    view = flat[offset:].view(rows, vocab)
+    view.copy_(dev(lg))
+    tok, prob = ops.topk_sample(view, dev(inp["gumbel"]), k, 0.7)
+    t_ref, p_ref = oracle.get().topk_sample(lg, inp["gumbel"], k, 0.7)
+    assert np.array_equal(tok.cpu().numpy(), t_ref)
+    np.testing.assert_allclose(to_f64(prob), p_ref, rtol=1e-5, atol=0)

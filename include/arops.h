@@ -321,7 +321,9 @@ AROPS_API int arops_set_streaming(int enable);
  * Top-k sampling kernel selection (process-wide): 0 = the slice kernel for
  * every call; 1 (the default) = the cluster kernels as described at
  * arops_topk_sample (registers for few rows, shared memory for many); 2 = the
- * shared-memory cluster kernel for every call.  Other values are clamped.
+ * shared-memory cluster kernel for every call; 3 = the streaming kernel (one
+ * CTA a row, the row streamed once through shared memory) for every call
+ * whose rows are 16-byte aligned, else as 2.  Other values are clamped.
  * Every kernel gives identical results; the control exists for measurement
  * and testing.  Returns the old setting.
  */

@@ -370,7 +370,8 @@ def set_topk_cluster(mode) -> int:
     """Which kernels top-k sampling may take: 0 (or False) the slice kernel
     only; 1 (or True, the default) the cluster kernels, registers for calls
     whose rows' 16-CTA clusters are all resident at once and shared memory for
-    the rest; 2 the shared-memory cluster kernel for every call.  Returns the
+    the rest; 2 the shared-memory cluster kernel for every call; 3 the
+    streaming kernel (one CTA a row) for 16-byte-aligned rows.  Returns the
     old mode.  Every kernel gives identical results."""
     return int(lib().arops_set_topk_cluster(int(mode)))
 

@@ -445,7 +445,7 @@ AROPS_API int arops_set_streaming(int enable)
 
 AROPS_API int arops_set_topk_cluster(int mode)
 {
-    return g_topk_cluster.exchange(mode < 0 ? 0 : (mode > 2 ? 2 : mode));
+    return g_topk_cluster.exchange(mode < 0 ? 0 : (mode > 3 ? 3 : mode));
 }
 
 AROPS_API uint64_t arops_launch_count(void)

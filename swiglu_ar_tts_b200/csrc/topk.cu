@@ -35,6 +35,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace arops {
 // Which kernels sampling calls may take (api.cu, arops_set_topk_cluster): 0
@@ -422,6 +423,42 @@ __device__ __forceinline__ void sample_decision(const uint64_t* ranked, int k,
     }
 }
 
+// The k largest of the block's candidate keys (row keys, cand_key; each
+// thread passes M of them, `valid` marking real ones; at least k valid in
+// all), ordered by counting (rank = number of larger keys), then the sampling
+// decision.  Every thread of the block must call it.
+template <typename T, int M>
+__device__ void rank_and_sample(const uint64_t (&key)[M], const bool (&valid)[M], int k,
+                                const float (&gdraw)[2], float temperature, int32_t* token_out,
+                                float* prob_out, SelectState& st, uint64_t* sel, uint64_t* ranked)
+{
+    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
+    {
+        int count = 0;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            count += valid[m] && selected(key[m], st);
+        int slot = selected_offset(count, reinterpret_cast<int*>(st.warp_top));
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            if (valid[m] && selected(key[m], st)) {
+                if (slot < k)
+                    sel[slot] = key[m];
+                ++slot;
+            }
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < k) {
+        const uint64_t mine = sel[threadIdx.x];
+        int rank = 0;
+        for (int j = 0; j < k; ++j)
+            rank += sel[j] > mine;
+        ranked[rank] = mine;
+    }
+    __syncthreads();
+    sample_decision<T>(ranked, k, gdraw, temperature, token_out, prob_out);
+}
+
 // The row's merge and decision, run by the CTA that arrived last: the k
 // largest of the slices' n = slices * k candidate keys (read through L2: other
 // CTAs wrote them), ranked by counting, then the sampling decision.
@@ -448,33 +485,7 @@ __device__ void merge_and_sample(const uint64_t* cand, int n, int k, const float
         key[m] = (i < n) ? __ldcg(cand + i) : 0ull;
         valid[m] = key[m] != 0ull;
     }
-    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
-    {
-        int count = 0;
-#pragma unroll
-        for (int m = 0; m < kMergePerThread; ++m)
-            count += valid[m] && selected(key[m], st);
-        int slot = selected_offset(count, reinterpret_cast<int*>(st.warp_top));
-#pragma unroll
-        for (int m = 0; m < kMergePerThread; ++m)
-            if (valid[m] && selected(key[m], st)) {
-                if (slot < k)
-                    sel[slot] = key[m];
-                ++slot;
-            }
-    }
-    __syncthreads();
-    // order the k candidates by counting: rank = number of larger keys
-    if ((int)threadIdx.x < k) {
-        const uint64_t mine = sel[threadIdx.x];
-        int rank = 0;
-        for (int j = 0; j < k; ++j)
-            rank += sel[j] > mine;
-        ranked[rank] = mine;
-    }
-    __syncthreads();
-
-    sample_decision<T>(ranked, k, gdraw, temperature, token_out, prob_out);
+    rank_and_sample<T>(key, valid, k, gdraw, temperature, token_out, prob_out, st, sel, ranked);
 }
 
 // VEC: rows start on 16-byte boundaries, so a thread loads its 16 logits as
@@ -1431,6 +1442,480 @@ topk_cluster_smem_kernel(const T* __restrict__ logits, int64_t vocab, int chunk,
                              prob_out);
 }
 
+// ---------------------------------------------------------------------------
+// Streaming variant for many rows: one CTA per row (a persistent grid of one
+// CTA an SM walks the rows), the row streamed once through a ring of
+// shared-memory stages filled by bulk copies (cp.async.bulk, mbarrier
+// completion, every wait bounded).  Instead of a select over the whole row,
+// the CTA keeps a running floor: from the row's first stage, the smallest of
+// the 16 warps' r-th largest lane maxima (r = ceil(k / 16)), below which at
+// least k of the row's keys lie above, so no key under it can be among the k
+// largest.  Each 16-byte vector is tested against the floor's value with a
+// few integer instructions; the rare vector holding a key at or above the
+// floor appends those keys (row keys, as cand_key) to a list in shared memory.
+// A list that would overflow is cut to its k largest (block select), which
+// raises the floor, and the stage is taken again a vector per thread at a
+// time.  At the end of the row the list holds every key that can be among
+// the k largest: the k largest of it are ranked and the decision taken as
+// in the other kernels.  No exchange between CTAs and no global scratch.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 512;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr uint32_t kRowStage = 48 * 1024;                     // bytes a stage
+constexpr int kRowStages = 3;                                 // stages in the ring
+constexpr int kRowVecs = (int)(kRowStage / 16) / kRowThreads;  // vectors a thread a stage
+constexpr int kRowListM = 9;                                  // list keys a thread at the end
+constexpr uint32_t kRowList = kRowListM * kRowThreads;        // list capacity
+constexpr size_t kRowSmem = (size_t)kRowStages * kRowStage + kRowList * sizeof(uint64_t);
+static_assert(kRowWarps * 4 >= kMaxTopK, "at most four lanes a warp make the floor");
+static_assert(kRowWarps % 4 == 0, "the warps' floors are read four at a time");
+static_assert(kRowList >= (uint32_t)kMaxTopK + kRowThreads * 8, "a cut list takes a sub-round");
+
+__device__ __forceinline__ uint32_t max_s16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Per-vector tests of the streaming kernel: the largest order value of a
+// vector (vmax), whether a vector holds a value at or above the floor's
+// (pass), and the order value of element e (ord; as KeyBits<T>::of).  While
+// the floor's value is not negative (the usual case: the k-th largest logit
+// is above zero), pass compares the raw bits as signed integers, which orders
+// non-negative floats by value and puts every negative one below: two bf16 at
+// a time with max.s16x2, three instructions for eight values.
+template <typename T>
+struct RowFilter;
+template <>
+struct RowFilter<__nv_bfloat16> {
+    static constexpr int E = 8;
+    uint32_t below2;  // order test: the floor's order value minus one, in both halves
+    uint32_t sbelow2;  // signed test: the floor's raw bits minus one, in both halves
+    bool all;          // floor order value 0: every vector passes
+    bool pos;          // the floor's value is +0 or above: the signed test applies
+    __device__ __forceinline__ void set(uint64_t floor)
+    {
+        const uint32_t fv = (uint32_t)(floor >> kIndexBits);
+        all = fv == 0u;
+        below2 = (fv - 1u) * 0x00010001u;
+        pos = fv >= 0x8000u;
+        sbelow2 = ((fv - 0x8000u - 1u) & 0xFFFFu) * 0x00010001u;
+    }
+    __device__ __forceinline__ static uint32_t max2(const uint4& x)
+    {
+        return max_u16x2(max_u16x2(ordered_bf16x2(x.x), ordered_bf16x2(x.y)),
+                         max_u16x2(ordered_bf16x2(x.z), ordered_bf16x2(x.w)));
+    }
+    __device__ __forceinline__ static uint32_t vmax(const uint4& x)
+    {
+        const uint32_t m = max2(x);
+        return max(m & 0xFFFFu, m >> 16);
+    }
+    template <bool POS>
+    __device__ __forceinline__ bool pass(const uint4& x) const
+    {
+        if constexpr (POS) {
+            const uint32_t m = max_s16x2(max_s16x2(x.x, x.y), max_s16x2(x.z, x.w));
+            return max_s16x2(m, sbelow2) != sbelow2;
+        } else {
+            return all || max_u16x2(max2(x), below2) != below2;
+        }
+    }
+    __device__ __forceinline__ static uint32_t ord(const uint4& x, int e)
+    {
+        const uint32_t w = e < 2 ? x.x : e < 4 ? x.y : e < 6 ? x.z : x.w;
+        const uint32_t o = ordered_bf16x2(w);
+        return (e & 1) ? (o >> 16) : (o & 0xFFFFu);
+    }
+};
+template <>
+struct RowFilter<float> {
+    static constexpr int E = 4;
+    uint32_t fv;
+    int sfv;  // the floor's raw bits (signed test)
+    bool pos;
+    __device__ __forceinline__ void set(uint64_t floor)
+    {
+        fv = (uint32_t)(floor >> kIndexBits);
+        pos = fv >= 0x80000000u;
+        sfv = (int)(fv & 0x7FFFFFFFu);
+    }
+    __device__ __forceinline__ static uint32_t vmax(const uint4& x)
+    {
+        return max(max(order_bits(__uint_as_float(x.x)), order_bits(__uint_as_float(x.y))),
+                   max(order_bits(__uint_as_float(x.z)), order_bits(__uint_as_float(x.w))));
+    }
+    template <bool POS>
+    __device__ __forceinline__ bool pass(const uint4& x) const
+    {
+        if constexpr (POS)
+            return max(max((int)x.x, (int)x.y), max((int)x.z, (int)x.w)) >= sfv;
+        else
+            return vmax(x) >= fv;
+    }
+    __device__ __forceinline__ static uint32_t ord(const uint4& x, int e)
+    {
+        const uint32_t w = e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w;
+        return order_bits(__uint_as_float(w));
+    }
+};
+
+// Rows start on 16-byte boundaries and hold a whole number of vectors (the
+// bulk copies need both).
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads, 1)
+topk_row_kernel(const T* __restrict__ logits, int64_t rows, int64_t vocab, int k,
+                const float* __restrict__ gumbel, float temperature,
+                int32_t* __restrict__ token_out, float* __restrict__ prob_out, unsigned* err_word)
+{
+    using F = RowFilter<T>;
+    constexpr int E = F::E;
+    constexpr uint32_t kStageVecs = kRowStage / 16;
+    extern __shared__ uint4 topk_row_smem[];  // the ring of stages, then the list
+    __shared__ SelectState st;
+    __shared__ uint64_t sel[kMaxTopK];
+    __shared__ uint64_t ranked[kMaxTopK];
+    __shared__ __align__(8) uint64_t bars[kRowStages];
+    __shared__ uint64_t s_floor;
+    __shared__ uint32_t s_count;   // keys appended to the list (may run past its capacity)
+    __shared__ int s_over;         // an append found the list full
+    __shared__ uint16_t s_vlist[kStageVecs];  // per warp: its vectors at or above the floor
+    __shared__ uint32_t s_wfloor[kRowWarps];
+    __shared__ __align__(16) uint32_t s_wlv[kRowWarps];  // per warp: r-th largest of its lanes' appended values
+
+    const int tid = (int)threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    uint64_t* list = reinterpret_cast<uint64_t*>(topk_row_smem + (size_t)kRowStages * kStageVecs);
+    const uint32_t row_bytes = (uint32_t)vocab * (uint32_t)sizeof(T);
+    const int nst = (int)((row_bytes + kRowStage - 1) / kRowStage);
+    const int64_t my_rows =
+        rows > (int64_t)blockIdx.x ? (rows - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+    const int64_t total = my_rows * nst;  // stages this CTA streams
+
+    if (tid == 0) {
+        for (int s = 0; s < kRowStages; ++s)
+            mbar_init(smem_addr(&bars[s]), 1);
+        mbar_init_fence();
+    }
+    // the first row into L2 while the previous kernel drains, a stage a thread
+    if (my_rows > 0 && tid < nst) {
+        const uint32_t off = (uint32_t)tid * kRowStage;
+        prefetch_l2(reinterpret_cast<const unsigned char*>(logits + (int64_t)blockIdx.x * vocab) + off,
+                    min(kRowStage, row_bytes - off));
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_allow_dependents();
+
+    // The producer (thread 0) walks the same sequence of (row, stage, slot)
+    // as the consumers, counters instead of divisions.
+    int64_t issued = 0;  // stages requested (meaningful in thread 0 only)
+    int64_t prow = blockIdx.x;
+    int pst = 0, pslot = 0;
+    auto issue = [&]() {
+        const uint32_t off = (uint32_t)pst * kRowStage;
+        const uint32_t bytes = min(kRowStage, row_bytes - off);
+        const uint32_t bar = smem_addr(&bars[pslot]);
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(smem_addr(topk_row_smem + (size_t)pslot * kStageVecs),
+                  reinterpret_cast<const unsigned char*>(logits + prow * vocab) + off, bytes, bar);
+        ++issued;
+        if (++pst == nst) {
+            pst = 0;
+            prow += gridDim.x;
+        }
+        if (++pslot == kRowStages)
+            pslot = 0;
+    };
+    if (tid == 0)
+        while (issued < kRowStages && issued < total)
+            issue();
+
+    F filt;
+    uint64_t floor = 0;
+    uint32_t lval = 0;  // largest order value among the keys this lane appended (this row)
+    const int r = (k + kRowWarps - 1) / kRowWarps;
+    float gdraw[2] = {0.f, 0.f};
+    // list length when the stage began, read while no thread appends (after
+    // the previous stage's last barrier, before the next stage's first)
+    uint32_t cnt0 = 0;
+    bool ok = true;
+    int s = 0, buf = 0;
+    uint32_t phase = 0;
+    int64_t row = blockIdx.x;
+    for (int64_t g = 0; g < total; ++g) {
+        ok = ok && mbar_wait(smem_addr(&bars[buf]), phase);
+        if (__syncthreads_or(!ok)) {
+            // a copy did not land in time: record it, let this CTA's copies
+            // still in flight finish (bounded), and give up
+            if (tid == 0) {
+                record_device_error(err_word, kDeviceErrTimeout);
+                uint32_t ph = phase;
+                for (int64_t q = g, b = buf; q < issued; ++q) {
+                    mbar_wait(smem_addr(&bars[b]), ph);
+                    if (++b == kRowStages) {
+                        b = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            return;
+        }
+        // every thread is done with stage g - 1: its slot takes stage g - 1 + stages
+        if (tid == 0 && g >= 1 && issued < total)
+            issue();
+        const uint4* sb = topk_row_smem + (size_t)buf * kStageVecs;
+        const int nvs = (int)(min(kRowStage, row_bytes - (uint32_t)s * kRowStage) / 16);
+        const int64_t jbase = (int64_t)s * kStageVecs;  // row vector index of sb[0]
+
+        if (s == 0) {
+            // a new row: the floor from this stage's values
+            uint32_t mx = 0;
+#pragma unroll
+            for (int i = 0; i < kRowVecs; ++i) {
+                const int j = tid + i * kRowThreads;
+                if (j < nvs)
+                    mx = max(mx, F::vmax(sb[j]));
+            }
+            uint32_t cur = mx, rth = 0;
+            for (int got = 0; got < r;) {
+                const uint32_t w = __reduce_max_sync(0xFFFFFFFFu, cur);
+                rth = w;
+                if (w == 0u)
+                    break;
+                got += __popc(__ballot_sync(0xFFFFFFFFu, cur == w));
+                if (cur == w)
+                    cur = 0;
+            }
+            if (lane == 0) {
+                s_wfloor[warp] = rth;
+                s_wlv[warp] = 0;
+            }
+            lval = 0;
+            if (tid == 0) {
+                s_count = 0;
+                s_over = 0;
+            }
+            if (tid < 32) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    if (tid + 32 * q < k)
+                        gdraw[q] = __ldg(gumbel + row * k + tid + 32 * q);
+            }
+            __syncthreads();
+            uint32_t fv = 0xFFFFFFFFu;
+#pragma unroll
+            for (int w = 0; w < kRowWarps; ++w)
+                fv = min(fv, s_wfloor[w]);
+            floor = (uint64_t)fv << kIndexBits;
+            filt.set(floor);
+            if (tid == 0)
+                s_floor = floor;
+            cnt0 = 0;
+        }
+
+        // The keys at or above the floor of the vectors this warp listed,
+        // entries [q0, q0 + 32) of its list (one a lane; wn listed in all),
+        // appended to the list: one atomic a warp.  Every lane calls it.
+        uint16_t* wlist = s_vlist + warp * (kRowVecs * 32);
+        auto take = [&](uint32_t q0, uint32_t wn) {
+            const uint32_t q = q0 + (uint32_t)lane;
+            const uint32_t fv = (uint32_t)(floor >> kIndexBits);
+            const uint32_t flo = (uint32_t)floor & ((1u << kIndexBits) - 1u);
+            uint32_t o[E], inv0 = 0, mask = 0;
+            if (q < wn) {
+                const int j = wlist[q];
+                const uint4 x = sb[j];
+                inv0 = (1u << kIndexBits) - 1u - (uint32_t)((jbase + j) * E);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    o[e] = F::ord(x, e);
+                    if (o[e] > fv || (o[e] == fv && inv0 - (uint32_t)e >= flo)) {
+                        mask |= 1u << e;
+                        lval = max(lval, o[e]);
+                    }
+                }
+            }
+            const uint32_t n = (uint32_t)__popc(mask);
+            uint32_t incl = n;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d)
+                    incl += v;
+            }
+            const uint32_t tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            if (tot == 0u)
+                return;
+            uint32_t base = 0;
+            if (lane == 0)
+                base = atomicAdd(&s_count, tot);
+            uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 0) + incl - n;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (mask & (1u << e)) {
+                    if (slot < kRowList)
+                        list[slot] = ((uint64_t)o[e] << kIndexBits) | (uint64_t)(inv0 - (uint32_t)e);
+                    else
+                        s_over = 1;
+                    ++slot;
+                }
+        };
+        // Each warp lists its vectors of the stage that hold a value at or
+        // above the floor's (a ballot an iteration, into its own part of
+        // s_vlist), then forms and appends their keys itself, a vector a
+        // lane: no block barrier between the two.
+        uint32_t wn = 0;  // vectors this warp listed
+        auto scan = [&](auto pos) {
+            uint32_t pm = 0;  // this thread's vectors that pass
+#pragma unroll
+            for (int i = 0; i < kRowVecs; ++i) {
+                const int j = tid + i * kRowThreads;
+                if (j < nvs && filt.template pass<decltype(pos)::value>(sb[j]))
+                    pm |= 1u << i;
+            }
+            if (__any_sync(0xFFFFFFFFu, pm != 0u)) {  // rare once the floor has risen
+#pragma unroll
+                for (int i = 0; i < kRowVecs; ++i) {
+                    const bool p = (pm >> i) & 1u;
+                    const uint32_t b = __ballot_sync(0xFFFFFFFFu, p);
+                    if (p)
+                        wlist[wn + __popc(b & ((1u << lane) - 1u))] =
+                            (uint16_t)(tid + i * kRowThreads);
+                    wn += __popc(b);
+                }
+            }
+        };
+        if (filt.pos)
+            scan(std::true_type{});
+        else
+            scan(std::false_type{});
+        __syncwarp();
+        for (uint32_t q0 = 0; q0 < wn; q0 += 32)
+            take(q0, wn);
+        if (wn > 0u) {
+            // A second floor: the r-th largest of the warp's lanes' largest
+            // appended values (each lane's keys are its own, so r of them are
+            // at or above it in every warp, 16 r >= k in all).  It only rises
+            // as the row goes on.
+            uint32_t cur = lval, rth = 0;
+            for (int got = 0; got < r;) {
+                const uint32_t w = __reduce_max_sync(0xFFFFFFFFu, cur);
+                rth = w;
+                if (w == 0u)
+                    break;
+                got += __popc(__ballot_sync(0xFFFFFFFFu, cur == w));
+                if (cur == w)
+                    cur = 0;
+            }
+            if (lane == 0)
+                s_wlv[warp] = rth;
+        }
+        __syncthreads();
+
+        if (s_over) {
+            // The list ran full in this stage: drop the stage's appends, and
+            // take the listed vectors again, 32 a warp at a time, cutting the
+            // list to its k largest (which raises the floor) whenever a round
+            // might not fit.
+            __syncthreads();  // every thread has read s_over
+            if (tid == 0) {
+                s_count = cnt0;
+                s_over = 0;
+            }
+            __syncthreads();
+            for (int i = 0; i < kRowVecs; ++i) {
+                const uint32_t n = s_count;
+                __syncthreads();  // every thread has read it before any appends
+                if (n > kRowList - (uint32_t)(kRowThreads * E)) {
+                    uint64_t key[kRowListM];
+                    bool valid[kRowListM];
+#pragma unroll
+                    for (int m = 0; m < kRowListM; ++m) {
+                        const uint32_t q = (uint32_t)(tid + m * kRowThreads);
+                        valid[m] = q < n;
+                        key[m] = valid[m] ? list[q] : 0ull;
+                    }
+                    select_top_k<KeyBits<T>::V + kIndexBits>(key, valid, k, st);
+                    int c = 0;
+#pragma unroll
+                    for (int m = 0; m < kRowListM; ++m)
+                        c += valid[m] && selected(key[m], st);
+                    int slot = selected_offset(c, reinterpret_cast<int*>(st.warp_top));
+#pragma unroll
+                    for (int m = 0; m < kRowListM; ++m)
+                        if (valid[m] && selected(key[m], st)) {
+                            if (slot < k)
+                                list[slot] = key[m];
+                            ++slot;
+                        }
+                    if (tid == 0) {
+                        const uint64_t t = (st.tau >> st.shift) << st.shift;
+                        s_floor = max(s_floor, t);
+                        s_count = (uint32_t)k;
+                    }
+                    __syncthreads();
+                    floor = s_floor;
+                    filt.set(floor);
+                }
+                if ((uint32_t)(32 * i) < wn)
+                    take((uint32_t)(32 * i), wn);
+                __syncthreads();
+            }
+        }
+        cnt0 = s_count;
+        {
+            // the floor rises to the smallest of the warps' second floors
+            uint32_t fv2 = 0xFFFFFFFFu;
+#pragma unroll
+            for (int w = 0; w < kRowWarps; w += 4) {
+                const uint4 v = *reinterpret_cast<const uint4*>(&s_wlv[w]);
+                fv2 = min(fv2, min(min(v.x, v.y), min(v.z, v.w)));
+            }
+            const uint64_t nf = (uint64_t)fv2 << kIndexBits;
+            if (nf > floor) {
+                floor = nf;
+                filt.set(floor);
+                if (tid == 0)
+                    s_floor = max(s_floor, nf);
+            }
+        }
+
+        if (s == nst - 1) {
+            // the row's last stage: the k largest of the list, ranked, and the decision
+            const uint32_t n = min(s_count, kRowList);
+            auto finish = [&](auto m_tag) {
+                constexpr int M = decltype(m_tag)::value;
+                uint64_t key[M];
+                bool valid[M];
+#pragma unroll
+                for (int m = 0; m < M; ++m) {
+                    const uint32_t q = (uint32_t)(tid + m * kRowThreads);
+                    valid[m] = q < n;
+                    key[m] = valid[m] ? list[q] : 0ull;
+                }
+                rank_and_sample<T>(key, valid, k, gdraw, temperature, token_out + row,
+                                   prob_out + row, st, sel, ranked);
+            };
+            // usually a few hundred keys: two a thread
+            if (n <= 2u * kRowThreads)
+                finish(std::integral_constant<int, 2>{});
+            else
+                finish(std::integral_constant<int, kRowListM>{});
+        }
+        if (++s == nst) {
+            s = 0;
+            row += gridDim.x;
+        }
+        if (++buf == kRowStages) {
+            buf = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
 }  // namespace
 
 int topk_slices(int64_t vocab)
@@ -1709,6 +2194,38 @@ cudaError_t launch_cluster_smem(const T* logits, const float* gumbel, int32_t* t
     return err;
 }
 
+// The streaming kernel on a persistent grid of one CTA an SM (its shared
+// memory holds one); rows must be 16-byte aligned whole vectors.
+template <typename T>
+cudaError_t launch_row(const T* logits, const float* gumbel, int32_t* token_out, float* prob_out,
+                       int64_t rows, int64_t vocab, int k, float temperature, cudaStream_t stream,
+                       bool* launched)
+{
+    constexpr auto kernel = topk_row_kernel<T>;
+    *launched = false;
+    DeviceInfo di;
+    if (current_device_info(&di) != cudaSuccess)
+        return cudaSuccess;
+    unsigned* word = nullptr;
+    if (device_error_word(&word) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return cudaSuccess;
+    }
+    if (set_cluster_attrs<kernel>(1, kRowSmem, false) != cudaSuccess)
+        return cudaSuccess;
+    const unsigned grid = (unsigned)std::min<int64_t>(rows, di.sm_count);
+    *launched = true;
+    cudaError_t err = launch(kernel, dim3(grid), dim3(kRowThreads), kRowSmem, stream, logits, rows,
+                             vocab, k, gumbel, temperature, token_out, prob_out, word);
+    if (err != cudaSuccess) {  // attributes of another context
+        (void)cudaGetLastError();
+        if (set_cluster_attrs<kernel>(1, kRowSmem, true) == cudaSuccess)
+            err = launch(kernel, dim3(grid), dim3(kRowThreads), kRowSmem, stream, logits, rows,
+                         vocab, k, gumbel, temperature, token_out, prob_out, word);
+    }
+    return err;
+}
+
 }  // namespace
 
 cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t* token_out,
@@ -1719,6 +2236,26 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
     const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
     const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
     const int mode = topk_cluster_mode();
+    // Many rows (more than half as many as SMs): the streaming kernel, one CTA
+    // a row.  151,936 bf16 logits on B200, back to back: 128 rows 21 against
+    // 34 us on the shared-memory cluster kernel, 256 rows 42 against 64 us;
+    // at 64 rows the cluster kernel is faster (18 against 21 us).
+    bool many = false;
+    if (mode == 1 && vec) {
+        DeviceInfo di;
+        many = current_device_info(&di) == cudaSuccess && rows * 2 > di.sm_count;
+    }
+    if ((mode == 3 || many) && vec) {
+        bool launched = false;
+        cudaError_t err =
+            dtype == AROPS_BF16
+                ? launch_row(static_cast<const __nv_bfloat16*>(logits), gumbel, token_out,
+                             prob_out, rows, vocab, k, temperature, stream, &launched)
+                : launch_row(static_cast<const float*>(logits), gumbel, token_out, prob_out,
+                             rows, vocab, k, temperature, stream, &launched);
+        if (launched)
+            return err;
+    }
     if (mode != 0) {
         bool launched = false;
         cudaError_t err = cudaSuccess;

@@ -179,7 +179,7 @@ def main() -> None:
                     help="shared-memory streaming kernels instead of the default register kernels")
     ap.add_argument("--no-chain-pdl", action="store_true",
                     help="decode steps without programmatic dependent launch")
-    ap.add_argument("--topk-mode", type=int, default=1, choices=(0, 1, 2),
+    ap.add_argument("--topk-mode", type=int, default=1, choices=(0, 1, 2, 3),
                     help="top-k kernels: 0 slice, 1 cluster (default), 2 shared-memory cluster")
     ap.add_argument("--json", action="store_true")
     a = ap.parse_args()

@@ -1,7 +1,8 @@
 """Fused softmax + top-k sampling on the GPU against the oracle: the sampled
 token bit for bit (the decision is taken in fp32 on both sides), its
-probability within the fp32 bound.  Both kernels are run: the single-pass
-cluster kernel (the default) and the slice kernel."""
+probability within the fp32 bound.  Every kernel is run: the cluster kernels
+(registers or shared memory), the streaming kernel (one CTA a row) and the
+slice kernel."""
 import numpy as np
 import pytest
 import torch
@@ -15,10 +16,10 @@ from tolerance import to_f64
 pytestmark = pytest.mark.gpu
 
 
-MODES = {"slice": 0, "cluster": 1, "smem": 2}  # arops_set_topk_cluster
+MODES = {"slice": 0, "cluster": 1, "smem": 2, "row": 3}  # arops_set_topk_cluster
 
 
-@pytest.fixture(params=["cluster", "smem", "slice"])
+@pytest.fixture(params=["cluster", "smem", "row", "slice"])
 def kernel(request):
     old = ops.set_topk_cluster(MODES[request.param])
     yield request.param
@@ -223,13 +224,13 @@ def test_topk_sample_cluster_kernel_leaves_the_workspace_alone():
 
 @pytest.mark.parametrize("rows", [1, 7, 12, 64, 300])
 def test_topk_sample_kernels_agree_bit_for_bit(rows):
-    """The three kernels give the same tokens and the same probabilities, bit
+    """The four kernels give the same tokens and the same probabilities, bit
     for bit, over many rows (mode 1 at 12 rows of 151,936: the register kernel
-    on 8-CTA clusters)."""
+    on 8-CTA clusters; mode 3 at 300 rows: two rows and more a CTA)."""
     inp = inputs.topk_inputs(rows, 151936, 50, "bf16", seed=rows)
     lg, g = dev(inp["logits"]), dev(inp["gumbel"])
     out = {}
-    for mode in (1, 2, 0):
+    for mode in (1, 2, 3, 0):
         old = ops.set_topk_cluster(mode)
         try:
             tok, prob = ops.topk_sample(lg, g, 50, 0.8)
@@ -237,17 +238,18 @@ def test_topk_sample_kernels_agree_bit_for_bit(rows):
         finally:
             ops.set_topk_cluster(old)
         out[mode] = (tok.cpu(), prob.cpu())
-    for mode in (1, 2):
+    for mode in (1, 2, 3):
         assert torch.equal(out[mode][0], out[0][0]), mode
         assert torch.equal(out[mode][1], out[0][1]), mode
 
 
-@pytest.mark.parametrize("rows", [5, 20])
+@pytest.mark.parametrize("rows", [5, 20, 100])
 def test_topk_sample_in_a_graph_with_pdl(rows):
     """Sampling captured in a CUDA graph behind another kernel, with
     programmatic dependent launch (the end of a decode step): the register
-    cluster kernel (5 rows) and the shared-memory one (20 rows) replayed on
-    new logits and draws each time, every replay against the oracle."""
+    cluster kernel (5 rows), the shared-memory one (20 rows) and the streaming
+    one (100 rows) replayed on new logits and draws each time, every replay
+    against the oracle."""
     vocab, k = 151936, 50
     lg = torch.empty(rows, vocab, dtype=torch.bfloat16, device="cuda")
     g = torch.empty(rows, k, dtype=torch.float32, device="cuda")
@@ -310,7 +312,7 @@ def test_topk_sample_ties_across_cta_boundaries(kernel, dtype):
         assert list(tok) == [9490, 9446, 18980, 151900]  # greedy: the first index of the maximum
 
 
-@pytest.mark.parametrize("mode,touched", [(1, False), (2, False), (0, True)])
+@pytest.mark.parametrize("mode,touched", [(1, False), (2, False), (3, False), (0, True)])
 def test_topk_sample_workspace_use_by_kernel(mode, touched):
     """The cluster kernels (one row: registers; 64 rows, more than a B200 holds
     clusters of 16 CTAs at once: shared memory) leave the workspace as it was;
@@ -360,12 +362,12 @@ print("ok")
 """
 
 
-@pytest.mark.parametrize("rows", [5, 40])
+@pytest.mark.parametrize("rows", [5, 40, 100])
 def test_topk_sample_first_call_inside_a_graph_capture(rows):
     """A fresh process whose first sampling call is made while a CUDA graph is
     being captured (the one-time occupancy lookup and kernel attributes of the
-    cluster kernels run inside the capture): register kernel (5 rows) and
-    shared-memory kernel (40 rows)."""
+    cluster kernels run inside the capture): register kernel (5 rows),
+    shared-memory kernel (40 rows) and streaming kernel (100 rows)."""
     import os
     import subprocess
     import sys
@@ -393,3 +395,37 @@ def test_topk_sample_ten_rows(dtype, offset):
     t_ref, p_ref = oracle.get().topk_sample(lg, inp["gumbel"], k, 0.7)
     assert np.array_equal(tok.cpu().numpy(), t_ref)
     np.testing.assert_allclose(to_f64(prob), p_ref, rtol=1e-5, atol=0)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rows", [4, 160])
+def test_topk_sample_streaming_list_overflow(dtype, rows):
+    """The streaming kernel's candidate list running full, against the oracle:
+    ascending rows (every stage beats the ones before it), a first stage far
+    below the rest (its floor lets all of the next stage through), constant
+    rows (every key ties), and coarse values with long runs of ties; 4 rows,
+    and 160 (more rows than SMs: CTAs that walk two rows)."""
+    rng = np.random.default_rng(31 + rows)
+    v, k = 151936, 50
+    lg = np.empty((rows, v))
+    for r in range(rows):
+        kind = r % 4
+        if kind == 0:
+            lg[r] = np.linspace(-4.0, 4.0, v) + r * 1e-3
+        elif kind == 1:
+            lg[r] = rng.standard_normal(v)
+            lg[r, :16384] = -30.0 + rng.standard_normal(16384) * 0.01
+        elif kind == 2:
+            lg[r] = 0.5 + r
+        else:
+            lg[r] = np.round(rng.standard_normal(v) * 2) / 2
+    inp = {"logits": torch.from_numpy(lg).float().to(dtype),
+           "gumbel": torch.from_numpy(rng.gumbel(size=(rows, k)).astype(np.float32))}
+    old = ops.set_topk_cluster(3)
+    try:
+        _check(inp, k, 1.0, f"list overflow {dtype} rows={rows}")
+        tok, _ = _run({"logits": inp["logits"], "gumbel": torch.zeros(rows, k)}, k, 1.0)
+        assert np.array_equal(tok, np.argmax(inp["logits"].float().numpy(), axis=1))
+        assert ops.device_errors(clear=True) == 0
+    finally:
+        ops.set_topk_cluster(old)

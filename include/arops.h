@@ -219,11 +219,18 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  * the device at once (a few rows: 7 of 151936 logits on a B200) holds the
  * logits in registers; larger calls use clusters of up to 8 CTAs holding
  * chunks of up to ~76 KB of logits in shared memory, many rows at once.
- * Where neither can run (or arops_set_topk_cluster(0)) it is the slice
+ * Calls with more rows than half the device's SMs whose rows start on
+ * 16-byte boundaries and hold whole 16-byte vectors take the streaming
+ * kernel instead: one CTA a row (a grid of at most one CTA an SM walking the
+ * rows), the row read once through shared memory by bulk copies against a
+ * running floor, no workspace byte touched either.
+ * Where none can run (or arops_set_topk_cluster(0)) it is the slice
  * kernel: each 4096-logit slice's CTA writes its top_k candidates to the
  * workspace, and the last CTA of a row to finish (counted on the row's
  * arrival counter) merges them and takes the decision; no CTA waits for
- * another.  All three give identical results.  A counter found non-zero at the start of a slice-kernel call (a
+ * another.  All four give identical results.  A bulk copy of the streaming
+ * kernel that does not land within a second sets AROPS_DEVICE_ERR_TIMEOUT
+ * (bit 1 of the device error word) and its CTA abandons its rows.  A counter found non-zero at the start of a slice-kernel call (a
  * workspace that was not cleared) sets AROPS_DEVICE_ERR_WORKSPACE in the
  * device error word, and that row's outputs are then undefined.
  */

@@ -1716,43 +1716,28 @@ topk_row_kernel(const T* __restrict__ logits, int64_t rows, int64_t vocab, int k
             cnt0 = 0;
         }
 
-        // The keys at or above the floor of the vectors this warp listed,
-        // entries [q0, q0 + 32) of its list (one a lane; wn listed in all),
-        // appended to the list: one atomic a warp.  Every lane calls it.
+        // The keys at or above the floor of entry q of this warp's list,
+        // appended to the list (one atomic a vector; a handful of vectors a
+        // warp and stage once the floor has risen).
         uint16_t* wlist = s_vlist + warp * (kRowVecs * 32);
-        auto take = [&](uint32_t q0, uint32_t wn) {
-            const uint32_t q = q0 + (uint32_t)lane;
+        auto take = [&](uint32_t q) {
             const uint32_t fv = (uint32_t)(floor >> kIndexBits);
             const uint32_t flo = (uint32_t)floor & ((1u << kIndexBits) - 1u);
-            uint32_t o[E], inv0 = 0, mask = 0;
-            if (q < wn) {
-                const int j = wlist[q];
-                const uint4 x = sb[j];
-                inv0 = (1u << kIndexBits) - 1u - (uint32_t)((jbase + j) * E);
+            const int j = wlist[q];
+            const uint4 x = sb[j];
+            const uint32_t inv0 = (1u << kIndexBits) - 1u - (uint32_t)((jbase + j) * E);
+            uint32_t o[E], mask = 0;
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    o[e] = F::ord(x, e);
-                    if (o[e] > fv || (o[e] == fv && inv0 - (uint32_t)e >= flo)) {
-                        mask |= 1u << e;
-                        lval = max(lval, o[e]);
-                    }
+            for (int e = 0; e < E; ++e) {
+                o[e] = F::ord(x, e);
+                if (o[e] > fv || (o[e] == fv && inv0 - (uint32_t)e >= flo)) {
+                    mask |= 1u << e;
+                    lval = max(lval, o[e]);
                 }
             }
-            const uint32_t n = (uint32_t)__popc(mask);
-            uint32_t incl = n;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-                if (lane >= d)
-                    incl += v;
-            }
-            const uint32_t tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
-            if (tot == 0u)
+            if (mask == 0u)
                 return;
-            uint32_t base = 0;
-            if (lane == 0)
-                base = atomicAdd(&s_count, tot);
-            uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 0) + incl - n;
+            uint32_t slot = atomicAdd(&s_count, (uint32_t)__popc(mask));
 #pragma unroll
             for (int e = 0; e < E; ++e)
                 if (mask & (1u << e)) {
@@ -1769,13 +1754,18 @@ topk_row_kernel(const T* __restrict__ logits, int64_t rows, int64_t vocab, int k
         // lane: no block barrier between the two.
         uint32_t wn = 0;  // vectors this warp listed
         auto scan = [&](auto pos) {
+            // all of the thread's loads first (a full stage needs no bounds
+            // test; the last one of a row reads stale but in-bounds slots
+            // past its end, which the mask drops)
+            uint4 v[kRowVecs];
+#pragma unroll
+            for (int i = 0; i < kRowVecs; ++i)
+                v[i] = sb[tid + i * kRowThreads];
             uint32_t pm = 0;  // this thread's vectors that pass
 #pragma unroll
-            for (int i = 0; i < kRowVecs; ++i) {
-                const int j = tid + i * kRowThreads;
-                if (j < nvs && filt.template pass<decltype(pos)::value>(sb[j]))
+            for (int i = 0; i < kRowVecs; ++i)
+                if (filt.template pass<decltype(pos)::value>(v[i]) && tid + i * kRowThreads < nvs)
                     pm |= 1u << i;
-            }
             if (__any_sync(0xFFFFFFFFu, pm != 0u)) {  // rare once the floor has risen
 #pragma unroll
                 for (int i = 0; i < kRowVecs; ++i) {
@@ -1793,13 +1783,14 @@ topk_row_kernel(const T* __restrict__ logits, int64_t rows, int64_t vocab, int k
         else
             scan(std::false_type{});
         __syncwarp();
-        for (uint32_t q0 = 0; q0 < wn; q0 += 32)
-            take(q0, wn);
-        if (wn > 0u) {
+        for (uint32_t q = (uint32_t)lane; q < wn; q += 32)
+            take(q);
+        if (wn > 0u && s_wlv[warp] <= (uint32_t)(floor >> kIndexBits)) {
             // A second floor: the r-th largest of the warp's lanes' largest
             // appended values (each lane's keys are its own, so r of them are
             // at or above it in every warp, 16 r >= k in all).  It only rises
-            // as the row goes on.
+            // as the row goes on.  Only a warp whose value holds the floor
+            // down updates it (the others' stay valid, if lower).
             uint32_t cur = lval, rth = 0;
             for (int got = 0; got < r;) {
                 const uint32_t w = __reduce_max_sync(0xFFFFFFFFu, cur);
@@ -1860,8 +1851,8 @@ topk_row_kernel(const T* __restrict__ logits, int64_t rows, int64_t vocab, int k
                     floor = s_floor;
                     filt.set(floor);
                 }
-                if ((uint32_t)(32 * i) < wn)
-                    take((uint32_t)(32 * i), wn);
+                if ((uint32_t)(32 * i + lane) < wn)
+                    take((uint32_t)(32 * i + lane));
                 __syncthreads();
             }
         }

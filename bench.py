@@ -316,7 +316,9 @@ def _time_alone(op: str, rows, device, peak: float, peak_kind: str, launches: in
         f()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    torch.cuda._sleep(int(1e7))
+    # a head start long enough for the host to queue every launch before the
+    # first one runs (~50 ms), so that the figure is the device's alone
+    torch.cuda._sleep(int(1e8))
     e0.record()
     for i in range(launches):
         fns[i % len(fns)]()

@@ -141,7 +141,7 @@ def time_op(fns, iters: int) -> list[float]:
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(iters)]
-    torch.cuda._sleep(int(1e7))  # let the host queue ahead of the device
+    torch.cuda._sleep(int(5e7))  # let the host queue ahead of the device
     for i, (a, b) in enumerate(ev):
         a.record()
         fns[i % len(fns)]()
@@ -158,7 +158,7 @@ def time_back_to_back(fns, iters: int) -> float:
         f()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda._sleep(int(1e7))
+    torch.cuda._sleep(int(5e7))
     e0.record()
     for i in range(iters):
         fns[i % len(fns)]()

@@ -8,11 +8,13 @@
 // rank): Gumbel-max sampling from softmax(logits / T) restricted to the top k.
 // prob_out is that token's probability under the same restricted softmax.
 //
-// Three kernels give the same results.  The cluster kernels (second half of
+// Four kernels give the same results.  The cluster kernels (second half of
 // this file) run a row per thread-block cluster with the selection exchanged
 // through distributed shared memory: logits in registers on clusters of up
 // to 16 CTAs while every row's cluster is resident at once (a few rows), in
-// shared memory on clusters of up to 8 for more rows.  The slice kernel serves
+// shared memory on clusters of up to 8 for more rows.  The streaming kernel
+// (after them) runs a row per CTA for calls with many rows, streaming it
+// through shared memory against a running floor.  The slice kernel serves
 // calls where no cluster launch is possible: grid (slices, rows).  A CTA turns
 // its 4096-logit slice into
 // keys (order-preserving bits of the value, then the inverted position, so

@@ -372,7 +372,7 @@ AROPS_API const char* arops_last_error(void);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 AROPS_API int arops_version(void);
 
-#define AROPS_VERSION 20100
+#define AROPS_VERSION 20200
 
 #ifdef __cplusplus
 }

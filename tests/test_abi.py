@@ -38,7 +38,7 @@ def test_header_declares_the_operators():
 def test_every_declared_symbol_is_exported(L):
     for n in _declared_symbols():
         assert hasattr(L, n), n
-    assert L.arops_version() == 20100
+    assert L.arops_version() == 20200
 
 
 def test_status_strings(L):

@@ -47,7 +47,7 @@ def _build_and_run(tmp_path, compiler, flags, suffix):
                     f"-L{LIBDIR}", "-larops", f"-Wl,-rpath,{LIBDIR}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
     lines = dict(line.split(" ", 1) for line in out.strip().splitlines())
-    assert lines["version"] == "20100"
+    assert lines["version"] == "20200"
     assert lines["null"].startswith("1 ")  # AROPS_ERR_INVALID before any launch
     assert lines["reason"].strip()
     assert lines["odd"] == "1"  # odd head_dim

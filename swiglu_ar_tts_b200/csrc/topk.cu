@@ -1463,8 +1463,8 @@ topk_cluster_smem_kernel(const T* __restrict__ logits, int64_t vocab, int chunk,
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 512;
 constexpr int kRowWarps = kRowThreads / 32;
-constexpr uint32_t kRowStage = 48 * 1024;                     // bytes a stage
-constexpr int kRowStages = 3;                                 // stages in the ring
+constexpr uint32_t kRowStage = 80 * 1024;                     // bytes a stage
+constexpr int kRowStages = 2;                                 // stages in the ring
 constexpr int kRowVecs = (int)(kRowStage / 16) / kRowThreads;  // vectors a thread a stage
 constexpr int kRowListM = 9;                                  // list keys a thread at the end
 constexpr uint32_t kRowList = kRowListM * kRowThreads;        // list capacity
@@ -2229,14 +2229,14 @@ cudaError_t launch_topk_sample(const void* logits, const float* gumbel, int32_t*
     const size_t esize = dtype == AROPS_BF16 ? 2 : 4;
     const bool vec = aligned16(logits) && (vocab * esize) % 16 == 0;
     const int mode = topk_cluster_mode();
-    // Many rows (more than half as many as SMs): the streaming kernel, one CTA
-    // a row.  151,936 bf16 logits on B200, back to back: 128 rows 21 against
-    // 34 us on the shared-memory cluster kernel, 256 rows 42 against 64 us;
-    // at 64 rows the cluster kernel is faster (18 against 21 us).
+    // Many rows (more than a quarter as many as SMs): the streaming kernel, one
+    // CTA a row.  151,936 bf16 logits on B200, back to back: 64 rows 16.1
+    // against 18.3 us on the shared-memory cluster kernel, 128 rows 17.7
+    // against 34.3, 256 rows 31.2 against 63.5; at 32 rows 16.0 against 15.1.
     bool many = false;
     if (mode == 1 && vec) {
         DeviceInfo di;
-        many = current_device_info(&di) == cudaSuccess && rows * 2 > di.sm_count;
+        many = current_device_info(&di) == cudaSuccess && rows * 4 > di.sm_count;
     }
     if ((mode == 3 || many) && vec) {
         bool launched = false;

@@ -219,7 +219,7 @@ AROPS_API arops_status arops_swiglu(const void* gate, const void* up, void* out,
  * the device at once (a few rows: 7 of 151936 logits on a B200) holds the
  * logits in registers; larger calls use clusters of up to 8 CTAs holding
  * chunks of up to ~76 KB of logits in shared memory, many rows at once.
- * Calls with more rows than half the device's SMs whose rows start on
+ * Calls with more rows than a quarter of the device's SMs whose rows start on
  * 16-byte boundaries and hold whole 16-byte vectors take the streaming
  * kernel instead: one CTA a row (a grid of at most one CTA an SM walking the
  * rows), the row read once through shared memory by bulk copies against a

@@ -115,3 +115,16 @@ def test_topk_sample_argument_errors(L):
     assert L.arops_topk_sample_prepare(None, 1 << 20, None) == 1
     assert L.arops_topk_sample_prepare(16, (1 << 18) - 1, None) == 1  # smaller than the counters
     assert L.arops_launch_count() == before
+
+
+def test_sampling_kernel_selection_is_clamped(L):
+    """arops_set_topk_cluster takes 0 (slice), 1 (default), 2 (shared-memory
+    cluster) and 3 (streaming), clamps anything else, and returns the old
+    mode; a host setting, so no GPU is needed."""
+    old = ops.set_topk_cluster(1)
+    try:
+        for mode, kept in ((0, 0), (2, 2), (3, 3), (7, 3), (-4, 0), (1, 1)):
+            ops.set_topk_cluster(mode)
+            assert ops.set_topk_cluster(mode) == kept, mode
+    finally:
+        ops.set_topk_cluster(old)

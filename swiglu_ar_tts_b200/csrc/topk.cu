@@ -1449,17 +1449,19 @@ topk_cluster_smem_kernel(const T* __restrict__ logits, int64_t vocab, int chunk,
 // CTA an SM walks the rows), the row streamed once through a ring of
 // shared-memory stages filled by bulk copies (cp.async.bulk, mbarrier
 // completion, every wait bounded).  Instead of a select over the whole row,
-// the CTA keeps a running floor: from the row's first stage, the smallest of
-// the 16 warps' r-th largest lane maxima (r = ceil(k / 16)), below which at
-// least k of the row's keys lie above, so no key under it can be among the k
-// largest.  Each 16-byte vector is tested against the floor's value with a
-// few integer instructions; the rare vector holding a key at or above the
-// floor appends those keys (row keys, as cand_key) to a list in shared memory.
-// A list that would overflow is cut to its k largest (block select), which
-// raises the floor, and the stage is taken again a vector per thread at a
-// time.  At the end of the row the list holds every key that can be among
-// the k largest: the k largest of it are ranked and the decision taken as
-// in the other kernels.  No exchange between CTAs and no global scratch.
+// the CTA keeps a running floor that at least k of the row's keys reach, so
+// that no key under it can be among the k largest: first the smallest of the
+// 16 warps' r-th largest lane maxima of the row's first stage (r = ceil(k /
+// 16)), then, as keys are taken, the smallest of the warps' r-th largest lane
+// values among the keys each lane appended.  Each 16-byte vector is tested
+// against the floor's value with a few integer instructions; each warp lists
+// its rare vectors holding a value at or above it and appends their keys (row
+// keys, as cand_key) to a list in shared memory.  A list that would overflow
+// is cut to its k largest (block select), which raises the floor, and the
+// stage is taken again.  At the end of the row the list holds every key that
+// can be among the k largest: the k largest of it are ranked and the decision
+// taken as in the other kernels.  No exchange between CTAs and no global
+// scratch.
 // ---------------------------------------------------------------------------
 constexpr int kRowThreads = 512;
 constexpr int kRowWarps = kRowThreads / 32;
